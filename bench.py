@@ -1,0 +1,413 @@
+"""Benchmark: quantized GEMV HBM GB/s and decoder-layer us/token on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one step): batch-1 decode of a 36-layer Qwen3-8B-like stack
+(hidden 4096, 32 q heads and 8 kv heads of dim 128, MLP 12288), seven
+projections per layer with per-matrix grids mixed 75.1% ternary / 6.0%
+2-bit / 18.8% 3-bit by parameter count (q at 3 bits, k and v at 2 bits).
+Each layer is ONE grouped launch (tb_layer_gemv) over its seven matrices.
+Weights are seeded N(0, 0.02) draws quantized on the GPU by the library
+(absmax scales, round-half-even), 2.01 GB packed, resident in HBM; the
+working set is 16x the L2, so no L2 flush is needed.  The other hot-path
+rows (scales + pack, unpack, small-batch GEMM) are timed in the same run
+and reported under "rows".
+
+Multi-GPU: the path does not shard (single-GPU method); N ranks run N
+independent replicas, one per GPU, and `value` is the sum of their bytes
+over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from decode_gemv_tb_b200 import build as tbbuild  # noqa: E402
+from decode_gemv_tb_b200 import synth, tb  # noqa: E402
+
+METRIC = "quantized GEMV achieved HBM GB/s (% of B200 peak); decoder-layer µs/token"
+SPEC_HBM_GBS = 8000.0
+
+
+def algo_bytes(N, K, grid, M=1, ybytes=4):
+    """packed codes + bf16 scales + activations + outputs of one product."""
+    bits = 3 if grid == synth.INT3 else 2
+    return N * K * bits // 8 + N * (K // 128) * 2 + M * K * 2 + M * N * ybytes
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi samples during the timed region."""
+
+    def __init__(self, gpu: int):
+        self.gpu = gpu
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait()
+            self.f.close()
+
+    def summary(self):
+        if not self.proc or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload
+
+class DecodeStack:
+    """Packed, resident 36-layer stack with one input and one output per
+    projection; x vectors and y outputs live in single flat buffers so the
+    end-to-end variant moves them with one copy each way per step."""
+
+    def __init__(self, dev, layers=None):
+        self.dev = dev
+        stack = synth.config3_stack()
+        if layers is not None:
+            stack = stack[:layers]
+        self.stack = stack
+        self.layers = []
+        self.bytes_per_layer = []
+        xs, ys = 0, 0
+        for mats in stack:
+            for m in mats:
+                xs += m.K
+                ys += m.N
+        self.x_all = torch.empty(xs, dtype=torch.bfloat16, device=dev)
+        self.y_all = torch.empty(ys, dtype=torch.float32, device=dev)
+        xo, yo = 0, 0
+        self.packed_bytes = 0
+        for li, mats in enumerate(stack):
+            items, b = [], 0
+            for m in mats:
+                W = synth.gaussian_weights(m.N, m.K, seed=m.seed, device=dev, dtype=torch.bfloat16)
+                s = tb.tb_scales_absmax(W, m.grid)
+                p = tb.tb_pack(W, m.grid, s)
+                del W
+                x = self.x_all[xo:xo + m.K]
+                x.copy_(synth.activations(m.K, seed=m.seed, device=dev))
+                y = self.y_all[yo:yo + m.N]
+                xo += m.K
+                yo += m.N
+                items.append((p, m.grid, s, x, y, m.N, m.K))
+                b += algo_bytes(m.N, m.K, m.grid)
+                self.packed_bytes += p.numel()
+            self.layers.append((items, tb.linear_items(items)))
+            self.bytes_per_layer.append(b)
+        torch.cuda.synchronize(dev)
+        self.step_bytes = sum(self.bytes_per_layer)
+
+    def step(self, stream):
+        for _, arr in self.layers:
+            tb.tb_layer_gemv(arr, stream)
+
+
+def time_region(fn, steps, warmup, stream, dist=None):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    return ms
+
+
+def rows_section(dev, stream):
+    """Time the other hot-path rows once each (median of 5 after warm-up)."""
+    out = {}
+
+    def med(fn, reps=5):
+        for _ in range(2):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    # scales + pack of one Qwen3-14B-like layer, outlier weights (config-5 recipe)
+    mats = synth.config5_stack()[0]
+    Ws = [(synth.outlier_weights(m.N, m.K, seed=m.seed, device=dev), m) for m in mats]
+    bufs = []
+    for W, m in Ws:
+        s = torch.empty((m.N, m.K // 128), dtype=torch.bfloat16, device=dev)
+        p = torch.empty(tb.packed_bytes(m.grid, m.N, m.K), dtype=torch.uint8, device=dev)
+        bufs.append((W, m, s, p))
+
+    def pack_layer():
+        for W, m, s, p in bufs:
+            tb.tb_scales_absmax(W, m.grid, s)
+            tb.tb_pack(W, m.grid, s, p)
+
+    ms = med(pack_layer)
+    rw = sum(2 * m.N * m.K * 2 + 2 * m.N * (m.K // 128) * 2 + tb.packed_bytes(m.grid, m.N, m.K) for _, m, _, _ in bufs)
+    out["scales_pack_14b_layer"] = {"ms": ms, "GB_s": rw / ms / 1e6, "weights": sum(m.N * m.K for _, m, _, _ in bufs),
+                                    "bytes_read_written": rw}
+
+    # unpack of the 3-bit q projection
+    W, m, s, p = bufs[0]
+    codes = torch.empty((m.N, m.K), dtype=torch.int8, device=dev)
+    ms = med(lambda: tb.tb_unpack(p, m.grid, m.N, m.K, codes))
+    ub = tb.packed_bytes(m.grid, m.N, m.K) + m.N * m.K
+    out["unpack_q_5120x5120_int3"] = {"ms": ms, "GB_s": ub / ms / 1e6}
+
+    # small-batch GEMM, Qwen3-14B-like gate (17408 x 5120), int2 and int3
+    gate = [(W, m, s, p) for W, m, s, p in bufs if m.name.endswith("gate")][0]
+    W = gate[0]
+    g = {}
+    for grid in (synth.INT2, synth.INT3):
+        s = tb.tb_scales_absmax(W, grid)
+        p = tb.tb_pack(W, grid, s)
+        for M in synth.CONFIG4_M:
+            X = synth.activations(W.shape[1], seed=4000 + M, device=dev, M=M)
+            Y = torch.empty((M, W.shape[0]), dtype=torch.float32, device=dev)
+            ms = med(lambda: tb.tb_gemm(p, grid, s, X, W.shape[0], W.shape[1], Y))
+            fl = 2.0 * M * W.shape[0] * W.shape[1]
+            by = algo_bytes(W.shape[0], W.shape[1], grid, M=M)
+            g[f"{synth.GRID_NAMES[grid]}_M{M}"] = {"us": ms * 1e3, "TFLOP_s": fl / ms / 1e9, "GB_s": by / ms / 1e6}
+    out["gemm_gate_17408x5120"] = g
+    del bufs, Ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline(seconds_budget=20.0):
+    """The oracle as it stands, single-threaded fp64, on a bounded sample of
+    the same workload: GEMV of the stack's layer-0 projections (as many as
+    fit the time budget), GB/s on the same algorithmic bytes."""
+    sys.path.insert(0, ROOT)
+    from oracle import tb_oracle as oracle
+
+    oracle.build()
+    mats = synth.config3_stack()[0]
+    done_bytes, t_total, names = 0, 0.0, []
+    for m in mats:
+        W = synth.gaussian_weights(m.N, m.K, seed=m.seed, dtype=torch.bfloat16)
+        wb = W.view(torch.int16).numpy().view("uint16")
+        s = oracle.scales_absmax(wb, m.grid)
+        p, _ = oracle.pack(wb, m.grid, s)
+        x = synth.activations(m.K, seed=m.seed).view(torch.int16).numpy().view("uint16")
+        t0 = time.perf_counter()
+        oracle.gemv64(p, m.grid, s, x, m.N, m.K)
+        t_total += time.perf_counter() - t0
+        done_bytes += algo_bytes(m.N, m.K, m.grid)
+        names.append(m.name)
+        if t_total > seconds_budget:
+            break
+    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"fp64 oracle GEMV over {'+'.join(names)} of the 36-layer stack "
+                      f"({done_bytes / 1e6:.1f} MB algorithmic), {t_total:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, timed as it stands, per step a bounded
+    sample of the workload (layer-0 k, v projections)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import tb_oracle as oracle
+
+    oracle.build()
+    mats = [m for m in synth.config3_stack()[0] if m.name.endswith((".k", ".v"))]
+    prob = []
+    for m in mats:
+        W = synth.gaussian_weights(m.N, m.K, seed=m.seed, dtype=torch.bfloat16)
+        wb = W.view(torch.int16).numpy().view("uint16")
+        s = oracle.scales_absmax(wb, m.grid)
+        p, _ = oracle.pack(wb, m.grid, s)
+        x = synth.activations(m.K, seed=m.seed).view(torch.int16).numpy().view("uint16")
+        prob.append((p, m, s, x))
+    step_bytes = sum(algo_bytes(m.N, m.K, m.grid) for _, m, _, _ in prob)
+
+    def step():
+        for p, m, s, x in prob:
+            oracle.gemv64(p, m.grid, s, x, m.N, m.K)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = step_bytes * args.steps / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "qwen3_8b_like_decode_stack_36L_mixed_grids (sample: layer-0 k+v GEMV)",
+                       "batch": 1},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": "fp64 single-threaded oracle GEMV of layer-0 k and v (1024x4096, 2-bit) "
+                                       "per step"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=None, help="fewer layers (debug only)")
+    ap.add_argument("--no-rows", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    tbbuild.build()
+    tb.load()
+    stream = torch.cuda.current_stream(dev).cuda_stream
+
+    S = DecodeStack(dev, layers=args.layers)
+    n_layers = len(S.layers)
+    hbm_peak, bf16_peak, bf16_sus, peak_src = measured_peaks()
+
+    # --- device-resident timing (the headline `value`)
+    with Clocks(local) as clk:
+        ms = time_region(lambda: S.step(stream), args.steps, args.warmup, torch.cuda.current_stream(dev), dist)
+    clocks = clk.summary()
+    ms_step = ms / args.steps
+    value = world * S.step_bytes / (ms_step * 1e-3) / 1e9
+    us_layer = ms_step * 1e3 / n_layers
+    launch_us = ms_step * 1e3 / n_layers  # one grouped launch per layer
+    achieved = S.bytes_per_layer[0] / (launch_us * 1e-6) / 1e9
+    avg_layer_bytes = S.step_bytes / n_layers
+    achieved = avg_layer_bytes / (launch_us * 1e-6) / 1e9
+
+    # --- end to end through the public API: H2D of all x, launches, D2H of all y
+    x_host = torch.empty_like(S.x_all, device="cpu").pin_memory()
+    x_host.copy_(S.x_all.cpu())
+    y_host = torch.empty_like(S.y_all, device="cpu").pin_memory()
+
+    def e2e_step():
+        S.x_all.copy_(x_host, non_blocking=True)
+        S.step(stream)
+        y_host.copy_(S.y_all, non_blocking=True)
+
+    ms_e2e = time_region(e2e_step, args.steps, args.warmup, torch.cuda.current_stream(dev), dist)
+    e2e_value = world * S.step_bytes / (ms_e2e / args.steps * 1e-3) / 1e9
+
+    rows = None if args.no_rows else rows_section(dev, torch.cuda.current_stream(dev))
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        profile_traffic = None
+        tp = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(tp):
+            with open(tp) as f:
+                profile_traffic = json.load(f).get("k_linear_layer_bytes_per_launch")
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"qwen3_8b_like_decode_stack_{n_layers}L_mixed_grids", "batch": 1,
+                       "layers": n_layers, "hidden": 4096, "mlp": 12288, "kv_dim": 1024,
+                       "grid_mix": {synth.GRID_NAMES[g]: round(v, 4) for g, v in synth.grid_fractions(S.stack).items()},
+                       "packed_GB": S.packed_bytes / 1e9, "step_algorithmic_bytes": S.step_bytes,
+                       "l2": "working set larger than L2 (no flush)", "parallelism": f"replicas{world}"},
+            "decoder_layer_us_per_token": us_layer,
+            "tokens_per_s_equivalent": 1e6 / (us_layer * n_layers),
+            "frac_of_spec_8TBs": value / world / SPEC_HBM_GBS,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": profile_traffic,
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                         else "fallback 6.65 TB/s", "kernel": "k_linear<1> (tb_layer_gemv)"},
+            "e2e": {"value": e2e_value, "unit": "GB/s",
+                    "h2d_bytes_per_step": S.x_all.numel() * 2, "d2h_bytes_per_step": S.y_all.numel() * 4},
+            "gpu_launches": n_layers * args.steps,
+            "clocks": clocks,
+            "rows": rows,
+        }
+        if cpu:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

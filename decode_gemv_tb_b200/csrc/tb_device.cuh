@@ -1,0 +1,92 @@
+// tb_device.cuh -- device-side pieces shared by the sm_100a kernels:
+// grid constants, the packed layout, bf16 helpers and launch descriptors.
+//
+// Format (declared in include/tb.h): w = c * s, one bf16 scale per 128
+// weights along K, per-layer grid ternary / 2-bit / 3-bit (ThinkBit page
+// "ThinkBit은 2비트 양자화에서 추론 능력 보존을 추론 평가로 검증한다",
+// onedev.kr/papers/1416, section 어떻게 동작하나).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tb {
+
+constexpr int kGroup = 128;      // weights per scale
+constexpr int kMaxItems = 16;    // grouped-launch capacity
+
+enum Grid : int { kTernary = 0, kInt2 = 1, kInt3 = 2 };
+enum DType : int { kF32 = 0, kBF16 = 1 };
+
+__host__ __device__ inline int grid_qmin(int g) { return g == kTernary ? -1 : (g == kInt2 ? -2 : -4); }
+__host__ __device__ inline int grid_qmax(int g) { return g == kInt3 ? 3 : 1; }
+__host__ __device__ inline int grid_offset(int g) { return g == kInt3 ? 4 : 2; }
+// bytes of one packed row of K weights
+__host__ __device__ inline int64_t row_bytes(int g, int64_t K) { return g == kInt3 ? 3 * K / 8 : K / 4; }
+
+// ---- one linear layer inside a launch ------------------------------------
+struct Item {
+    const uint8_t* packed;
+    const uint16_t* scales;
+    const uint16_t* X;   // [M][ldx] bf16
+    void* Y;             // [M][ldy]
+    int64_t N, K, ldx, ldy;
+    int32_t grid, ydt, M;
+    int32_t unit_begin;  // first CTA index of this item
+};
+
+struct Launch {
+    Item it[kMaxItems];
+    int32_t n_items;
+};
+
+// ---- cache-controlled loads ----------------------------------------------
+// Streamed weights: read once, keep them out of L1.
+__device__ __forceinline__ uint2 ld_stream_u2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint16_t ld_stream_u16(const void* p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+// Activations: small, re-read by every CTA: cache in L1.
+__device__ __forceinline__ uint4 ld_act_u4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
+
+// bf16x2 a*b+c, one rounding (exact whenever the true result is a bf16)
+__device__ __forceinline__ uint32_t hfma2_bf16(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// (a & b) | c  in one LOP3
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+// bitwise select: (a & ~m) | (b & m); LOP3 table 0xCA is "x ? y : z"
+__device__ __forceinline__ uint32_t bit_mux(uint32_t a, uint32_t b, uint32_t m) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xCA;" : "=r"(d) : "r"(m), "r"(b), "r"(a));
+    return d;
+}
+
+}  // namespace tb

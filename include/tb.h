@@ -1,0 +1,186 @@
+/*
+ * tb.h -- C interface of libtb_b200: ThinkBit scalar low-bit weights on
+ * NVIDIA B200 (sm_100a).  Quantize/pack, unpack, batch-1 GEMV, small-batch
+ * GEMM (M <= 64) and a grouped launcher for a decoder layer's projections.
+ *
+ * What the method fixes -- ThinkBit page, "ThinkBit은 2비트 양자화에서 추론
+ * 능력 보존을 추론 평가로 검증한다" (onedev.kr/papers/1416):
+ *   section 어떻게 동작하나 ("how it works"): the storage format is strictly
+ *     scalar.  A weight is w = c * s, an integer codeword c times a bf16
+ *     scale s; one scale serves 128 consecutive weights; the codeword grid
+ *     is chosen per layer among ternary {-1,0,1}, 2-bit {-2,-1,0,1} and
+ *     3-bit {-4,...,3}; dequantization is one multiplication (no codebook,
+ *     no rotation, no zero point).
+ *   section 무엇과 다른가 ("what is different"): the per-layer grids are
+ *     mixed within one model (75.3% ternary, 6.0% 2-bit, 18.7% 3-bit on
+ *     Qwen3-1.7B), codewords come out of a rounding step.
+ *   section 무엇인가 ("what it is"): decoding a token reads every weight,
+ *     so decode speed is bound by memory bandwidth.
+ *   section 전제와 한계 ("assumptions and limits"): released checkpoints
+ *     keep the 2- and 3-bit codewords in 4-bit containers because no kernel
+ *     reads them directly; this library is such a reader.
+ *
+ * ------------------------------------------------------------------------
+ * FORMAT (this library's definition; the pages give no bit layout)
+ *
+ *   W is [N][K] row-major: N outputs, K inputs (y = W x), K % 128 == 0.
+ *   Scales: bf16, [N][K/128]; scale (n, j) covers k in [128 j, 128 j + 128).
+ *   Stored code u = c + offset (offset 2 for the 2-bit container, 4 for
+ *   3 bits), so every stored code is an unsigned bit pattern.
+ *
+ *   TB_GRID_TERNARY, TB_GRID_INT2 -- 2 bits per code, 16 codes per uint32:
+ *     row n: K/16 little-endian uint32 words (K/4 bytes); word i holds codes
+ *     k = 16i .. 16i+15; code 16i+2m is at bits [2m, 2m+1] and code
+ *     16i+2m+1 at bits [16+2m, 17+2m], m = 0..7 (even codes in the low
+ *     half-word, odd codes in the high one).  Ternary codes use u in
+ *     {1,2,3}; a stored 0 in a ternary row decodes as -2.
+ *   TB_GRID_INT3 -- 3 bits per code, 32 codes per three uint32 bit-planes:
+ *     row n: K/32 blocks of three uint32 (3K/8 bytes); block j holds codes
+ *     k = 32j .. 32j+31 in planes p = 0, 1, 2 (consecutive words); bit m of
+ *     plane p is bit p of u for code 32j+2m, bit 16+m of plane p is bit p of
+ *     u for code 32j+2m+1, m = 0..15.
+ *   Bytes per weight including the scales: 2.125 / 8 (ternary, 2-bit) and
+ *   3.125 / 8 (3-bit).
+ *
+ * QUANTIZATION RULES (readings where the pages are silent)
+ *   scale  s = bf16_rne(absmax / d), d = |qmin| = 1, 2, 4 for ternary,
+ *          2-bit, 3-bit; absmax over the finite weights of the group; a
+ *          scale that rounds to 0 becomes 1.0, one that rounds to infinity
+ *          becomes the largest finite bf16.
+ *   code   c = clamp(round_half_even(w / s), qmin, qmax), decided exactly
+ *          (the exact quotient, not a rounded one, is rounded).
+ *   NaN w gives code 0, +-Inf gives qmax / qmin, a scale that is not a
+ *   positive finite number gives code 0; every such weight is counted.
+ *
+ * PRODUCTS
+ *   y[n] = sum_k x[k] * c[n][k] * s[n][k/128], accumulated in fp32 per
+ *   128-group and scaled once per group; fp32 output, or bf16 rounded half
+ *   to even from the fp32 result.  Results are bitwise deterministic from
+ *   run to run (no atomics in any reduction).
+ *
+ * ------------------------------------------------------------------------
+ * CONVENTIONS
+ *   - Every pointer argument is DEVICE memory on the current CUDA device
+ *     unless the argument says otherwise.  The caller owns all buffers; the
+ *     library keeps no allocation between calls.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All calls
+ *     are asynchronous on `stream`; none synchronizes.
+ *   - Alignment: packed, W, x / X rows: 16 bytes; scales: 2 bytes; y / Y:
+ *     4 bytes (fp32) or 2 bytes (bf16).
+ *   - Argument errors are reported before anything is launched; a launch
+ *     failure is reported as TB_ERR_CUDA (cudaGetLastError is consumed).
+ *   - Outputs must not overlap inputs.
+ */
+#ifndef TB_B200_H
+#define TB_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TB_API __attribute__((visibility("default")))
+#else
+#define TB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *tb_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    TB_GRID_TERNARY = 0, /* {-1, 0, 1}, 2-bit container, offset 2 */
+    TB_GRID_INT2 = 1,    /* {-2, -1, 0, 1}, offset 2 */
+    TB_GRID_INT3 = 2     /* {-4, ..., 3}, three bit-planes, offset 4 */
+} tb_grid_t;
+
+typedef enum { TB_F32 = 0, TB_BF16 = 1 } tb_dtype_t;
+
+typedef enum {
+    TB_OK = 0,
+    TB_ERR_ARG = 1,         /* null pointer, unknown enum value, bad count */
+    TB_ERR_SHAPE = 2,       /* N < 1, K < 128, K % 128 != 0, M outside 1..64, ld too small */
+    TB_ERR_ALIGN = 3,       /* a pointer or leading dimension breaks the alignment rules */
+    TB_ERR_UNSUPPORTED = 4, /* valid request this build does not implement */
+    TB_ERR_CUDA = 5         /* a CUDA call or launch failed */
+} tb_status_t;
+
+/* Library version as 10000*major + 100*minor + patch. */
+TB_API int tb_version(void);
+
+/* Static text for a status code (never NULL). */
+TB_API const char *tb_status_string(tb_status_t status);
+
+/* Bytes of the packed codes of an N x K matrix (scales not included):
+ * N*K/4 for ternary and 2-bit, 3*N*K/8 for 3-bit; 0 for bad arguments. */
+TB_API size_t tb_packed_bytes(tb_grid_t grid, int64_t N, int64_t K);
+
+/* Bytes of the bf16 scales of an N x K matrix: N * (K/128) * 2; 0 for bad
+ * arguments. */
+TB_API size_t tb_scale_bytes(int64_t N, int64_t K);
+
+/* Group scales by absmax (rule above; ThinkBit page, 어떻게 동작하나, one
+ * bf16 scale per 128 weights).
+ *   W       [N][K] fp32 or bf16 (w_dtype), device.
+ *   scales  [N][K/128] bf16 bit patterns, device, written. */
+TB_API tb_status_t tb_scales_absmax(const void *W, tb_dtype_t w_dtype, int64_t N, int64_t K, tb_grid_t grid,
+                             uint16_t *scales, tb_stream_t stream);
+
+/* Round-to-nearest quantize and bit-pack (rules and layout above;
+ * ThinkBit page, 어떻게 동작하나 and 무엇과 다른가).
+ *   W          [N][K] fp32 or bf16 (w_dtype), device.
+ *   scales     [N][K/128] bf16, device (e.g. from tb_scales_absmax).
+ *   packed     tb_packed_bytes(grid, N, K) bytes, device, fully written.
+ *   bad_count  device int32, or NULL; when given, it is OVERWRITTEN with
+ *              the number of weights that met a NaN/Inf weight or an
+ *              invalid scale. */
+TB_API tb_status_t tb_pack(const void *W, tb_dtype_t w_dtype, int64_t N, int64_t K, tb_grid_t grid,
+                    const uint16_t *scales, void *packed, int32_t *bad_count, tb_stream_t stream);
+
+/* Inverse of the bit layout: codes[n][k] = c (int8), device, [N][K]. */
+TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int64_t K, int8_t *codes,
+                      tb_stream_t stream);
+
+/* Batch-1 GEMV y = W x over packed W (ThinkBit page, 무엇인가: one read of
+ * every weight per decoded token; 전제와 한계: the direct 2/3-bit reader).
+ *   packed, scales  as produced by tb_pack.
+ *   x               [K] bf16, device, 16-byte aligned.
+ *   y               [N] fp32 or bf16 (y_dtype), device, written. */
+TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *x, void *y,
+                    tb_dtype_t y_dtype, int64_t N, int64_t K, tb_stream_t stream);
+
+/* Small-batch GEMM Y = X W^T, 1 <= M <= 64.
+ *   X  [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device.
+ *   Y  [M][ldy] fp32 or bf16, ldy >= N, device; Y[m][n] for n < N written. */
+TB_API tb_status_t tb_gemm(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *X, int64_t ldx,
+                    void *Y, tb_dtype_t y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                    tb_stream_t stream);
+
+/* One linear layer of a grouped launch. */
+typedef struct {
+    const void *packed;     /* device */
+    const uint16_t *scales; /* device */
+    const uint16_t *x;      /* [K] bf16, device, 16-byte aligned */
+    void *y;                /* [N], device */
+    int64_t N, K;
+    int32_t grid;    /* tb_grid_t */
+    int32_t y_dtype; /* tb_dtype_t */
+} tb_linear_t;
+
+#define TB_MAX_LAYER_ITEMS 16
+
+/* Mixed-grid grouped GEMV: every item is an independent y = W x with its
+ * own grid, shape, input and output, all run by ONE kernel launch (e.g. a
+ * decoder layer's q, k, v, o, gate, up and down projections, each on its
+ * own grid; ThinkBit page, 무엇과 다른가: grids chosen per layer).
+ *   items    HOST array of n_items descriptors (read before returning).
+ *   n_items  1 .. TB_MAX_LAYER_ITEMS.
+ * Outputs of different items must not overlap. */
+TB_API tb_status_t tb_layer_gemv(const tb_linear_t *items, int n_items, tb_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TB_B200_H */

@@ -1,0 +1,110 @@
+"""The C interface on the host (no GPU needed): the shared library loads,
+exports every entry point include/tb.h declares, computes sizes in closed
+form and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from decode_gemv_tb_b200 import build as tbbuild
+from decode_gemv_tb_b200 import tb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tb.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tbbuild.build()
+    return tb.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*TB_API\s+(?:const\s+)?[a-z_0-9]+\s*\*?\s*(tb_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("tb_pack", "tb_unpack", "tb_gemv", "tb_gemm", "tb_layer_gemv", "tb_scales_absmax",
+                 "tb_packed_bytes", "tb_scale_bytes", "tb_status_string", "tb_version"):
+        assert must in names
+    assert set(names) == set(tb.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", tb.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = {line.split()[-1] for line in out.stdout.splitlines() if " T " in line}
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+    # nothing but the C interface is exported
+    assert {n for n in exported if not n.startswith("tb_")} <= {"_init", "_fini"}
+
+
+def test_sizes_closed_form(lib):
+    for grid, bits in ((0, 2), (1, 2), (2, 3)):
+        for N, K in ((1, 128), (256, 1024), (17408, 5120), (5120, 17408)):
+            assert tb.packed_bytes(grid, N, K) == N * K * bits // 8
+            assert tb.scale_bytes(N, K) == N * (K // 128) * 2
+            # 2.125 / 3.125 bits per weight including scales
+            assert 8 * (tb.packed_bytes(grid, N, K) + tb.scale_bytes(N, K)) == N * K * (bits + 0.125)
+    assert tb.packed_bytes(1, 4, 100) == 0 and tb.packed_bytes(7, 4, 128) == 0 and tb.scale_bytes(0, 128) == 0
+    assert lib.tb_version() >= 100
+    for s in range(6):
+        assert lib.tb_status_string(s)
+
+
+FAKE = 1 << 40  # a 256-byte-aligned address that is never dereferenced
+
+
+def test_argument_errors_before_launch(lib):
+    A = FAKE
+    # null pointers / bad enums -> TB_ERR_ARG (1)
+    assert lib.tb_gemv(0, 1, A, A, A, 0, 16, 128, 0) == 1
+    assert lib.tb_gemv(A, 9, A, A, A, 0, 16, 128, 0) == 1
+    assert lib.tb_gemv(A, 1, A, A, A, 5, 16, 128, 0) == 1
+    assert lib.tb_pack(A, 3, 16, 128, 1, A, A, 0, 0) == 1
+    assert lib.tb_layer_gemv(0, 1, 0) == 1
+    items = (tb.Linear * 17)()
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 17, 0) == 1
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 0, 0) == 1
+    # shapes -> TB_ERR_SHAPE (2)
+    assert lib.tb_gemv(A, 1, A, A, A, 0, 0, 128, 0) == 2
+    assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 100, 0) == 2
+    assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 0, 0) == 2
+    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 16, 65, 16, 128, 0) == 2
+    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 16, 0, 16, 128, 0) == 2
+    assert lib.tb_gemm(A, 1, A, A, 120, A, 0, 16, 4, 16, 128, 0) == 2
+    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 8, 4, 16, 128, 0) == 2
+    assert lib.tb_pack(A, 0, 16, 200, 1, A, A, 0, 0) == 2
+    assert lib.tb_unpack(A, 1, -1, 128, A, 0) == 2
+    # alignment -> TB_ERR_ALIGN (3)
+    assert lib.tb_gemv(A + 8, 1, A, A, A, 0, 16, 128, 0) == 3
+    assert lib.tb_gemv(A, 1, A + 1, A, A, 0, 16, 128, 0) == 3
+    assert lib.tb_gemv(A, 1, A, A + 2, A, 0, 16, 128, 0) == 3
+    assert lib.tb_gemv(A, 1, A, A, A + 2, 0, 16, 128, 0) == 3
+    assert lib.tb_gemm(A, 1, A, A, 132, A, 0, 16, 4, 16, 128, 0) == 3
+    assert lib.tb_pack(A + 4, 0, 16, 128, 1, A, A, 0, 0) == 3
+    items = (tb.Linear * 2)()
+    for i in range(2):
+        items[i] = tb.Linear(A, A, A, A, 16, 128, 1, 0)
+    items[1].x = A + 8
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0) == 3
+    items[1].x = A
+    items[1].K = 130
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0) == 2
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = tb._lib
+    tb._lib = None
+    try:
+        with pytest.raises(tb.TBError):
+            tb.load(str(tmp_path / "missing.so"))
+    finally:
+        tb._lib = saved

@@ -1,0 +1,247 @@
+"""CUDA path vs the CPU oracle, element by element, through the C
+interface.  Pack and unpack must be bit-exact; GEMV / GEMM outputs must be
+within |y - y_ref| <= 1e-5 * sum_k |x_k w_k| (fp32) or that plus
+4e-3 |y_ref| (bf16).  The oracle always packs from the same weights
+itself; nothing it consumes comes from the GPU."""
+import numpy as np
+import pytest
+import torch
+
+from decode_gemv_tb_b200 import synth
+from decode_gemv_tb_b200 import tb
+from tests.helpers import assert_within, u16, u32, w_np
+
+pytestmark = pytest.mark.gpu
+GRIDS = (tb.TERNARY, tb.INT2, tb.INT3)
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    tb.load()
+
+
+def gpu_quantize(W, grid):
+    s = tb.tb_scales_absmax(W, grid)
+    bad = torch.zeros(1, dtype=torch.int32, device=W.device)
+    p = tb.tb_pack(W, grid, s, bad_count=bad)
+    return s, p, int(bad.item())
+
+
+# ------------------------------------------------------------------ pack
+
+@pytest.mark.parametrize("grid", GRIDS)
+@pytest.mark.parametrize("wdt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", [(1, 128), (5, 256), (37, 640), (256, 1024), (2048, 2048)])
+def test_scales_pack_unpack_bitexact(oracle, grid, wdt, shape):
+    N, K = shape
+    W = synth.gaussian_weights(N, K, seed=N * 7 + K + grid, dtype=wdt).to(DEV)
+    s, p, bad = gpu_quantize(W, grid)
+    ws = w_np(W)
+    s_ref = oracle.scales_absmax(ws, grid)
+    assert np.array_equal(u16(s), s_ref)
+    p_ref, bad_ref = oracle.pack(ws, grid, s_ref)
+    assert np.array_equal(u32(p).reshape(p_ref.shape), p_ref)
+    assert bad == bad_ref == 0
+    codes = tb.tb_unpack(p, grid, N, K)
+    assert np.array_equal(codes.cpu().numpy(), oracle.unpack(p_ref, grid, N, K))
+
+
+def test_config1_exact_reconstruction(oracle):
+    """Config 1: codewords uniform on {-2..1}, scales |N(0,1)|*0.02+1e-3,
+    W = c*s in fp32; packing with those scales must give back c."""
+    N, K = synth.CONFIG1["N"], synth.CONFIG1["K"]
+    c = synth.uniform_codes(N, K, -2, 1, seed=1000)
+    s = synth.config1_scales(N, K, seed=1000)
+    W = (c.float() * s.float().repeat_interleave(128, dim=1)).to(DEV)
+    p = tb.tb_pack(W, tb.INT2, s.to(DEV))
+    assert np.array_equal(tb.tb_unpack(p, tb.INT2, N, K).cpu().numpy(), c.numpy())
+    p_ref, _ = oracle.pack(W.cpu().numpy(), tb.INT2, u16(s))
+    assert np.array_equal(u32(p).reshape(p_ref.shape), p_ref)
+
+
+@pytest.mark.parametrize("grid", GRIDS)
+def test_pack_edge_values(oracle, grid):
+    """Ties, clamps, NaN/Inf weights, invalid and tiny scales, subnormals."""
+    rng = np.random.default_rng(7 + grid)
+    N, K = 8, 256
+    sv = np.array([1.0, 0.5, 3.0, 0.375, 1e-20, 2.0 ** -126, 0.0, -1.0, np.inf, np.nan, 1e-38, 7.0e-39,
+                   0.015625, 1.5e-3, 2.0 ** -135, 4.0], dtype=np.float32)[: N * 2].reshape(N, 2)
+    s = torch.from_numpy(sv).to(torch.bfloat16)
+    sval = s.float().numpy()
+    W = np.empty((N, K), dtype=np.float32)
+    for n in range(N):
+        for j in range(2):
+            base = sval[n, j] if np.isfinite(sval[n, j]) and sval[n, j] > 0 else 1.0
+            k2 = rng.integers(-11, 12, size=128)          # odd/even multiples of s/2: ties and exact codes
+            blk = (k2 * np.float64(base) / 2).astype(np.float32)
+            blk[::7] = np.nextafter(blk[::7], np.float32(np.inf))
+            blk[::11] = np.nextafter(blk[::11], np.float32(-np.inf))
+            blk[5] = np.nan
+            blk[6] = np.inf
+            blk[9] = -np.inf
+            blk[10] = 3e38
+            blk[12] = 1e-45
+            W[n, 128 * j:128 * (j + 1)] = blk
+    Wt = torch.from_numpy(W).to(DEV)
+    bad = torch.zeros(1, dtype=torch.int32, device=DEV)
+    p = tb.tb_pack(Wt, grid, s.to(DEV), bad_count=bad)
+    p_ref, bad_ref = oracle.pack(W, grid, u16(s))
+    assert np.array_equal(u32(p).reshape(p_ref.shape), p_ref)
+    assert int(bad.item()) == bad_ref > 0
+    # the scales rule on the same data (NaN / Inf ignored, zero groups -> 1.0)
+    W2 = W.copy()
+    W2[3, :128] = 0.0
+    s_gpu = tb.tb_scales_absmax(torch.from_numpy(W2).to(DEV), grid)
+    assert np.array_equal(u16(s_gpu), oracle.scales_absmax(W2, grid))
+
+
+def test_pack_outliers_bf16(oracle):
+    """Config 5 distribution: bf16 N(0, 0.02) with 0.1% entries x20."""
+    W = synth.outlier_weights(512, 1024, seed=5001).to(DEV)
+    for grid in GRIDS:
+        s, p, bad = gpu_quantize(W, grid)
+        s_ref = oracle.scales_absmax(u16(W), grid)
+        p_ref, _ = oracle.pack(u16(W), grid, s_ref)
+        assert np.array_equal(u16(s), s_ref)
+        assert np.array_equal(u32(p).reshape(p_ref.shape), p_ref)
+
+
+# ------------------------------------------------------------------ GEMV
+
+def oracle_problem(oracle, grid, N, K, seed, wdt=torch.float32):
+    W = synth.gaussian_weights(N, K, seed=seed, dtype=wdt)
+    x = synth.activations(K, seed=seed)
+    ws = w_np(W)
+    s_ref = oracle.scales_absmax(ws, grid)
+    p_ref, _ = oracle.pack(ws, grid, s_ref)
+    return W, x, s_ref, p_ref
+
+
+def to_dev_packed(p_ref):
+    return torch.from_numpy(p_ref.reshape(-1).view(np.uint8).copy()).to(DEV)
+
+
+def to_dev_bits(a):
+    return torch.from_numpy(a.astype(np.uint16).view(np.int16).copy()).to(DEV).view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("grid", GRIDS)
+@pytest.mark.parametrize("shape", [(1, 128), (7, 256), (15, 384), (16, 1152), (17, 640), (33, 1024), (100, 2048),
+                                   (256, 1024)])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_gemv_parity_small(oracle, grid, shape, out):
+    N, K = shape
+    W, x, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=N * 31 + K)
+    y64, yabs = oracle.gemv64(p_ref, grid, s_ref, u16(x), N, K)
+    # GPU pipeline from the same W: scales, pack, GEMV
+    s, p, _ = gpu_quantize(W.to(DEV), grid)
+    guard = 64
+    ybuf = torch.full((N + guard,), 123.25, dtype=torch.float32 if out == "f32" else torch.bfloat16, device=DEV)
+    y = ybuf[:N]
+    tb.tb_gemv(p, grid, s, x.to(DEV), N, K, y=y)
+    assert_within(y, y64, yabs, out, oracle, f"gemv {shape} grid {grid}")
+    assert torch.all(ybuf[N:] == 123.25), "wrote past the end of y"
+
+
+@pytest.mark.parametrize("case", synth.config2_cases(), ids=lambda m: m.name)
+def test_gemv_config2(oracle, case):
+    N, K, grid = case.N, case.K, case.grid
+    W, x, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=case.seed)
+    y64, yabs = oracle.gemv64(p_ref, grid, s_ref, u16(x), N, K)
+    y = tb.tb_gemv(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), x.to(DEV), N, K)
+    assert_within(y, y64, yabs, "f32", oracle, case.name)
+
+
+def test_gemv_config1(oracle):
+    N, K = synth.CONFIG1["N"], synth.CONFIG1["K"]
+    c = synth.uniform_codes(N, K, -2, 1, seed=1000)
+    s = synth.config1_scales(N, K, seed=1000)
+    W = c.float() * s.float().repeat_interleave(128, dim=1)
+    x = synth.activations(K, seed=1000)
+    p_ref, _ = oracle.pack(W.numpy(), tb.INT2, u16(s))
+    y64, yabs = oracle.gemv64(p_ref, tb.INT2, u16(s), u16(x), N, K)
+    p = tb.tb_pack(W.to(DEV), tb.INT2, s.to(DEV))
+    y = tb.tb_gemv(p, tb.INT2, s.to(DEV), x.to(DEV), N, K)
+    assert_within(y, y64, yabs, "f32", oracle, "config1")
+
+
+@pytest.mark.parametrize("grid", GRIDS)
+def test_gemv_integer_exact_bitwise(oracle, grid):
+    """Integer x and power-of-two scales: every partial sum is exact, so the
+    GPU result equals the oracle's bit for bit."""
+    lo, hi = oracle.GRID_RANGE[grid]
+    N, K = 48, 1024
+    g = torch.Generator().manual_seed(99 + grid)
+    c = torch.randint(lo, hi + 1, (N, K), generator=g)
+    x = torch.randint(-8, 9, (K,), generator=g).to(torch.bfloat16)
+    s = torch.full((N, K // 128), 2.0 ** -5, dtype=torch.bfloat16)
+    W = c.float() * 2.0 ** -5
+    p_ref, _ = oracle.pack(W.numpy(), grid, u16(s))
+    y64, _ = oracle.gemv64(p_ref, grid, u16(s), u16(x), N, K)
+    y = tb.tb_gemv(to_dev_packed(p_ref), grid, s.to(DEV), x.to(DEV), N, K)
+    assert np.array_equal(y.cpu().numpy(), y64.astype(np.float32))
+
+
+def test_gemv_deterministic():
+    N, K = 1024, 4096
+    W = synth.gaussian_weights(N, K, seed=5, device=DEV)
+    x = synth.activations(K, seed=5, device=DEV)
+    for grid in GRIDS:
+        s, p, _ = gpu_quantize(W, grid)
+        y1 = tb.tb_gemv(p, grid, s, x, N, K)
+        y2 = tb.tb_gemv(p, grid, s, x, N, K)
+        assert torch.equal(y1, y2)
+
+
+# ------------------------------------------------------------------ grouped layer
+
+def test_layer_gemv_mixed_grids(oracle):
+    """Seven projections of reduced width, each on its own grid, one launch;
+    equals the per-matrix GEMV bit for bit and the oracle within tolerance."""
+    shapes = synth.qwen3_layer_shapes(512, 1536, kv_dim=128)
+    grids = [tb.INT3, tb.INT2, tb.INT2, tb.TERNARY, tb.INT3, tb.TERNARY, tb.TERNARY]
+    items, refs, singles = [], [], []
+    for i, ((name, N, K), grid) in enumerate(zip(shapes, grids)):
+        W, x, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=400 + i)
+        refs.append(oracle.gemv64(p_ref, grid, s_ref, u16(x), N, K))
+        p, s, xd = to_dev_packed(p_ref), to_dev_bits(s_ref), x.to(DEV)
+        y = torch.empty(N, dtype=torch.float32 if i % 2 == 0 else torch.bfloat16, device=DEV)
+        items.append((p, grid, s, xd, y, N, K))
+        singles.append(tb.tb_gemv(p, grid, s, xd, N, K, out_dtype=y.dtype))
+    tb.tb_layer_gemv(items)
+    for i, it in enumerate(items):
+        y = it[4]
+        assert_within(y, *refs[i], "f32" if i % 2 == 0 else "bf16", oracle, shapes[i][0])
+        assert torch.equal(y, singles[i])
+
+
+# ------------------------------------------------------------------ GEMM
+
+@pytest.mark.parametrize("grid", GRIDS)
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 9, 16, 17, 32, 64])
+def test_gemm_parity(oracle, grid, M):
+    N, K = 80, 768
+    W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=700 + M)
+    X = synth.activations(K, seed=800 + M, M=M)
+    Y64, Yabs = oracle.gemm64(p_ref, grid, s_ref, u16(X), N, K)
+    Y = tb.tb_gemm(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), X.to(DEV), N, K)
+    assert_within(Y, Y64, Yabs, "f32", oracle, f"gemm M={M}")
+
+
+def test_gemm_strided_bf16_out(oracle):
+    N, K, M = 40, 512, 12
+    W, _, s_ref, p_ref = oracle_problem(oracle, tb.INT2, N, K, seed=900)
+    Xfull = synth.activations(K + 64, seed=901, M=M)
+    X = Xfull[:, :K]
+    Y64, Yabs = oracle.gemm64(p_ref, tb.INT2, s_ref, u16(X.contiguous()), N, K)
+    Ybuf = torch.zeros((M, N + 24), dtype=torch.bfloat16, device=DEV)
+    rc = tb.load().tb_gemm(to_dev_packed(p_ref).data_ptr(), tb.INT2, to_dev_bits(s_ref).data_ptr(),
+                           Xfull.to(DEV).data_ptr(), K + 64, Ybuf.data_ptr(), tb.BF16, N + 24, M, N, K,
+                           torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert_within(Ybuf[:, :N], Y64, Yabs, "bf16", oracle, "gemm strided")
+    assert torch.all(Ybuf[:, N:] == 0)
