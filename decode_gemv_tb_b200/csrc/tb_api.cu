@@ -2,6 +2,7 @@
 // then one launch on the caller's stream.  No allocation, no
 // synchronization, no host fallback: every computation runs in the kernels.
 #include <algorithm>
+#include <climits>
 #include <cstring>
 
 #include "../../include/tb.h"
@@ -40,6 +41,7 @@ tb_status_t check_out(const void* y, int ydt) {
 Item make_item(const void* packed, int grid, const uint16_t* scales, const uint16_t* X, int64_t ldx, void* Y,
                int ydt, int64_t ldy, int M, int64_t N, int64_t K) {
     Item it;
+    std::memset(&it, 0, sizeof(it));
     it.packed = static_cast<const uint8_t*>(packed);
     it.scales = scales;
     it.X = X;
@@ -51,28 +53,178 @@ Item make_item(const void* packed, int grid, const uint16_t* scales, const uint1
     it.grid = grid;
     it.ydt = ydt;
     it.M = M;
-    it.unit_begin = 0;
     return it;
 }
 
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// Workspace of one item: prepared activations [M][K] bf16, then per-group
+// (offset * sum x, 2^S) pairs [K/128][M].
+size_t item_workspace(int64_t M, int64_t K) {
+    return align256((size_t)(M * K * 2)) + align256((size_t)((K / kGroup) * M * 8));
+}
+
+// Batch-1 launches additionally need one counter per 32-row tile and two
+// 32-float partial-sum slots per warp (at most kMaxSKWarps warps, and never
+// more warps than tile-groups).
+constexpr int64_t kMaxSKWarps = 8192;
+size_t sk_extra_workspace(int64_t tiles, int64_t tile_groups) {
+    const int64_t w = std::min(kMaxSKWarps, std::max<int64_t>(tile_groups, 1));
+    return align256((size_t)(tiles * 4)) + align256((size_t)(w * 2 * 32 * 4));
+}
+
+int device_sms() {
+    static int sms[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (sms[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        sms[dev] = v;
+    }
+    return sms[dev];
+}
+
 // Orders items by per-tile cost (descending) so that the expensive tiles
-// are dispatched first, assigns CTA ranges and launches.
-tb_status_t launch_items(Item* items, int n, int nt, cudaStream_t st) {
+// are dispatched first, chooses how many warps share a 16-row tile (the
+// K split), lays out the workspace and launches.
+tb_status_t launch_items(Item* items, int n, int nt, void* ws, size_t ws_bytes, bool overlap, cudaStream_t st) {
     Launch L;
     std::memset(&L, 0, sizeof(L));
     int order[kMaxItems];
     for (int i = 0; i < n; ++i) order[i] = i;
     auto cost = [&](int i) { return row_bytes(items[i].grid, items[i].K); };
     std::stable_sort(order, order + n, [&](int a, int b) { return cost(a) > cost(b); });
-    int64_t ctas = 0;
+
+    // K split per item: about 16 groups (2048 weights) per warp, then more
+    // splits everywhere while the launch has too few warps to fill the GPU
+    // (each split needs at least one group).
+    int S[kMaxItems];
+    for (int i = 0; i < n; ++i) {
+        const int64_t G = items[i].K / kGroup;
+        int s = 1;
+        while (s < 8 && G / (2 * s) >= 16) s *= 2;
+        S[i] = s;
+    }
+    const int64_t want = (int64_t)device_sms() * 16;
+    for (;;) {
+        int64_t warps = 0;
+        bool grow = false;
+        for (int i = 0; i < n; ++i) warps += (items[i].N + 31) / 32 * S[i];
+        if (warps >= want) break;
+        for (int i = 0; i < n; ++i)
+            if (S[i] < 8 && items[i].K / kGroup >= 2 * S[i]) {
+                S[i] *= 2;
+                grow = true;
+            }
+        if (!grow) break;
+    }
+    int64_t gpw = 0;  // most groups any warp handles
+    for (int i = 0; i < n; ++i) gpw = std::max<int64_t>(gpw, (items[i].K / kGroup + S[i] - 1) / S[i]);
+    L.scl_stride = (int32_t)((gpw + 3) / 4 * 4 + 2);  // >= gpw, = 2 mod 4
+    if (linear_smem_bytes(nt, L.scl_stride) > 227 * 1024) return TB_ERR_UNSUPPORTED;
+
+    size_t need = 0;
+    int64_t ctas = 0, prep = 0;
+    char* w = static_cast<char*>(ws);
     for (int j = 0; j < n; ++j) {
-        L.it[j] = items[order[j]];
-        L.it[j].unit_begin = (int32_t)ctas;
-        ctas += (L.it[j].N + 15) / 16;
+        Item it = items[order[j]];
+        it.ksplit = S[order[j]];
+        it.cta_begin = (int32_t)ctas;
+        it.prep_begin = (int32_t)prep;
+        it.xs = reinterpret_cast<uint16_t*>(w + need);
+        it.cf = reinterpret_cast<float2*>(w + need + align256((size_t)(it.M * it.K * 2)));
+        need += item_workspace(it.M, it.K);
+        const int64_t tiles_per_cta = 8 / it.ksplit;
+        ctas += ((it.N + 31) / 32 + tiles_per_cta - 1) / tiles_per_cta;
+        prep += (it.K / kGroup) * it.M;
+        L.it[j] = it;
     }
     L.n_items = n;
-    if (ctas > 0x7FFFFFFF) return TB_ERR_SHAPE;
-    return cuda_status(launch_linear(L, nt, (int)ctas, st));
+    if (!ws || ws_bytes < need) return TB_ERR_ARG;
+    if (ctas > 0x7FFFFFFF || prep > 0x7FFFFFFF) return TB_ERR_SHAPE;
+    return cuda_status(launch_linear(L, nt, (int)ctas, (int)prep, overlap, st));
+}
+
+// Batch-1 (M == 1) launch: preparation kernel + stream-K kernel.  3-bit
+// items form the first partition, 2-bit items the second (each warp works
+// on one code width only); warps are split between them by cost.
+tb_status_t launch_sk_items(const Item* items, int n, void* ws, size_t ws_bytes, bool overlap, cudaStream_t st) {
+    Launch P;
+    std::memset(&P, 0, sizeof(P));
+    SKLaunch L;
+    std::memset(&L, 0, sizeof(L));
+    int order[kMaxItems], n3 = 0;
+    for (int i = 0; i < n; ++i)
+        if (items[i].grid == TB_GRID_INT3) order[n3++] = i;
+    for (int i = 0, k = n3; i < n; ++i)
+        if (items[i].grid != TB_GRID_INT3) order[k++] = i;
+    char* w = static_cast<char*>(ws);
+    size_t need = 0;
+    int64_t prep = 0, tiles = 0, tg_all = 0;
+    int64_t tg = 0, cost = 0, part_cost[2] = {0, 0};
+    for (int j = 0; j < n; ++j) {
+        if (j == n3) tg = cost = 0;  // the 2-bit partition starts its positions again
+        Item it = items[order[j]];
+        it.prep_begin = (int32_t)prep;
+        it.xs = reinterpret_cast<uint16_t*>(w + need);
+        it.cf = reinterpret_cast<float2*>(w + need + align256((size_t)(it.K * 2)));
+        need += item_workspace(1, it.K);
+        prep += it.K / kGroup;
+        P.it[j] = it;
+
+        SKItem& s = L.it[j];
+        s.packed = it.packed;
+        s.scales = it.scales;
+        s.xs = it.xs;
+        s.cf = it.cf;
+        s.Y = it.Y;
+        s.N = it.N;
+        s.K = it.K;
+        s.rbytes = row_bytes(it.grid, it.K);
+        s.G = (int32_t)(it.K / kGroup);
+        s.T = (int32_t)((it.N + 31) / 32);
+        s.grid = it.grid;
+        s.ydt = it.ydt;
+        s.unit_cost = it.grid == TB_GRID_INT3 ? 3 : 2;
+        s.tg_base = tg;
+        s.tg_count = (int64_t)s.T * s.G;
+        s.cost_base = cost;
+        s.tile_base = (int32_t)tiles;
+        tg += s.tg_count;
+        tg_all += s.tg_count;
+        cost += s.tg_count * s.unit_cost;
+        part_cost[j < n3 ? 0 : 1] = cost;
+        tiles += s.T;
+    }
+    P.n_items = n;
+    L.n_items = n;
+    if (part_cost[0] >= ((int64_t)1 << 31) || part_cost[1] >= ((int64_t)1 << 31))
+        return TB_ERR_UNSUPPORTED;  // partition arithmetic is 32-bit
+    // layout with the device-independent bound on the warp count (the one
+    // tb_workspace_bytes uses), checked before any CUDA call
+    L.counters = reinterpret_cast<int32_t*>(w + need);
+    L.partials = reinterpret_cast<float*>(w + need + align256((size_t)(tiles * 4)));
+    need += sk_extra_workspace(tiles, tg_all);
+    P.zero = L.counters;
+    P.n_zero = (int32_t)tiles;
+    if (!ws || ws_bytes < need) return TB_ERR_ARG;
+    if (tiles > 0x7FFFFFFF || prep > 0x7FFFFFFF) return TB_ERR_SHAPE;
+    const int resident = gemv_sk_resident_warps();
+    if (resident <= 0) return TB_ERR_CUDA;
+    // at most the resident warps; at least about four tile-groups per warp
+    const int64_t W = std::max<int64_t>(1, std::min<int64_t>({(int64_t)resident, (tg_all + 3) / 4, kMaxSKWarps}));
+    const int64_t C = part_cost[0] + part_cost[1];
+    int64_t W3 = part_cost[0] == 0 ? 0 : (part_cost[1] == 0 ? W : (W * part_cost[0] + C / 2) / C);
+    if (part_cost[0] > 0) W3 = std::max<int64_t>(W3, 1);
+    if (part_cost[1] > 0) W3 = std::min<int64_t>(W3, W - 1);
+    const int64_t W2 = W - W3;
+    L.W = (int32_t)W;
+    L.part[0] = {0, n3, 0, (int32_t)W3, (uint32_t)part_cost[0],
+                 (uint32_t)(W3 ? (part_cost[0] + W3 - 1) / W3 : 1)};
+    L.part[1] = {n3, n - n3, (int32_t)W3, (int32_t)W2, (uint32_t)part_cost[1],
+                 (uint32_t)(W2 ? (part_cost[1] + W2 - 1) / W2 : 1)};
+    return cuda_status(launch_gemv_sk(P, (int)prep, L, (int)((W + 7) / 8), overlap, st));
 }
 
 }  // namespace
@@ -129,40 +281,72 @@ tb_status_t tb_unpack(const void* packed, tb_grid_t grid, int64_t N, int64_t K, 
     return cuda_status(launch_unpack(packed, grid, N, K, codes, static_cast<cudaStream_t>(stream)));
 }
 
+size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || M > 64 || !shape_ok(N, K)) return 0;
+    if (M == 1) {
+        const int64_t tiles = (N + 31) / 32;
+        return item_workspace(1, K) + sk_extra_workspace(tiles, tiles * (K / kGroup));
+    }
+    return item_workspace(std::min<int64_t>(M, 16), K);
+}
+
+size_t tb_layer_workspace_bytes(const tb_linear_t* items, int n_items) {
+    if (!items || n_items < 1 || n_items > TB_MAX_LAYER_ITEMS) return 0;
+    size_t b = 0;
+    int64_t tiles = 0, tgs = 0;
+    for (int i = 0; i < n_items; ++i) {
+        if (!shape_ok(items[i].N, items[i].K)) return 0;
+        b += item_workspace(1, items[i].K);
+        tiles += (items[i].N + 31) / 32;
+        tgs += (items[i].N + 31) / 32 * (items[i].K / kGroup);
+    }
+    return b + sk_extra_workspace(tiles, tgs);
+}
+
 tb_status_t tb_gemv(const void* packed, tb_grid_t grid, const uint16_t* scales, const uint16_t* x, void* y,
-                    tb_dtype_t y_dtype, int64_t N, int64_t K, tb_stream_t stream) {
+                    tb_dtype_t y_dtype, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                    tb_stream_t stream) {
     tb_status_t s = check_weights(packed, grid, scales, N, K);
     if (s != TB_OK) return s;
     if (!x) return TB_ERR_ARG;
     if ((s = check_out(y, y_dtype)) != TB_OK) return s;
-    if (!aligned(x, 16)) return TB_ERR_ALIGN;
+    if (!workspace) return TB_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(workspace, 256)) return TB_ERR_ALIGN;
     Item it = make_item(packed, grid, scales, x, K, y, y_dtype, N, 1, N, K);
-    return launch_items(&it, 1, 1, static_cast<cudaStream_t>(stream));
+    return launch_sk_items(&it, 1, workspace, workspace_bytes, false, static_cast<cudaStream_t>(stream));
 }
 
 tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, const uint16_t* X, int64_t ldx,
                     void* Y, tb_dtype_t y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                    tb_stream_t stream) {
+                    void* workspace, size_t workspace_bytes, tb_stream_t stream) {
     tb_status_t s = check_weights(packed, grid, scales, N, K);
     if (s != TB_OK) return s;
     if (!X) return TB_ERR_ARG;
     if ((s = check_out(Y, y_dtype)) != TB_OK) return s;
     if (M < 1 || M > 64 || ldx < K || ldy < N) return TB_ERR_SHAPE;
-    if (!aligned(X, 16) || ldx % 8 != 0) return TB_ERR_ALIGN;
+    if (!workspace) return TB_ERR_ARG;
+    if (!aligned(X, 16) || ldx % 8 != 0 || !aligned(workspace, 256)) return TB_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M == 1) {
+        Item it = make_item(packed, grid, scales, X, ldx, Y, y_dtype, N, 1, N, K);
+        return launch_sk_items(&it, 1, workspace, workspace_bytes, false, st);
+    }
     // column blocks of up to 16 batch rows per launch
     const size_t ysz = y_dtype == TB_F32 ? 4 : 2;
     for (int64_t m0 = 0; m0 < M; m0 += 16) {
         const int mb = (int)std::min<int64_t>(16, M - m0);
         Item it = make_item(packed, grid, scales, X + m0 * ldx, ldx, static_cast<char*>(Y) + m0 * ldy * ysz, y_dtype,
                             ldy, mb, N, K);
-        if ((s = launch_items(&it, 1, mb > 8 ? 2 : 1, st)) != TB_OK) return s;
+        if ((s = launch_items(&it, 1, mb > 8 ? 2 : 1, workspace, workspace_bytes, false, st)) != TB_OK) return s;
     }
     return TB_OK;
 }
 
-tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, tb_stream_t stream) {
+tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags, void* workspace,
+                          size_t workspace_bytes, tb_stream_t stream) {
     if (!items || n_items < 1 || n_items > TB_MAX_LAYER_ITEMS) return TB_ERR_ARG;
+    if ((flags & ~(unsigned)TB_FLAG_OVERLAP_PREVIOUS) != 0 || !workspace) return TB_ERR_ARG;
+    if (!aligned(workspace, 256)) return TB_ERR_ALIGN;
     Item its[kMaxItems];
     for (int i = 0; i < n_items; ++i) {
         const tb_linear_t& l = items[i];
@@ -173,7 +357,8 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, tb_stream_t str
         if (!aligned(l.x, 16)) return TB_ERR_ALIGN;
         its[i] = make_item(l.packed, l.grid, l.scales, l.x, l.K, l.y, l.y_dtype, l.N, 1, l.N, l.K);
     }
-    return launch_items(its, n_items, 1, static_cast<cudaStream_t>(stream));
+    return launch_sk_items(its, n_items, workspace, workspace_bytes, (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0,
+                           static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -29,16 +29,54 @@ __host__ __device__ inline int64_t row_bytes(int g, int64_t K) { return g == kIn
 struct Item {
     const uint8_t* packed;
     const uint16_t* scales;
-    const uint16_t* X;   // [M][ldx] bf16
-    void* Y;             // [M][ldy]
+    const uint16_t* X;   // [M][ldx] bf16 activations
+    void* Y;             // [M][ldy] outputs
+    uint16_t* xs;        // workspace: [M][K] prepared activations (see tb_linear.cu)
+    float2* cf;          // workspace: [K/128][M] per-group (offset * sum x, 2^S)
     int64_t N, K, ldx, ldy;
     int32_t grid, ydt, M;
-    int32_t unit_begin;  // first CTA index of this item
+    int32_t cta_begin;   // first CTA of this item in the main launch
+    int32_t prep_begin;  // first warp of this item in the preparation launch
+    int32_t ksplit;      // warps sharing one 32-row tile (1, 2, 4 or 8)
 };
 
 struct Launch {
     Item it[kMaxItems];
     int32_t n_items;
+    int32_t scl_stride;  // scales staged per row per warp (>= groups per warp)
+    int32_t* zero;       // int32 words the preparation kernel clears (stream-K tile counters)
+    int32_t n_zero;
+};
+
+// ---- stream-K batch-1 launch (see tb_linear.cu) ----------------------------
+struct SKItem {
+    const uint8_t* packed;
+    const uint16_t* scales;
+    const uint16_t* xs;  // prepared activations [K]
+    const float2* cf;    // [K/128] (offset * sum x, 2^S)
+    void* Y;
+    int64_t N, K, rbytes;
+    int64_t tg_base, tg_count, cost_base;  // partition (tb_partition.h)
+    int32_t unit_cost, G, T, grid, ydt;
+    int32_t tile_base;   // first tile counter of this item
+};
+
+// Two partitions side by side: the 3-bit items (it[0 .. n3)) on warps
+// [0, W3), the 2-bit items (it[n3 .. n_items)) on warps [W3, W); tile-group
+// and cost positions of the 2-bit items start again at 0.
+struct SKPart {
+    int32_t first, count;  // items
+    int32_t W0, W;         // first warp, warps
+    uint32_t C, Q;         // total cost, cost quota per warp (tb_partition.h)
+};
+
+struct SKLaunch {
+    SKItem it[kMaxItems];
+    int32_t n_items;
+    int32_t W;            // warps in the launch
+    SKPart part[2];       // [0]: 3-bit items, [1]: 2-bit items
+    int32_t* counters;    // one per 32-row tile, zeroed by the preparation kernel
+    float* partials;      // [W][2][32]
 };
 
 // ---- cache-controlled loads ----------------------------------------------
@@ -68,6 +106,17 @@ __device__ __forceinline__ uint4 ld_act_u4(const void* p) {
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t h) { return __uint_as_float(h << 16); }
+
+__device__ __forceinline__ float2 ld_act_f2(const void* p) {
+    float2 v;
+    asm volatile("ld.global.nc.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+    return v;
+}
+
+// Programmatic dependent launch (sm_90+): wait for the grids this one
+// depends on / let the dependent grid start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // bf16x2 a*b+c, one rounding (exact whenever the true result is a bf16)
 __device__ __forceinline__ uint32_t hfma2_bf16(uint32_t a, uint32_t b, uint32_t c) {

@@ -14,8 +14,20 @@ cudaError_t launch_pack(const void* W, int w_dtype, int64_t N, int64_t K, int gr
                         void* packed, int32_t* bad_count, cudaStream_t st);
 cudaError_t launch_unpack(const void* packed, int grid, int64_t N, int64_t K, int8_t* codes, cudaStream_t st);
 
-// Grouped linear launch (GEMV when every item has M == 1).  `nt` is the
-// number of 8-wide column tiles (1 or 2), `ctas` the total CTA count.
-cudaError_t launch_linear(const Launch& L, int nt, int ctas, cudaStream_t st);
+// Grouped linear launch (GEMV when every item has M == 1): the activation
+// preparation kernel, then the main kernel as its programmatic dependent.
+// `nt` is the number of 8-wide column tiles (1 or 2), `ctas` the main grid,
+// `prep_warps` the preparation warp count; `overlap` also launches the
+// preparation kernel as a programmatic dependent of the previous work.
+cudaError_t launch_linear(const Launch& L, int nt, int ctas, int prep_warps, bool overlap, cudaStream_t st);
+// dynamic shared memory of the main kernel
+size_t linear_smem_bytes(int nt, int scl_stride);
+
+struct SKLaunch;
+// Batch-1 path: preparation kernel (also clears P.zero) + stream-K kernel.
+cudaError_t launch_gemv_sk(const Launch& P, int prep_warps, const SKLaunch& L, int ctas, bool overlap,
+                           cudaStream_t st);
+// warps of the stream-K kernel resident at once on the current device (0 on error)
+int gemv_sk_resident_warps();
 
 }  // namespace tb

@@ -4,126 +4,87 @@
 // ThinkBit page "ThinkBit은 2비트 양자화에서 추론 능력 보존을 추론 평가로
 // 검증한다" (onedev.kr/papers/1416): section 무엇인가 -- every decoded token
 // reads every weight, so decode is bound by memory bandwidth; section
-// 어떻게 동작하나 -- w = c * s, one bf16 scale per 128 weights, dequant is
-// one multiply; section 전제와 한계 -- no kernel read the 2/3-bit codes
-// directly, so checkpoints ship in 4-bit containers.
+// 어떻게 동작하나 -- w = c * s, one bf16 scale per 128 weights, dequant is one
+// multiply; section 전제와 한계 -- no kernel read the 2/3-bit codes directly,
+// which is why checkpoints ship in 4-bit containers.
 //
-// Design (sm_100a):
-//  * One CTA (8 warps) owns a 16-row tile of one matrix; its warps split K
-//    by 128-groups (group g goes to warp g mod 8) and reduce through shared
-//    memory in a fixed order: deterministic, no global scratch, no atomics.
-//    The hardware block scheduler balances tiles of different cost; tiles
-//    of the most expensive matrices come first in blockIdx order.
-//  * Weights stream with 64-bit (2-bit container) or 32-bit (3-bit planes)
-//    L1-bypassing loads, PF groups ahead per warp, so every lane keeps
-//    several loads in flight.
-//  * Codes are decoded to exact bf16 integers with one LOP3 (mask the
-//    field, OR the exponent of 128.0) and one bf16x2 FMA (rescale the
-//    field position and subtract 128 + offset) per PAIR of codes.  The
-//    multiply-accumulate runs on the tensor pipe (mma.sync m16n8k16,
-//    fp32 accumulate), which keeps the FP32 and integer pipes free for the
-//    decode: at 2.125 bits/weight the SM issue budget is about 1.5
-//    instructions per weight, less than a CUDA-core decode + FMA costs.
-//  * Each 128-group is accumulated on its own (fp32, tensor pipe) and
-//    multiplied by its scale once; groups are summed in fp32.
+// The arithmetic per output row n and 128-group g is
+//     y[n] += s[n][g] * (sum_k u[n][k] x[k]  -  offset * sum_k x[k])
+// with u = c + offset the stored code (offset 2 or 4), so the codes never
+// need to be turned into signed values; the second sum does not depend on
+// the row and is computed once per call.
 //
-// Fragment mapping (m16n8k16, lane = 4 g + t): A rows are W rows
-// tile*16 + g and + 8.  A k-slot pairs (2t, 2t+1) and (2t+8, 2t+9) carry
-// one decoded code PAIR each; because the packed word keeps codes 2m and
-// 2m+1 in the same field of the two half-words, every pair is two
-// ADJACENT k, so the B fragment of one MMA is four consecutive x values:
-// x is read in its natural layout, no shuffling.
+// Decode without arithmetic.  A bf16 bit pattern P < 256 (exponent field 0
+// or 1) has the value P * 2^-133 exactly.  Masking one 2-bit field at bit
+// position p of each 16-bit half of a packed word therefore yields a bf16x2
+// register holding u * 2^(p-133) for two codes: one LOP3 per code pair, no
+// conversion, no magic-number subtraction.  The factor 2^(133-p) is folded
+// into the activations: a small preparation kernel writes
+//     xs[k] = x[k] * 2^(133 - S_g - p(k))          (exact: powers of two)
+// where S_g = exponent(max |x| of group g) + 7 keeps xs inside the bf16
+// range, plus per group (offset * sum x, 2^S_g).  The tensor pipe then
+// computes sum u * x * 2^-S_g exactly product by product, accumulating in
+// fp32 (mma.sync m16n8k16 bf16, the multiply-accumulate off the ALU and FMA
+// pipes, which the decode needs: at 2.125 bits/weight the SM has about 0.7
+// integer-pipe operations per weight at full HBM speed).
+//
+// Work split: a CTA of 8 warps owns 8/S tiles of 16 rows; the S warps of a
+// tile split K by contiguous 128-groups and reduce through shared memory in
+// a fixed order (deterministic, no atomics, no scratch beyond the prepared
+// activations).  Each warp streams its rows' packed codes into a private
+// shared-memory ring with L1-bypassing cp.async copies, kStages - 1 groups
+// ahead, so no registers are held by loads in flight.  The main kernel is a
+// programmatic dependent of the preparation kernel: it starts its weight
+// copies before waiting for the prepared activations.
 #include "tb_device.cuh"
 #include "tb_internal.h"
+#include "tb_partition.h"
+
+#include <algorithm>
 
 namespace tb {
 namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kPF = 4;  // groups in flight per warp
 
-// bf16 constants
-constexpr uint32_t kMag = 0x43004300u;  // 128.0 | 128.0
-constexpr uint32_t kOne = 0x3F803F80u, kHalf = 0x3F003F00u, kQuarter = 0x3E803E80u, kEighth = 0x3E003E00u,
-                   kSixteenth = 0x3D803D80u;
-// -(128 / 2^q + offset)
-constexpr uint32_t kN130 = 0xC302C302u, kN34 = 0xC208C208u, kN10 = 0xC120C120u;              // offset 2
-constexpr uint32_t kN132 = 0xC304C304u, kN68 = 0xC288C288u, kN36 = 0xC210C210u, kN20 = 0xC1A0C1A0u,
-                   kN12 = 0xC140C140u;                                                         // offset 4
+// ---- decode tables ---------------------------------------------------------
+// A decoded register holds the stored codes u of two codes as
+// bf16 u * 2^(p - 133): p is the field's bit position inside its 16-bit half
+// after masking.  The preparation kernel multiplies each activation by
+// 2^(133 - S - p) of the field its code lands in, and stores the activations
+// in the order the MMAs consume them.
+//
+// 2-bit word (16 codes k = 0..15, field m = codes 2m, 2m+1 at bits 2m and
+// 16+2m): fields 0..3 masked in place (p = 2m), fields 4..7 after >> 8
+// (p = 2m - 8).  MMA r of a word takes fields 2r, 2r+1 = codes 4r .. 4r+3,
+// natural order.
+__device__ __forceinline__ int pos_int2(int m) { return 2 * (m & 3); }
 
-__device__ __forceinline__ uint32_t dq_field(uint32_t v, uint32_t mask, uint32_t mul, uint32_t add) {
-    // (v & mask) | 128.0 = 128 + u * 2^q exactly; * 2^-q + add = c exactly
-    return hfma2_bf16(and_or(v, mask, kMag), mul, add);
-}
+// 3-bit block (32 codes, field m = codes 2m, 2m+1 = bit m / 16+m of each
+// plane).  Field positions after the decode below, and the two fields each
+// of the eight MMAs takes (A-operand k-slots 0-1 and 8-9 hold the first
+// field, 2-3 and 10-11... i.e. register a0/a1 = first field, a2/a3 = second).
+__constant__ int8_t kPosInt3[16] = {0, 1, 2, 3, 4, 5, 0, 1, 2, 3, 4, 5, 0, 1, 0, 1};
+__constant__ int8_t kMmaFieldInt3[8][2] = {{0, 1}, {3, 4}, {6, 7}, {9, 10}, {12, 13}, {2, 5}, {8, 11}, {14, 15}};
 
-// 2-bit word -> o[m] = bf16x2 (c[2m], c[2m+1]), m = 0..7
-__device__ __forceinline__ void dq_word2(uint32_t w, uint32_t (&o)[8]) {
-    const uint32_t w6 = w >> 6, w12 = w >> 12;
-    o[0] = dq_field(w, 0x00030003u, kOne, kN130);
-    o[1] = dq_field(w, 0x000C000Cu, kQuarter, kN34);
-    o[2] = dq_field(w, 0x00300030u, kSixteenth, kN10);
-    o[3] = dq_field(w6, 0x00030003u, kOne, kN130);
-    o[4] = dq_field(w6, 0x000C000Cu, kQuarter, kN34);
-    o[5] = dq_field(w6, 0x00300030u, kSixteenth, kN10);
-    o[6] = dq_field(w12, 0x00030003u, kOne, kN130);
-    o[7] = dq_field(w12, 0x000C000Cu, kQuarter, kN34);
-}
+__device__ __forceinline__ uint32_t shr_fma(uint32_t x, int k) { return __umulhi(x, 1u << (32 - k)); }
 
-// bit masks with bits set at positions s + {0, 3, 6, ...} in both halves
+// masks with a bit at first + 3i + shift (i < count) in both halves
 constexpr uint32_t bits_at(int first, int count, int shift) {
     uint32_t m = 0;
-    for (int i = 0; i < count; ++i) {
-        m |= 1u << (first + 3 * i + shift);
-        m |= 1u << (16 + first + 3 * i + shift);
-    }
+    for (int i = 0; i < count; ++i) m |= (1u << (first + 3 * i + shift)) | (1u << (16 + first + 3 * i + shift));
     return m;
 }
 
-// 3-bit block (planes p0, p1, p2) -> o[m] = bf16x2 (c[2m], c[2m+1]), m = 0..15.
-// Field m of the block is bit m of each plane (low half) and bit 16+m (high
-// half).  Shifting plane 1 left by 1 and plane 2 by 2 puts the three bits
-// of field m at m, m+1, m+2; a bit-select of the three planes assembles
-// every third field at once, and those fields are then cut out in pairs.
-__device__ __forceinline__ void dq_block3(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t (&o)[16]) {
-    const uint32_t q1 = p1 << 1, q2 = p2 << 2;
-    // fields m = 0, 3, 6, 9, 12
-    {
-        const uint32_t z = bit_mux(bit_mux(p0, q1, bits_at(0, 5, 1)), q2, bits_at(0, 5, 2));
-        const uint32_t z6 = z >> 6, z12 = z >> 12;
-        o[0] = dq_field(z, 0x00070007u, kOne, kN132);
-        o[3] = dq_field(z, 0x00380038u, kEighth, kN20);
-        o[6] = dq_field(z6, 0x00070007u, kOne, kN132);
-        o[9] = dq_field(z6, 0x00380038u, kEighth, kN20);
-        o[12] = dq_field(z12, 0x00070007u, kOne, kN132);
-    }
-    // fields m = 1, 4, 7, 10, 13
-    {
-        const uint32_t z = bit_mux(bit_mux(p0, q1, bits_at(1, 5, 1)), q2, bits_at(1, 5, 2));
-        const uint32_t z6 = z >> 6, z12 = z >> 12;
-        o[1] = dq_field(z, 0x000E000Eu, kHalf, kN68);
-        o[4] = dq_field(z, 0x00700070u, kSixteenth, kN12);
-        o[7] = dq_field(z6, 0x000E000Eu, kHalf, kN68);
-        o[10] = dq_field(z6, 0x00700070u, kSixteenth, kN12);
-        o[13] = dq_field(z12, 0x000E000Eu, kHalf, kN68);
-    }
-    // fields m = 2, 5, 8, 11
-    {
-        const uint32_t z = bit_mux(bit_mux(p0, q1, bits_at(2, 4, 1)), q2, bits_at(2, 4, 2));
-        const uint32_t z4 = z >> 4, z10 = z >> 10;
-        o[2] = dq_field(z, 0x001C001Cu, kQuarter, kN36);
-        o[5] = dq_field(z4, 0x000E000Eu, kHalf, kN68);
-        o[8] = dq_field(z4, 0x00700070u, kSixteenth, kN12);
-        o[11] = dq_field(z10, 0x000E000Eu, kHalf, kN68);
-    }
-    // fields m = 14, 15 (bits 14/15 and 30/31 of each plane)
-    {
-        const uint32_t r0 = p0 >> 14, r1 = p1 >> 13, r2 = p2 >> 12;
-        const uint32_t z14 = bit_mux(bit_mux(r0, r1, 0x00020002u), r2, 0x00040004u);
-        const uint32_t z15 = bit_mux(bit_mux(r0, r1, 0x00040004u), r2, 0x00080008u);
-        o[14] = dq_field(z14, 0x00070007u, kOne, kN132);
-        o[15] = dq_field(z15, 0x000E000Eu, kHalf, kN68);
-    }
+// d = A B (first MMA of a group: C is the constant zero, no re-zeroing of d)
+__device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "{\n .reg .f32 z;\n mov.f32 z, 0f00000000;\n"
+        " mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {z,z,z,z};\n}"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -135,179 +96,852 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Codes, scales of one 128-group for one lane (rows g and g + 8).
-struct Slot {
-    uint32_t a[3], b[3];  // 2-bit: words 2t, 2t+1 in a[0..1]; 3-bit: block t planes in a[0..2]
-    uint32_t sa, sb;      // bf16 scale bits, rows g and g + 8
-};
-
-template <int KIND>  // 0: 2-bit container, 1: 3-bit planes
-__device__ __forceinline__ void load_slot(Slot& s, const uint8_t* ra, const uint8_t* rb, const uint16_t* sa,
-                                          const uint16_t* sb, int64_t grp, int t) {
-    if (KIND == 0) {
-        const uint2 va = ld_stream_u2(ra + 32 * grp + 8 * t);
-        const uint2 vb = ld_stream_u2(rb + 32 * grp + 8 * t);
-        s.a[0] = va.x; s.a[1] = va.y; s.a[2] = 0;
-        s.b[0] = vb.x; s.b[1] = vb.y; s.b[2] = 0;
-    } else {
-        const uint8_t* pa = ra + 48 * grp + 12 * t;
-        const uint8_t* pb = rb + 48 * grp + 12 * t;
-#pragma unroll
-        for (int p = 0; p < 3; ++p) {
-            s.a[p] = ld_stream_u32(pa + 4 * p);
-            s.b[p] = ld_stream_u32(pb + 4 * p);
-        }
-    }
-    s.sa = ld_stream_u16(sa + grp);
-    s.sb = ld_stream_u16(sb + grp);
+// ---- cp.async (global -> shared, L1 bypass) ---------------------------------------
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-template <int KIND, int NT>
-__device__ __forceinline__ void compute_slot(const Slot& s, float (&acc)[NT][4], const uint16_t* const (&xr)[NT],
-                                             int64_t grp, int t) {
-    float d[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) d[nt][i] = 0.f;
-
-    if (KIND == 0) {
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            // x for codes 16*(2t+w) .. +15 of this group: two 16-byte loads per column tile
-            uint4 xv[NT][2];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const uint16_t* xp = xr[nt] + 128 * grp + 32 * t + 16 * w;
-                xv[nt][0] = ld_act_u4(xp);
-                xv[nt][1] = ld_act_u4(xp + 8);
-            }
-            uint32_t qa[8], qb[8];
-            dq_word2(s.a[w], qa);
-            dq_word2(s.b[w], qb);
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const uint4 v = xv[nt][r >> 1];
-                    const uint32_t b0 = (r & 1) ? v.z : v.x, b1 = (r & 1) ? v.w : v.y;
-                    mma16816(d[nt], qa[2 * r], qb[2 * r], qa[2 * r + 1], qb[2 * r + 1], b0, b1);
-                }
-            }
-        }
-    } else {
-        uint4 xv[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const uint16_t* xp = xr[nt] + 128 * grp + 32 * t;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) xv[nt][q] = ld_act_u4(xp + 8 * q);
-        }
-        uint32_t qa[16], qb[16];
-        dq_block3(s.a[0], s.a[1], s.a[2], qa);
-        dq_block3(s.b[0], s.b[1], s.b[2], qb);
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const uint4 v = xv[nt][r >> 1];
-                const uint32_t b0 = (r & 1) ? v.z : v.x, b1 = (r & 1) ? v.w : v.y;
-                mma16816(d[nt], qa[2 * r], qb[2 * r], qa[2 * r + 1], qb[2 * r + 1], b0, b1);
-            }
-        }
+// ---------------------------------------------------------------------------
+// Preparation: one warp per (item, activation row m, group g).
+__global__ void __launch_bounds__(kThreads) k_prep(const __grid_constant__ Launch L, int total_warps) {
+    pdl_trigger();  // the main kernel may start streaming weights now
+    const int wi = blockIdx.x * kWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (L.zero) {  // stream-K tile counters (the previous call may still use them: after the wait)
+        pdl_wait();
+        for (int i = blockIdx.x * kThreads + threadIdx.x; i < L.n_zero; i += gridDim.x * kThreads) L.zero[i] = 0;
     }
-    const float fa = bf16_bits_to_float(s.sa), fb = bf16_bits_to_float(s.sb);
+    if (wi >= total_warps) return;
+    int ii = 0;
+    for (int i = 1; i < L.n_items; ++i)
+        if (wi >= L.it[i].prep_begin) ii = i;
+    const Item& I = L.it[ii];
+    const int64_t K = I.K;
+    const int M = I.M, grid = I.grid;
+    const int64_t wl = wi - I.prep_begin;
+    const int64_t grp = wl / M;
+    const int m = (int)(wl - grp * M);
+    pdl_wait();  // x may be written by the previous kernel in the stream
+    const uint16_t* xg = I.X + m * I.ldx + grp * kGroup;
+    // group statistics over the natural order: lane holds x[4 lane .. 4 lane + 3]
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(xg + 4 * lane));
+    const uint32_t hv[4] = {raw.x & 0xFFFFu, raw.x >> 16, raw.y & 0xFFFFu, raw.y >> 16};
+    int e = 0;
+    float sum = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        acc[nt][0] = fmaf(fa, d[nt][0], acc[nt][0]);
-        acc[nt][1] = fmaf(fa, d[nt][1], acc[nt][1]);
-        acc[nt][2] = fmaf(fb, d[nt][2], acc[nt][2]);
-        acc[nt][3] = fmaf(fb, d[nt][3], acc[nt][3]);
+    for (int j = 0; j < 4; ++j) {
+        e = max(e, (int)((hv[j] >> 7) & 0xFFu));
+        sum += bf16_bits_to_float(hv[j]);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    // S = exponent of max|x| + 7 (a zero / subnormal group counts as 2^-126)
+    const int S = min(max(e, 1) - 127 + 7, 127);
+    // output slots 4 lane .. 4 lane + 3 of the group, in MMA order
+    uint32_t out[2] = {0, 0};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int o = 4 * lane + j;
+        int src, p;
+        if (grid == kInt3) {
+            const int ob = o & 31, r = ob >> 2, sl = ob & 3;
+            const int f = kMmaFieldInt3[r][sl >> 1];
+            src = (o & ~31) + 2 * f + (sl & 1);
+            p = kPosInt3[f];
+        } else {
+            src = o;
+            p = pos_int2((o & 15) >> 1);
+        }
+        const int sh = 133 - S - p;  // 1 .. 252: applied as two exact power-of-two factors
+        const int s1 = sh >> 1, s2 = sh - s1;
+        const float v = bf16_bits_to_float(xg[src]) * __int_as_float((s1 + 127) << 23) *
+                        __int_as_float((s2 + 127) << 23);
+        const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(v));  // exact: 8 significant bits
+        out[j >> 1] |= b << (16 * (j & 1));
+    }
+    *reinterpret_cast<uint2*>(I.xs + (int64_t)m * K + grp * kGroup + 4 * lane) = make_uint2(out[0], out[1]);
+    if (lane == 0) {
+        const float off = grid == kInt3 ? 4.f : 2.f;
+        I.cf[grp * M + m] = make_float2(off * sum, __int_as_float((S + 127) << 23));
     }
 }
 
-template <int KIND, int NT>
-__device__ __forceinline__ void run_tile(const Item& I, int64_t tile, float (*red)[NT * 4][32]) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int64_t N = I.N, K = I.K, G = K / kGroup;
-    const int64_t rowA = tile * 16 + g, rowB = rowA + 8;
-    const int64_t rA = rowA < N ? rowA : N - 1, rB = rowB < N ? rowB : N - 1;
-    const int64_t rbytes = KIND == 0 ? K / 4 : 3 * K / 8;
-    const uint8_t* pa = I.packed + rA * rbytes;
-    const uint8_t* pb = I.packed + rB * rbytes;
-    const uint16_t* sa = I.scales + rA * G;
-    const uint16_t* sb = I.scales + rB * G;
-    const uint16_t* xr[NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int col = nt * 8 + g;
-        xr[nt] = I.X + (int64_t)(col < I.M ? col : I.M - 1) * I.ldx;
-    }
-
-    float acc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-
-    // this warp's groups: warp, warp + 8, warp + 16, ...
-    const int64_t ng = G > warp ? (G - warp + kWarps - 1) / kWarps : 0;
-    Slot buf[kPF];
-#pragma unroll
-    for (int i = 0; i < kPF; ++i)
-        if (i < ng) load_slot<KIND>(buf[i], pa, pb, sa, sb, warp + (int64_t)kWarps * i, t);
-    for (int64_t base = 0; base < ng; base += kPF) {
-#pragma unroll
-        for (int i = 0; i < kPF; ++i) {
-            const int64_t step = base + i;
-            if (step < ng) {
-                const Slot cur = buf[i];
-                if (step + kPF < ng) load_slot<KIND>(buf[i], pa, pb, sa, sb, warp + kWarps * (step + kPF), t);
-                compute_slot<KIND, NT>(cur, acc, xr, warp + kWarps * step, t);
-            }
-        }
-    }
-
-    // cross-warp reduction in a fixed order
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) red[warp][nt * 4 + i][lane] = acc[nt][i];
-    __syncthreads();
-    for (int e = threadIdx.x; e < NT * 4 * 32; e += kThreads) {
-        const int nt = e / 128, i = (e / 32) & 3, ln = e & 31;
-        const int64_t row = tile * 16 + (ln >> 2) + ((i >> 1) ? 8 : 0);
-        const int col = nt * 8 + 2 * (ln & 3) + (i & 1);
-        if (row < N && col < I.M) {
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) v += red[w][nt * 4 + i][ln];
-            if (I.ydt == kF32) static_cast<float*>(I.Y)[(int64_t)col * I.ldy + row] = v;
-            else static_cast<__nv_bfloat16*>(I.Y)[(int64_t)col * I.ldy + row] = __float2bfloat16_rn(v);
-        }
-    }
-}
+// ---------------------------------------------------------------------------
+// Main kernel.
+//
+// A warp owns a 32-row tile (two 16-row MMA tiles sharing every activation
+// fragment) and a contiguous range of 128-groups of K; the item's ksplit (S)
+// warps of a tile cover K and reduce in shared memory.  Shared memory per
+// CTA: a ring of kStages group stages per warp (32 rows x one group of
+// packed codes: 1 KB for 2 bits, 1.5 KB for 3), the warp's scales for its
+// whole group range, and the cross-warp reduction buffer.
+constexpr int kStages = 4;
+constexpr int kStageBytes = 1536;
+constexpr int kRingBytes = kWarps * kStages * kStageBytes;
+constexpr int kRows = 32;  // rows per warp tile
 
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 2) k_linear(const __grid_constant__ Launch L) {
-    __shared__ float red[kWarps][NT * 4][32];
+struct Cols {
+    const uint16_t* xs[NT];   // prepared activations of column 8 nt + g, at 32 t of group gb
+    const float2* cf[NT][2];  // (offset * sum, 2^S) of columns 8 nt + 2t, + 1, at group gb
+};
+
+template <int NT>
+__device__ __forceinline__ void mma_tiles(float (&d)[2][NT][4], const uint32_t (&a)[2][4], const uint4 (&xv)[NT],
+                                          bool hi) {
+#pragma unroll
+    for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+            mma16816(d[rt][nt], a[rt][0], a[rt][1], a[rt][2], a[rt][3], hi ? xv[nt].z : xv[nt].x,
+                     hi ? xv[nt].w : xv[nt].y);
+}
+
+// One 128-group: decode the lane's codes of rows g, g+8 (MMA tile 0) and
+// g+16, g+24 (MMA tile 1) from the stage, run the MMAs, scale, accumulate.
+template <int KIND, int NT, bool M1>
+__device__ __forceinline__ void group_step(const uint8_t* stage, int g, int t, const uint16_t* const (&xs)[NT],
+                                           const float2* const (&cf)[NT][2], const float (&sc)[4],
+                                           float (&acc)[2][NT][4]) {
+    float d[2][NT][4];
+#pragma unroll
+    for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) d[rt][nt][0] = d[rt][nt][1] = d[rt][nt][2] = d[rt][nt][3] = 0.f;
+    if (KIND == 0) {
+        uint2 wv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) wv[q] = *reinterpret_cast<const uint2*>(stage + (g + 8 * q) * 32 + 8 * t);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            uint4 xv[2][NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                xv[0][nt] = ld_act_u4(xs[nt] + 16 * w);
+                xv[1][nt] = ld_act_u4(xs[nt] + 16 * w + 8);
+            }
+            uint32_t W[4], H[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                W[q] = w ? wv[q].y : wv[q].x;
+                H[q] = shr_fma(W[q], 8);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                // fields 2r, 2r+1: r < 2 in place, r >= 2 from the >> 8 copy
+                const uint32_t m0 = 0x00030003u << (4 * (r & 1)), m1 = 0x000C000Cu << (4 * (r & 1));
+                uint32_t a[2][4];
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt) {
+                    const uint32_t A = r < 2 ? W[2 * rt] : H[2 * rt], B = r < 2 ? W[2 * rt + 1] : H[2 * rt + 1];
+                    a[rt][0] = A & m0;
+                    a[rt][1] = B & m0;
+                    a[rt][2] = A & m1;
+                    a[rt][3] = B & m1;
+                }
+                mma_tiles<NT>(d, a, xv[r >> 1], r & 1);
+            }
+        }
+    } else {
+        uint32_t P[4][3];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+                P[q][p] = *reinterpret_cast<const uint32_t*>(stage + (g + 8 * q) * 48 + 12 * t + 4 * p);
+        uint4 xv[4][NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) xv[q][nt] = ld_act_u4(xs[nt] + 8 * q);
+        // planes 1 and 2 shifted left by 1 and 2: field m's three bits at m, m+1, m+2
+        uint32_t q1[4], q2[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            q1[q] = P[q][1] << 1;
+            q2[q] = P[q][2] << 2;
+        }
+        uint32_t zA[4], zB[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // sets A (fields 0,3,6,9,12) and B (1,4,7,10,13)
+            zA[q] = bit_mux(bit_mux(P[q][0], q1[q], bits_at(0, 5, 1)), q2[q], bits_at(0, 5, 2));
+            zB[q] = bit_mux(bit_mux(P[q][0], q1[q], bits_at(1, 5, 1)), q2[q], bits_at(1, 5, 2));
+        }
+        auto emit = [&](int r, const uint32_t (&fa)[4], uint32_t ma, const uint32_t (&fb)[4], uint32_t mb) {
+            uint32_t a[2][4];
+#pragma unroll
+            for (int rt = 0; rt < 2; ++rt) {
+                a[rt][0] = fa[2 * rt] & ma;
+                a[rt][1] = fa[2 * rt + 1] & ma;
+                a[rt][2] = fb[2 * rt] & mb;
+                a[rt][3] = fb[2 * rt + 1] & mb;
+            }
+            mma_tiles<NT>(d, a, xv[r >> 1], r & 1);
+        };
+        emit(0, zA, 0x00070007u, zB, 0x000E000Eu);
+        emit(1, zA, 0x00380038u, zB, 0x00700070u);
+        uint32_t s6A[4], s6B[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            s6A[q] = shr_fma(zA[q], 6);
+            s6B[q] = shr_fma(zB[q], 6);
+        }
+        emit(2, s6A, 0x00070007u, s6B, 0x000E000Eu);
+        emit(3, s6A, 0x00380038u, s6B, 0x00700070u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            s6A[q] = shr_fma(zA[q], 12);
+            s6B[q] = shr_fma(zB[q], 12);
+        }
+        emit(4, s6A, 0x00070007u, s6B, 0x000E000Eu);
+        uint32_t zC[4], zC6[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // set C (fields 2,5,8,11)
+            zC[q] = bit_mux(bit_mux(P[q][0], q1[q], bits_at(2, 4, 1)), q2[q], bits_at(2, 4, 2));
+            zC6[q] = shr_fma(zC[q], 6);
+        }
+        emit(5, zC, 0x001C001Cu, zC, 0x00E000E0u);
+        emit(6, zC6, 0x001C001Cu, zC6, 0x00E000E0u);
+        // fields 14, 15 use plane bits 14/15 and 30/31, which the left shifts push out of the word:
+        // realign the raw planes to the right instead, plane p by 14 - p, so plane p of field 14
+        // lands at bit p (and 16 + p), of field 15 at bit p + 1 (and 17 + p)
+        uint32_t z14[4], z15[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t r0 = shr_fma(P[q][0], 14), r1 = shr_fma(P[q][1], 13), r2 = shr_fma(P[q][2], 12);
+            z14[q] = bit_mux(bit_mux(r0, r1, 0x00020002u), r2, 0x00040004u);
+            z15[q] = bit_mux(bit_mux(r0, r1, 0x00040004u), r2, 0x00080008u);
+        }
+        emit(7, z14, 0x00070007u, z15, 0x000E000Eu);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const float2 c0 = ld_act_f2(cf[nt][0]);
+        const float2 c1 = M1 ? c0 : ld_act_f2(cf[nt][1]);
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt) {
+            acc[rt][nt][0] = fmaf(sc[2 * rt], fmaf(c0.y, d[rt][nt][0], -c0.x), acc[rt][nt][0]);
+            acc[rt][nt][2] = fmaf(sc[2 * rt + 1], fmaf(c0.y, d[rt][nt][2], -c0.x), acc[rt][nt][2]);
+            if (!M1) {
+                acc[rt][nt][1] = fmaf(sc[2 * rt], fmaf(c1.y, d[rt][nt][1], -c1.x), acc[rt][nt][1]);
+                acc[rt][nt][3] = fmaf(sc[2 * rt + 1], fmaf(c1.y, d[rt][nt][3], -c1.x), acc[rt][nt][3]);
+            }
+        }
+    }
+}
+
+template <int KIND, int NT, bool M1>
+__device__ __forceinline__ void run_tile(const Item& I, int64_t cta_local, int scl_stride, uint8_t* smem) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int S = I.ksplit;
+    const int tl = warp / S, ks = warp - tl * S;
+    const int64_t N = I.N, K = I.K, G = K / kGroup;
+    const int M = I.M;
+    const int64_t row0 = (cta_local * (kWarps / S) + tl) * kRows;
+    const bool active = row0 < N;
+    constexpr int RB = KIND == 0 ? 32 : 48;  // bytes of one row in one group
+    const int64_t rbytes = KIND == 0 ? K / 4 : 3 * K / 8;
+    const int64_t gb = G * ks / S, ge = G * (ks + 1) / S;
+    const int ng = active ? (int)(ge - gb) : 0;
+
+    uint8_t* ring = smem + warp * (kStages * kStageBytes);
+    uint16_t* scl = reinterpret_cast<uint16_t*>(smem + kRingBytes) + warp * kRows * scl_stride;
+    float* red = reinterpret_cast<float*>(smem + kRingBytes + kWarps * kRows * scl_stride * 2);
+
+    // --- copies: the stage is kRows rows x RB bytes = (2 or 3) 16-byte chunks per lane;
+    //     chunk c = lane + 32 i goes to row c / (RB/16), part c % (RB/16)
+    constexpr int NCH = KIND == 0 ? 2 : 3;
+    const uint8_t* src[NCH];
+    uint32_t dst[NCH];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+        const int c = lane + 32 * i, r = c / (RB / 16), part = c % (RB / 16);
+        const int64_t row = min(row0 + r, N - 1);
+        src[i] = I.packed + row * rbytes + gb * RB + 16 * part;
+        dst[i] = r * RB + 16 * part;
+    }
+    const uint32_t ring_s = smem_u32(ring);
+    int issued = 0;
+    auto issue = [&]() {  // copies of the warp's next group into stage issued % kStages
+        if (issued < ng) {
+            const uint32_t st = ring_s + (issued & (kStages - 1)) * kStageBytes;
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) cp_async16(st + dst[i], src[i] + (int64_t)issued * RB);
+        }
+        ++issued;
+        cp_commit();
+    };
+#pragma unroll
+    for (int j = 0; j < kStages - 1; ++j) issue();
+
+    // --- this warp's scales, all groups of its range: lane r stages row r (row r, group j at
+    //     scl[r * stride + j]; stride = 2 mod 4 keeps the 32 rows in distinct banks)
+    {
+        const uint16_t* sp = I.scales + min(row0 + lane, N - 1) * G + gb;
+        for (int j = 0; j < ng; ++j) scl[lane * scl_stride + j] = ld_stream_u16(sp + j);
+    }
+
+    const uint16_t* xs[NT];
+    const float2* cf[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int colB = nt * 8 + g, c0 = nt * 8 + 2 * t;
+        xs[nt] = I.xs + (int64_t)(colB < M ? colB : M - 1) * K + 32 * t + gb * kGroup;
+        cf[nt][0] = I.cf + (c0 < M ? c0 : M - 1) + gb * M;
+        cf[nt][1] = I.cf + (c0 + 1 < M ? c0 + 1 : M - 1) + gb * M;
+    }
+    float acc[2][NT][4];
+#pragma unroll
+    for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[rt][nt][0] = acc[rt][nt][1] = acc[rt][nt][2] = acc[rt][nt][3] = 0.f;
+
+    pdl_wait();  // prepared activations are ready past this point
+#pragma unroll 1
+    for (int j = 0; j < ng; ++j) {
+        cp_wait<kStages - 2>();
+        __syncwarp();  // every lane's copies of this stage (and the scales) are visible
+        const uint8_t* stage = ring + (j & (kStages - 1)) * kStageBytes;
+        float sc[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sc[q] = bf16_bits_to_float(scl[(g + 8 * q) * scl_stride + j]);
+        issue();  // refills the stage read in step j - 1 (every lane is past it)
+        group_step<KIND, NT, M1>(stage, g, t, xs, cf, sc, acc);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            xs[nt] += kGroup;
+            cf[nt][0] += M;
+            cf[nt][1] += M;
+        }
+    }
+    cp_wait<0>();
+
+    constexpr int NV = 2 * NT * 4;  // accumulators per lane
+    if (S > 1) {
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) red[(warp * NV + (rt * NT + nt) * 4 + i) * 32 + lane] = acc[rt][nt][i];
+        __syncthreads();
+        if (ks != 0 || !active) return;
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float v = acc[rt][nt][i];
+                    for (int s2 = 1; s2 < S; ++s2) v += red[((warp + s2) * NV + (rt * NT + nt) * 4 + i) * 32 + lane];
+                    acc[rt][nt][i] = v;
+                }
+    } else if (!active) {
+        return;
+    }
+#pragma unroll
+    for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int64_t row = row0 + 16 * rt + g + ((i >> 1) ? 8 : 0);
+                const int col = nt * 8 + 2 * t + (i & 1);
+                if (row < N && col < M && (!M1 || col == 0)) {
+                    const float v = acc[rt][nt][i];
+                    if (I.ydt == kF32) static_cast<float*>(I.Y)[(int64_t)col * I.ldy + row] = v;
+                    else static_cast<__nv_bfloat16*>(I.Y)[(int64_t)col * I.ldy + row] = __float2bfloat16_rn(v);
+                }
+            }
+}
+
+template <int NT, bool M1>
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2) k_linear(const __grid_constant__ Launch L) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    // Every CTA of this grid is resident once all have passed this point, so
+    // a dependent launch (the next overlapped call) cannot starve it.
+    pdl_trigger();
     const int u = blockIdx.x;
     int ii = 0;
     for (int i = 1; i < L.n_items; ++i)
-        if (u >= L.it[i].unit_begin) ii = i;
+        if (u >= L.it[i].cta_begin) ii = i;
     const Item& I = L.it[ii];
-    const int64_t tile = u - I.unit_begin;
-    if (I.grid == kInt3) run_tile<1, NT>(I, tile, red);
-    else run_tile<0, NT>(I, tile, red);
+    if (I.grid == kInt3) run_tile<1, NT, M1>(I, u - I.cta_begin, L.scl_stride, smem);
+    else run_tile<0, NT, M1>(I, u - I.cta_begin, L.scl_stride, smem);
+}
+
+// ---------------------------------------------------------------------------
+// Stream-K batch-1 kernel.
+//
+// Persistent warps, one contiguous equal-cost range of tile-groups each
+// (tb_partition.h), across tile and item boundaries: the cp.async ring never
+// drains at a tile boundary.  A tile whose K the warp covers entirely is
+// written directly; a tile shared by several warps is combined by the last
+// of them to finish (per-tile arrival counter), which adds the partial sums
+// in warp order, so the result does not depend on timing.
+#ifndef TB_SK_STAGES
+#define TB_SK_STAGES 4
+#endif
+constexpr int kSKStages = TB_SK_STAGES;  // ring depth: kSKStages - 1 groups in flight per warp
+
+// Per-warp shared memory: kSKStages stages, each the weights of one
+// tile-group (32 rows x 32 or 48 bytes), its prepared activations (128 bf16,
+// stored as two 128-byte halves 16 bytes apart so the four t-lanes of an
+// LDS.128 hit distinct banks) and the 16-byte chunk holding its
+// (offset * sum x, 2^S) pair.
+constexpr int kSKW = 1536;               // weights
+constexpr int kSKX = kSKW;               // activations: 272 bytes
+constexpr int kSKC = kSKX + 272;         // (sum, 2^S) chunk: 16 bytes
+constexpr int kSKStageB = kSKC + 16;     // 1824
+constexpr int kSKWarpB = kSKStages * kSKStageB;
+
+// ---- per-step helpers -----------------------------------------------------------
+__device__ __forceinline__ uint32_t sk_xs_dst(int c) { return 16 * c + (c >= 8 ? 16 : 0); }
+
+// One 128-group of the 32-row tile from a stage: decode, MMAs, scale, accumulate
+// (batch 1: the prepared activations and the (sum, 2^S) pair come from the stage).
+// cofs: byte offset of this group's (sum, 2^S) pair inside the 16-byte chunk (8 for odd groups);
+// srow: bf16 scale of row `lane` (shuffled to rows g, g+8, g+16, g+24 only at the end, so the load
+// behind it has the whole step to land)
+template <int KIND>
+__device__ __forceinline__ void sk_step(const uint8_t* stage, uint32_t srow, int cofs, int g, int t,
+                                        float (&acc)[4]) {
+    float d[2][4];
+    bool first = true;  // the first MMA of each chain starts from zero
+    auto mma = [&](int rt, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+        if (first) mma16816_z(d[rt], a0, a1, a2, a3, b0, b1);
+        else mma16816(d[rt], a0, a1, a2, a3, b0, b1);
+    };
+    // B fragment for codes 32 t + 8 q .. + 7 of the group
+    auto xfrag = [&](int q) {
+        const int c = 4 * t + q;  // 16-byte chunk of the 256-byte activation slice
+        return *reinterpret_cast<const uint4*>(stage + kSKX + sk_xs_dst(c));
+    };
+    if (KIND == 0) {
+        uint2 wv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) wv[q] = *reinterpret_cast<const uint2*>(stage + (g + 8 * q) * 32 + 8 * t);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            const uint4 xv0 = xfrag(2 * w), xv1 = xfrag(2 * w + 1);
+            uint32_t W[4], H[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                W[q] = w ? wv[q].y : wv[q].x;
+                H[q] = shr_fma(W[q], 8);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t m0 = 0x00030003u << (4 * (r & 1)), m1 = 0x000C000Cu << (4 * (r & 1));
+                const uint4 v = (r >> 1) ? xv1 : xv0;
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt) {
+                    const uint32_t A = r < 2 ? W[2 * rt] : H[2 * rt], B = r < 2 ? W[2 * rt + 1] : H[2 * rt + 1];
+                    mma(rt, A & m0, B & m0, A & m1, B & m1, (r & 1) ? v.z : v.x, (r & 1) ? v.w : v.y);
+                }
+                first = false;
+            }
+        }
+    } else {
+        uint4 xv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xv[q] = xfrag(q);
+        // the two 16-row MMA tiles one after the other (keeps the live decode state small)
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt) {
+            uint32_t P[2][3];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int p = 0; p < 3; ++p)
+                    P[h][p] = *reinterpret_cast<const uint32_t*>(stage + (g + 8 * (2 * rt + h)) * 48 + 12 * t + 4 * p);
+            uint32_t q1[2], q2[2], zA[2], zB[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                q1[h] = P[h][1] << 1;
+                q2[h] = P[h][2] << 2;
+                zA[h] = bit_mux(bit_mux(P[h][0], q1[h], bits_at(0, 5, 1)), q2[h], bits_at(0, 5, 2));
+                zB[h] = bit_mux(bit_mux(P[h][0], q1[h], bits_at(1, 5, 1)), q2[h], bits_at(1, 5, 2));
+            }
+            bool first3 = true;
+            auto emit = [&](int r, const uint32_t (&fa)[2], uint32_t ma, const uint32_t (&fb)[2], uint32_t mb) {
+                const uint4 v = xv[r >> 1];
+                if (first3) mma16816_z(d[rt], fa[0] & ma, fa[1] & ma, fb[0] & mb, fb[1] & mb, (r & 1) ? v.z : v.x,
+                                       (r & 1) ? v.w : v.y);
+                else mma16816(d[rt], fa[0] & ma, fa[1] & ma, fb[0] & mb, fb[1] & mb, (r & 1) ? v.z : v.x,
+                              (r & 1) ? v.w : v.y);
+                first3 = false;
+            };
+            emit(0, zA, 0x00070007u, zB, 0x000E000Eu);
+            emit(1, zA, 0x00380038u, zB, 0x00700070u);
+            uint32_t sA[2], sB[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                sA[h] = shr_fma(zA[h], 6);
+                sB[h] = shr_fma(zB[h], 6);
+            }
+            emit(2, sA, 0x00070007u, sB, 0x000E000Eu);
+            emit(3, sA, 0x00380038u, sB, 0x00700070u);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                sA[h] = shr_fma(zA[h], 12);
+                sB[h] = shr_fma(zB[h], 12);
+            }
+            emit(4, sA, 0x00070007u, sB, 0x000E000Eu);
+            uint32_t zC[2], zC6[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                zC[h] = bit_mux(bit_mux(P[h][0], q1[h], bits_at(2, 4, 1)), q2[h], bits_at(2, 4, 2));
+                zC6[h] = shr_fma(zC[h], 6);
+            }
+            emit(5, zC, 0x001C001Cu, zC, 0x00E000E0u);
+            emit(6, zC6, 0x001C001Cu, zC6, 0x00E000E0u);
+            // fields 14, 15 (plane bits 14/15, 30/31) from the raw planes, plane p realigned right
+            // by 14 - p: plane p of field 14 lands at bit p (16 + p), of field 15 at bit p + 1
+            uint32_t z14[2], z15[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t r0 = shr_fma(P[h][0], 14), r1 = shr_fma(P[h][1], 13), r2 = shr_fma(P[h][2], 12);
+                z14[h] = bit_mux(bit_mux(r0, r1, 0x00020002u), r2, 0x00040004u);
+                z15[h] = bit_mux(bit_mux(r0, r1, 0x00040004u), r2, 0x00080008u);
+            }
+            emit(7, z14, 0x00070007u, z15, 0x000E000Eu);
+        }
+    }
+    const float2 c = *reinterpret_cast<const float2*>(stage + kSKC + cofs);
+    float sc[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) sc[q] = bf16_bits_to_float(__shfl_sync(0xffffffffu, srow, g + 8 * q));
+#pragma unroll
+    for (int rt = 0; rt < 2; ++rt) {
+        acc[2 * rt] = fmaf(sc[2 * rt], fmaf(c.y, d[rt][0], -c.x), acc[2 * rt]);
+        acc[2 * rt + 1] = fmaf(sc[2 * rt + 1], fmaf(c.y, d[rt][2], -c.x), acc[2 * rt + 1]);
+    }
+}
+
+__device__ __forceinline__ void cp_async16_if(uint32_t dst, const void* src, bool p) {
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.b32 q, %2, 0;\n @q cp.async.cg.shared.global [%0], [%1], 16;\n}" ::"r"(dst),
+        "l"(src), "r"((int)p)
+        : "memory");
+}
+
+// End of a segment [seg_grp, end_grp) of a tile: write y, or hand the
+// partial sums over and combine them if this warp arrives last.
+//   item: index into L.it; part: the partition the item belongs to;
+//   wg: this warp's index in the launch.
+__device__ __noinline__ void sk_flush(const SKLaunch& L, int part, int64_t wg, int item, uint32_t tile,
+                                      int32_t seg_grp, int32_t end_grp, bool first_seg, float v0, float v1, float v2,
+                                      float v3) {
+    const SKItem& I = L.it[item];
+    const SKPart& P = L.part[part];
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int64_t row0 = (int64_t)tile * kRows;
+    const float v[4] = {v0, v1, v2, v3};
+    if (seg_grp == 0 && end_grp == I.G) {
+        if (t == 0) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t row = row0 + g + 8 * q;
+                if (row < I.N) {
+                    if (I.ydt == kF32) static_cast<float*>(I.Y)[row] = v[q];
+                    else static_cast<__nv_bfloat16*>(I.Y)[row] = __float2bfloat16_rn(v[q]);
+                }
+            }
+        }
+        return;
+    }
+    float* mine = L.partials + (wg * 2 + (first_seg ? 0 : 1)) * kRows;
+    if (t == 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) __stcg(mine + g + 8 * q, v[q]);
+    }
+    __threadfence();
+    __syncwarp();
+    // contributors of this tile: the owners of its first and last tile-group (within the partition)
+    const uint32_t A = (uint32_t)I.tg_base + tile * (uint32_t)I.G;
+    const uint32_t pA = (uint32_t)I.cost_base + (A - (uint32_t)I.tg_base) * (uint32_t)I.unit_cost;
+    const uint32_t w0 = part_owner(pA, P.Q), w1 = part_owner(pA + (uint32_t)(I.G - 1) * I.unit_cost, P.Q);
+    int last = 0;
+    if (lane == 0) last = atomicAdd(L.counters + I.tile_base + tile, 1) == (int)(w1 - w0);
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
+    __threadfence();
+    float sum = 0.f;
+    for (uint32_t w = w0; w <= w1; ++w) {
+        // a warp that starts inside this tile has it as its first segment (slot 0), an earlier one
+        // as its last (slot 1)
+        const uint32_t wb = part_first_tg(L.it + P.first, P.count, w * P.Q);
+        sum += __ldcg(L.partials + ((int64_t)(P.W0 + w) * 2 + (wb >= A ? 0 : 1)) * kRows + lane);
+    }
+    const int64_t row = row0 + lane;
+    if (row < I.N) {
+        if (I.ydt == kF32) static_cast<float*>(I.Y)[row] = sum;
+        else static_cast<__nv_bfloat16*>(I.Y)[row] = __float2bfloat16_rn(sum);
+    }
+}
+
+// One warp of the stream-K kernel for code width KIND (0: 2-bit, 1: 3-bit).
+template <int KIND>
+__device__ __forceinline__ void sk_warp(const SKLaunch& L, int part, uint32_t w, int64_t wg, uint8_t* base) {
+    constexpr int RB = KIND ? 48 : 32;  // bytes of one row in one group
+    constexpr int NCH = KIND ? 3 : 2;   // 16-byte chunks per lane per stage
+    const SKPart& P = L.part[part];
+    const SKItem* items = L.it + P.first;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    uint32_t tb, te;
+    part_range(items, P.count, w, P.Q, P.C, &tb, &te);
+    if (tb >= te) return;
+    const int32_t nsteps = (int32_t)(te - tb);
+
+    const uint32_t base_s = smem_u32(base);
+
+    // ---- locate the first tile-group
+    int c_item = 0;
+    for (int i = 1; i < P.count; ++i)
+        if (tb >= (uint32_t)items[i].tg_base) c_item = i;
+    uint32_t c_tile;
+    int32_t c_grp;
+    {
+        const uint32_t local = tb - (uint32_t)items[c_item].tg_base, G = (uint32_t)items[c_item].G;
+        c_tile = local / G;
+        c_grp = (int32_t)(local - c_tile * G);
+    }
+
+    // ---- issue cursor and this lane's copy sources
+    int i_item = c_item;
+    uint32_t i_tile = c_tile;
+    int32_t i_grp = c_grp, i_G = items[c_item].G;
+    const uint8_t* wsrc[NCH];
+    const uint16_t* i_sp;
+    const uint16_t* i_xs;
+    const float2* i_cf;
+    auto set_tile = [&](int item, uint32_t tile, int32_t grp) {
+        const SKItem& I = items[item];
+        const int64_t row0 = (int64_t)tile * kRows, nm1 = I.N - 1;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int c = lane + 32 * i, r = KIND ? c / 3 : c >> 1, pp = KIND ? c - 3 * r : c & 1;
+            wsrc[i] = I.packed + min(row0 + r, nm1) * I.rbytes + (int64_t)grp * RB + 16 * pp;
+        }
+        i_sp = I.scales + min(row0 + lane, nm1) * I.G + grp;
+        i_xs = I.xs + (int64_t)grp * kGroup + 8 * (lane & 15);
+        i_cf = I.cf + (grp & ~1);
+        i_G = I.G;
+    };
+    set_tile(i_item, i_tile, i_grp);
+    auto advance_issue = [&]() {
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) wsrc[i] += RB;
+        ++i_sp;
+        i_xs += kGroup;
+        i_cf += (i_grp & 1) ? 2 : 0;
+        if (++i_grp == i_G) {
+            i_grp = 0;
+            if (++i_tile == (uint32_t)items[i_item].T) {
+                i_tile = 0;
+                ++i_item;
+            }
+            if (i_item < P.count) set_tile(i_item, i_tile, 0);
+        }
+    };
+    auto issue_weights = [&](uint32_t st) {
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) cp_async16(st + 512 * i + 16 * lane, wsrc[i]);
+    };
+    auto issue_acts = [&](uint32_t st, const uint16_t* xs, const float2* cf) {
+        cp_async16_if(st + kSKX + sk_xs_dst(lane & 15), xs, lane < 16);
+        cp_async16_if(st + kSKC, cf, lane == 16);
+    };
+
+    // ---- prologue: weights and scales of the first steps before waiting for the preparation
+    //      kernel, their activation copies after it (one commit group per step).  Scales ride in
+    //      a register ring, one per stage: this lane's row, loaded kSKStages - 1 steps ahead.
+    uint32_t sring[kSKStages];
+    const uint16_t* pro_xs[kSKStages - 1];
+    const float2* pro_cf[kSKStages - 1];
+#pragma unroll
+    for (int k = 0; k < kSKStages - 1; ++k) {
+        if (k < nsteps) {
+            issue_weights(base_s + k * kSKStageB);
+            sring[k] = __ldg(i_sp);
+            pro_xs[k] = i_xs;
+            pro_cf[k] = i_cf;
+            advance_issue();
+        }
+    }
+    pdl_wait();  // prepared activations and zeroed tile counters are ready past this point
+#pragma unroll
+    for (int k = 0; k < kSKStages - 1; ++k) {
+        if (k < nsteps) issue_acts(base_s + k * kSKStageB, pro_xs[k], pro_cf[k]);
+        cp_commit();
+    }
+
+    // ---- main loop, unrolled by the ring size so every stage offset is a constant
+    int32_t c_G = items[c_item].G, seg_grp = c_grp;
+    bool first_seg = true;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int32_t j0 = 0; j0 < nsteps; j0 += kSKStages) {
+#pragma unroll
+        for (int u = 0; u < kSKStages; ++u) {
+            const int32_t j = j0 + u;
+            if (j < nsteps) {
+                cp_wait<kSKStages - 2>();
+                __syncwarp();  // stage u (every lane's copies) is visible
+                const uint32_t srow = sring[u];
+                if (j + kSKStages - 1 < nsteps) {
+                    const uint32_t st = base_s + ((u + kSKStages - 1) % kSKStages) * kSKStageB;
+                    issue_weights(st);
+                    issue_acts(st, i_xs, i_cf);
+                    sring[(u + kSKStages - 1) % kSKStages] = __ldg(i_sp);
+                    advance_issue();
+                }
+                cp_commit();
+                sk_step<KIND>(base + u * kSKStageB, srow, (c_grp & 1) * 8, g, t, acc);
+                ++c_grp;
+                const bool more = j + 1 < nsteps;
+                if (c_grp == c_G || !more) {
+                    sk_flush(L, part, wg, P.first + c_item, c_tile, seg_grp, c_grp, first_seg, acc[0], acc[1], acc[2],
+                             acc[3]);
+                    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+                    first_seg = false;
+                    seg_grp = c_grp = 0;
+                    if (more) {
+                        if (++c_tile == (uint32_t)items[c_item].T) {
+                            c_tile = 0;
+                            ++c_item;
+                        }
+                        c_G = items[c_item].G;
+                    }
+                }
+            }
+        }
+    }
+    cp_wait<0>();
+}
+
+__global__ void __launch_bounds__(kThreads, 2) k_gemv_sk(const __grid_constant__ SKLaunch L) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5;
+    const int64_t wg = (int64_t)blockIdx.x * kWarps + warp;
+    if (wg >= L.W) return;  // whole warps; the kernel has no CTA-wide barrier
+    uint8_t* base = smem + warp * kSKWarpB;
+    if (wg < L.part[0].W0 + L.part[0].W) sk_warp<1>(L, 0, (uint32_t)(wg - L.part[0].W0), wg, base);
+    else sk_warp<0>(L, 1, (uint32_t)(wg - L.part[1].W0), wg, base);
+}
+
+size_t gemv_sk_smem_bytes() { return (size_t)kWarps * kSKWarpB; }
+
+bool sk_prepare_device(int dev) {
+    static bool ready[64] = {false};
+    if (dev < 0 || dev >= 64) return false;
+    if (!ready[dev]) {
+        if (cudaFuncSetAttribute((const void*)k_gemv_sk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gemv_sk_smem_bytes()) != cudaSuccess)
+            return false;
+        ready[dev] = true;
+    }
+    return true;
+}
+
+cudaError_t launch_pdl(const void* fn, void** args, unsigned grid, size_t smem, cudaStream_t st, bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+// The dynamic shared memory limit is raised once per device and kernel (to
+// the largest size any launch may ask for), so that later launches, including
+// ones recorded into a CUDA graph, make no attribute calls.
+template <int NT, bool M1>
+cudaError_t launch_main(const Launch& L, int ctas, size_t smem, cudaStream_t st) {
+    const void* fn = (const void*)k_linear<NT, M1>;
+    static bool ready[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !ready[dev]) {
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) ready[dev] = true;
+    }
+    void* args[] = {const_cast<Launch*>(&L)};
+    return launch_pdl(fn, args, (unsigned)ctas, smem, st, true);
 }
 
 }  // namespace
 
-cudaError_t launch_linear(const Launch& L, int nt, int ctas, cudaStream_t st) {
-    if (nt == 1) k_linear<1><<<ctas, kThreads, 0, st>>>(L);
-    else k_linear<2><<<ctas, kThreads, 0, st>>>(L);
-    return cudaGetLastError();
+cudaError_t launch_gemv_sk(const Launch& P, int prep_warps, const SKLaunch& L, int ctas, bool overlap,
+                           cudaStream_t st) {
+    {
+        void* args[] = {const_cast<Launch*>(&P), &prep_warps};
+        cudaError_t e = launch_pdl((const void*)k_prep, args,
+                                   (unsigned)std::max((prep_warps + kWarps - 1) / kWarps, 1), 0, st, overlap);
+        if (e != cudaSuccess) return e;
+    }
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!sk_prepare_device(dev)) return cudaErrorInvalidDevice;
+    void* args[] = {const_cast<SKLaunch*>(&L)};
+    return launch_pdl((const void*)k_gemv_sk, args, (unsigned)ctas, gemv_sk_smem_bytes(), st, true);
+}
+
+// Warps of the stream-K kernel that are resident at once on the current
+// device (its grid is sized to exactly this, so every warp runs from the
+// start: the partition is only balanced if no warp waits for a slot).
+int gemv_sk_resident_warps() {
+    static int warps[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (warps[dev] == 0) {
+        int sms = 0, per_sm = 0;
+        if (!sk_prepare_device(dev)) return 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv_sk, kThreads, gemv_sk_smem_bytes()) !=
+                cudaSuccess ||
+            per_sm < 1)
+            return 0;
+        warps[dev] = sms * per_sm * kWarps;
+    }
+    return warps[dev];
+}
+
+size_t linear_smem_bytes(int nt, int scl_stride) {
+    return (size_t)kRingBytes + (size_t)kWarps * kRows * scl_stride * 2 + (size_t)kWarps * 2 * nt * 4 * 32 * 4;
+}
+
+cudaError_t launch_linear(const Launch& L, int nt, int ctas, int prep_warps, bool overlap, cudaStream_t st) {
+    {
+        void* args[] = {const_cast<Launch*>(&L), &prep_warps};
+        cudaError_t e = launch_pdl((const void*)k_prep, args, (unsigned)((prep_warps + kWarps - 1) / kWarps), 0,
+                                   st, overlap);
+        if (e != cudaSuccess) return e;
+    }
+    bool m1 = true;
+    for (int i = 0; i < L.n_items; ++i) m1 = m1 && L.it[i].M == 1;
+    const size_t smem = linear_smem_bytes(nt, L.scl_stride);
+    if (nt == 1) return m1 ? launch_main<1, true>(L, ctas, smem, st) : launch_main<1, false>(L, ctas, smem, st);
+    return launch_main<2, false>(L, ctas, smem, st);
 }
 
 }  // namespace tb

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(PKG, "libtb_b200.so")
 TERNARY, INT2, INT3 = 0, 1, 2
 F32, BF16 = 0, 1
 MAX_LAYER_ITEMS = 16
+FLAG_OVERLAP_PREVIOUS = 1
 
 STATUS = {0: "TB_OK", 1: "TB_ERR_ARG", 2: "TB_ERR_SHAPE", 3: "TB_ERR_ALIGN", 4: "TB_ERR_UNSUPPORTED", 5: "TB_ERR_CUDA"}
 
@@ -31,9 +32,11 @@ SIGNATURES = {
     "tb_scales_absmax": (_I32, [_P, _I32, _I64, _I64, _I32, _P, _P]),
     "tb_pack": (_I32, [_P, _I32, _I64, _I64, _I32, _P, _P, _P, _P]),
     "tb_unpack": (_I32, [_P, _I32, _I64, _I64, _P, _P]),
-    "tb_gemv": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I64, _P]),
-    "tb_gemm": (_I32, [_P, _I32, _P, _P, _I64, _P, _I32, _I64, _I64, _I64, _I64, _P]),
-    "tb_layer_gemv": (_I32, [_P, _I32, _P]),
+    "tb_workspace_bytes": (_SZ, [_I64, _I64, _I64]),
+    "tb_layer_workspace_bytes": (_SZ, [_P, _I32]),
+    "tb_gemv": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I64, _P, _SZ, _P]),
+    "tb_gemm": (_I32, [_P, _I32, _P, _P, _I64, _P, _I32, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
+    "tb_layer_gemv": (_I32, [_P, _I32, ctypes.c_uint, _P, _SZ, _P]),
 }
 
 
@@ -148,22 +151,36 @@ def tb_unpack(packed: torch.Tensor, grid: int, N: int, K: int, codes: torch.Tens
     return codes
 
 
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(load().tb_workspace_bytes(M, N, K))
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """Caller-owned scratch for the products (256-byte aligned)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
 def tb_gemv(packed: torch.Tensor, grid: int, scales: torch.Tensor, x: torch.Tensor, N: int, K: int,
-            y: torch.Tensor | None = None, out_dtype=torch.float32) -> torch.Tensor:
+            y: torch.Tensor | None = None, out_dtype=torch.float32, ws: torch.Tensor | None = None) -> torch.Tensor:
     if y is None:
         y = torch.empty(N, dtype=out_dtype, device=x.device)
+    if ws is None:
+        ws = workspace(workspace_bytes(1, N, K), x.device)
     _check(load().tb_gemv(_dev(packed, "packed"), grid, _bits(scales, "scales"), _bits(x, "x"), _dev(y, "y"),
-                          _ydtype(y.dtype), N, K, _stream(x)), "tb_gemv")
+                          _ydtype(y.dtype), N, K, _dev(ws, "workspace"), ws.numel(), _stream(x)), "tb_gemv")
     return y
 
 
 def tb_gemm(packed: torch.Tensor, grid: int, scales: torch.Tensor, X: torch.Tensor, N: int, K: int,
-            Y: torch.Tensor | None = None, out_dtype=torch.float32) -> torch.Tensor:
+            Y: torch.Tensor | None = None, out_dtype=torch.float32, ws: torch.Tensor | None = None) -> torch.Tensor:
     M = X.shape[0]
     if Y is None:
         Y = torch.empty((M, N), dtype=out_dtype, device=X.device)
+    if ws is None:
+        ws = workspace(workspace_bytes(M, N, K), X.device)
     _check(load().tb_gemm(_dev(packed, "packed"), grid, _bits(scales, "scales"), _bits(X, "X"), X.stride(0),
-                          _dev(Y, "Y"), _ydtype(Y.dtype), Y.stride(0), M, N, K, _stream(X)), "tb_gemm")
+                          _dev(Y, "Y"), _ydtype(Y.dtype), Y.stride(0), M, N, K, _dev(ws, "workspace"), ws.numel(),
+                          _stream(X)), "tb_gemm")
     return Y
 
 
@@ -176,10 +193,17 @@ def linear_items(items) -> ctypes.Array:
     return arr
 
 
-def tb_layer_gemv(items, stream: int | None = None) -> None:
+def layer_workspace_bytes(arr: ctypes.Array) -> int:
+    return int(load().tb_layer_workspace_bytes(ctypes.cast(arr, ctypes.c_void_p), len(arr)))
+
+
+def tb_layer_gemv(items, ws: torch.Tensor | None = None, flags: int = 0, stream: int | None = None) -> None:
     """items: list of (packed, grid, scales, x, y, N, K), or a prebuilt
     linear_items() array (reused without re-marshalling)."""
     arr = items if isinstance(items, ctypes.Array) else linear_items(items)
     if stream is None:
         stream = torch.cuda.current_stream().cuda_stream
-    _check(load().tb_layer_gemv(ctypes.cast(arr, ctypes.c_void_p), len(arr), stream), "tb_layer_gemv")
+    if ws is None:
+        ws = workspace(layer_workspace_bytes(arr), torch.device("cuda", torch.cuda.current_device()))
+    _check(load().tb_layer_gemv(ctypes.cast(arr, ctypes.c_void_p), len(arr), flags, ws.data_ptr(), ws.numel(),
+                                stream), "tb_layer_gemv")

@@ -55,14 +55,17 @@
  * PRODUCTS
  *   y[n] = sum_k x[k] * c[n][k] * s[n][k/128], accumulated in fp32 per
  *   128-group and scaled once per group; fp32 output, or bf16 rounded half
- *   to even from the fp32 result.  Results are bitwise deterministic from
- *   run to run (no atomics in any reduction).
+ *   to even from the fp32 result.  Error bound: |y - y_exact| <= 1e-5 *
+ *   sum_k |x[k] c[n][k] s[n][k/128]| (plus 4e-3 |y| for bf16 outputs).
+ *   Results are bitwise deterministic from run to run (no atomics in any
+ *   reduction).
  *
  * ------------------------------------------------------------------------
  * CONVENTIONS
  *   - Every pointer argument is DEVICE memory on the current CUDA device
- *     unless the argument says otherwise.  The caller owns all buffers; the
- *     library keeps no allocation between calls.
+ *     unless the argument says otherwise.  The caller owns all buffers,
+ *     including the products' scratch workspace; the library allocates
+ *     nothing and keeps no allocation between calls.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All calls
  *     are asynchronous on `stream`; none synchronizes.
  *   - Alignment: packed, W, x / X rows: 16 bytes; scales: 2 bytes; y / Y:
@@ -142,20 +145,35 @@ TB_API tb_status_t tb_pack(const void *W, tb_dtype_t w_dtype, int64_t N, int64_t
 TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int64_t K, int8_t *codes,
                       tb_stream_t stream);
 
+/* Scratch ("workspace") of the products below.  Each call first writes a
+ * prepared copy of its activations (bf16, K per activation row, scaled by
+ * powers of two) and per-128-group sums into the workspace, then reads them;
+ * batch-1 calls also keep per-tile arrival counters and partial sums there
+ * (tiles of K split between warps are combined in a fixed order).
+ *   - device memory, 256-byte aligned, at least the size returned here;
+ *   - owned by the caller, written by every call: two calls that share a
+ *     workspace must be ordered (e.g. the same stream);
+ *   - no other state is kept between calls.
+ * Returns 0 for bad arguments. */
+TB_API size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K); /* tb_gemv: M = 1; tb_gemm: its M */
+
 /* Batch-1 GEMV y = W x over packed W (ThinkBit page, 무엇인가: one read of
  * every weight per decoded token; 전제와 한계: the direct 2/3-bit reader).
  *   packed, scales  as produced by tb_pack.
- *   x               [K] bf16, device, 16-byte aligned.
- *   y               [N] fp32 or bf16 (y_dtype), device, written. */
+ *   x               [K] bf16, device, 16-byte aligned; finite, |x| < 2^120.
+ *   y               [N] fp32 or bf16 (y_dtype), device, written.
+ *   workspace       tb_workspace_bytes(1, N, K) bytes (see above). */
 TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *x, void *y,
-                    tb_dtype_t y_dtype, int64_t N, int64_t K, tb_stream_t stream);
+                           tb_dtype_t y_dtype, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                           tb_stream_t stream);
 
 /* Small-batch GEMM Y = X W^T, 1 <= M <= 64.
- *   X  [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device.
- *   Y  [M][ldy] fp32 or bf16, ldy >= N, device; Y[m][n] for n < N written. */
-TB_API tb_status_t tb_gemm(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *X, int64_t ldx,
-                    void *Y, tb_dtype_t y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                    tb_stream_t stream);
+ *   X          [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device.
+ *   Y          [M][ldy] fp32 or bf16, ldy >= N, device; Y[m][n] for n < N written.
+ *   workspace  tb_workspace_bytes(M, N, K) bytes. */
+TB_API tb_status_t tb_gemm(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *X,
+                           int64_t ldx, void *Y, tb_dtype_t y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                           void *workspace, size_t workspace_bytes, tb_stream_t stream);
 
 /* One linear layer of a grouped launch. */
 typedef struct {
@@ -170,14 +188,28 @@ typedef struct {
 
 #define TB_MAX_LAYER_ITEMS 16
 
+/* Allow the call's kernels to start before earlier work in the stream has
+ * finished (programmatic dependent launch): they begin streaming the packed
+ * weights and scales at once and wait for the earlier work only before
+ * touching activations, outputs or the workspace.  The caller promises that
+ * no earlier work still in flight writes the packed weights or scales of
+ * this call (true for resident model weights during decode). */
+#define TB_FLAG_OVERLAP_PREVIOUS 1u
+
+/* Workspace bytes of tb_layer_gemv for these items (0 for bad arguments). */
+TB_API size_t tb_layer_workspace_bytes(const tb_linear_t *items, int n_items);
+
 /* Mixed-grid grouped GEMV: every item is an independent y = W x with its
- * own grid, shape, input and output, all run by ONE kernel launch (e.g. a
- * decoder layer's q, k, v, o, gate, up and down projections, each on its
+ * own grid, shape, input and output, all run by ONE main kernel launch (e.g.
+ * a decoder layer's q, k, v, o, gate, up and down projections, each on its
  * own grid; ThinkBit page, 무엇과 다른가: grids chosen per layer).
- *   items    HOST array of n_items descriptors (read before returning).
- *   n_items  1 .. TB_MAX_LAYER_ITEMS.
+ *   items      HOST array of n_items descriptors (read before returning).
+ *   n_items    1 .. TB_MAX_LAYER_ITEMS.
+ *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS.
+ *   workspace  tb_layer_workspace_bytes(items, n_items) bytes.
  * Outputs of different items must not overlap. */
-TB_API tb_status_t tb_layer_gemv(const tb_linear_t *items, int n_items, tb_stream_t stream);
+TB_API tb_status_t tb_layer_gemv(const tb_linear_t *items, int n_items, unsigned flags, void *workspace,
+                                 size_t workspace_bytes, tb_stream_t stream);
 
 #ifdef __cplusplus
 }

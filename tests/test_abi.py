@@ -31,7 +31,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("tb_pack", "tb_unpack", "tb_gemv", "tb_gemm", "tb_layer_gemv", "tb_scales_absmax",
-                 "tb_packed_bytes", "tb_scale_bytes", "tb_status_string", "tb_version"):
+                 "tb_packed_bytes", "tb_scale_bytes", "tb_status_string", "tb_version", "tb_workspace_bytes",
+                 "tb_layer_workspace_bytes"):
         assert must in names
     assert set(names) == set(tb.SIGNATURES), "binding and header disagree"
 
@@ -62,42 +63,70 @@ def test_sizes_closed_form(lib):
 FAKE = 1 << 40  # a 256-byte-aligned address that is never dereferenced
 
 
+def test_workspace_sizes(lib):
+    al = lambda b: (b + 255) // 256 * 256
+    for M, N, K in ((4, 100, 5120), (16, 17408, 17408), (64, 7, 1024)):
+        # prepared activations (2 bytes per element) + per-group pairs (8 bytes), each 256-byte aligned
+        Mb = min(M, 16)
+        assert tb.workspace_bytes(M, N, K) == al(2 * Mb * K) + al(8 * Mb * (K // 128))
+    for N, K in ((1, 128), (256, 1024), (17408, 5120)):
+        # batch 1 adds a counter per 32-row tile and two 32-float slots per warp
+        tiles = (N + 31) // 32
+        warps = min(8192, tiles * (K // 128))
+        assert tb.workspace_bytes(1, N, K) == al(2 * K) + al(8 * (K // 128)) + al(4 * tiles) + al(256 * warps)
+    assert tb.workspace_bytes(0, 8, 128) == 0 and tb.workspace_bytes(1, 8, 100) == 0
+    assert tb.workspace_bytes(65, 8, 128) == 0 and tb.workspace_bytes(1, 0, 128) == 0
+    items = (tb.Linear * 3)()
+    for i, (N, K) in enumerate(((4096, 4096), (1024, 4096), (4096, 12288))):
+        items[i] = tb.Linear(FAKE, FAKE, FAKE, FAKE, N, K, 1, 0)
+    tiles = sum((N + 31) // 32 for N in (4096, 1024, 4096))
+    tgs = sum((N + 31) // 32 * (K // 128) for N, K in ((4096, 4096), (1024, 4096), (4096, 12288)))
+    per = sum(al(2 * K) + al(8 * (K // 128)) for K in (4096, 4096, 12288))
+    assert tb.layer_workspace_bytes(items) == per + al(4 * tiles) + al(256 * min(8192, tgs))
+
+
 def test_argument_errors_before_launch(lib):
     A = FAKE
+    W = 1 << 20  # workspace size, never touched
     # null pointers / bad enums -> TB_ERR_ARG (1)
-    assert lib.tb_gemv(0, 1, A, A, A, 0, 16, 128, 0) == 1
-    assert lib.tb_gemv(A, 9, A, A, A, 0, 16, 128, 0) == 1
-    assert lib.tb_gemv(A, 1, A, A, A, 5, 16, 128, 0) == 1
+    assert lib.tb_gemv(0, 1, A, A, A, 0, 16, 128, A, W, 0) == 1
+    assert lib.tb_gemv(A, 9, A, A, A, 0, 16, 128, A, W, 0) == 1
+    assert lib.tb_gemv(A, 1, A, A, A, 5, 16, 128, A, W, 0) == 1
+    assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 128, 0, W, 0) == 1
+    assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 128, A, 16, 0) == 1  # workspace too small
     assert lib.tb_pack(A, 3, 16, 128, 1, A, A, 0, 0) == 1
-    assert lib.tb_layer_gemv(0, 1, 0) == 1
+    assert lib.tb_layer_gemv(0, 1, 0, A, W, 0) == 1
     items = (tb.Linear * 17)()
-    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 17, 0) == 1
-    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 0, 0) == 1
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 17, 0, A, W, 0) == 1
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 0, 0, A, W, 0) == 1
     # shapes -> TB_ERR_SHAPE (2)
-    assert lib.tb_gemv(A, 1, A, A, A, 0, 0, 128, 0) == 2
-    assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 100, 0) == 2
-    assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 0, 0) == 2
-    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 16, 65, 16, 128, 0) == 2
-    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 16, 0, 16, 128, 0) == 2
-    assert lib.tb_gemm(A, 1, A, A, 120, A, 0, 16, 4, 16, 128, 0) == 2
-    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 8, 4, 16, 128, 0) == 2
+    assert lib.tb_gemv(A, 1, A, A, A, 0, 0, 128, A, W, 0) == 2
+    assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 100, A, W, 0) == 2
+    assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 0, A, W, 0) == 2
+    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 16, 65, 16, 128, A, W, 0) == 2
+    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 16, 0, 16, 128, A, W, 0) == 2
+    assert lib.tb_gemm(A, 1, A, A, 120, A, 0, 16, 4, 16, 128, A, W, 0) == 2
+    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 8, 4, 16, 128, A, W, 0) == 2
     assert lib.tb_pack(A, 0, 16, 200, 1, A, A, 0, 0) == 2
     assert lib.tb_unpack(A, 1, -1, 128, A, 0) == 2
     # alignment -> TB_ERR_ALIGN (3)
-    assert lib.tb_gemv(A + 8, 1, A, A, A, 0, 16, 128, 0) == 3
-    assert lib.tb_gemv(A, 1, A + 1, A, A, 0, 16, 128, 0) == 3
-    assert lib.tb_gemv(A, 1, A, A + 2, A, 0, 16, 128, 0) == 3
-    assert lib.tb_gemv(A, 1, A, A, A + 2, 0, 16, 128, 0) == 3
-    assert lib.tb_gemm(A, 1, A, A, 132, A, 0, 16, 4, 16, 128, 0) == 3
+    assert lib.tb_gemv(A + 8, 1, A, A, A, 0, 16, 128, A, W, 0) == 3
+    assert lib.tb_gemv(A, 1, A + 1, A, A, 0, 16, 128, A, W, 0) == 3
+    assert lib.tb_gemv(A, 1, A, A + 2, A, 0, 16, 128, A, W, 0) == 3
+    assert lib.tb_gemv(A, 1, A, A, A + 2, 0, 16, 128, A, W, 0) == 3
+    assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 128, A + 16, W, 0) == 3
+    assert lib.tb_gemm(A, 1, A, A, 132, A, 0, 16, 4, 16, 128, A, W, 0) == 3
     assert lib.tb_pack(A + 4, 0, 16, 128, 1, A, A, 0, 0) == 3
     items = (tb.Linear * 2)()
     for i in range(2):
         items[i] = tb.Linear(A, A, A, A, 16, 128, 1, 0)
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 2, A, W, 0) == 1  # unknown flag
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0, A + 64, W, 0) == 3
     items[1].x = A + 8
-    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0) == 3
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0, A, W, 0) == 3
     items[1].x = A
     items[1].K = 130
-    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0) == 2
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0, A, W, 0) == 2
 
 
 def test_binding_fails_loudly_without_library(tmp_path):
