@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <climits>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/tb.h"
 #include "tb_device.cuh"
@@ -359,6 +360,62 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
     }
     return launch_sk_items(its, n_items, workspace, workspace_bytes, (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0,
                            static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+// ---- tb_gemv_noalloc: tb_gemv over a fixed, statically allocated scratch ----
+//
+// Same kernels and results as tb_gemv; the workspace is this file-scope
+// device array instead of caller memory, so the call allocates nothing.
+// The only state that must start at zero (the per-tile arrival counters)
+// is zeroed by the preparation kernel of every call, so the array needs no
+// clearing; every call rewrites what it reads.  All calls on a device
+// share the one array: calls that may run at the same time (different
+// streams, or different host threads without stream ordering) race on it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TB_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxScratchDevices] = {};
+
+// Address of the array on the current device, looked up once per device
+// (with that device current) and cached; nullptr if the lookup fails.
+void* noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxScratchDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+        g_scratch_ptr[dev] = p;
+    }
+    return g_scratch_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+tb_status_t tb_gemv_noalloc(const void* packed, tb_grid_t grid, const uint16_t* scales, const uint16_t* x, void* y,
+                            tb_dtype_t y_dtype, int64_t N, int64_t K, tb_stream_t stream) {
+    tb_status_t s = check_weights(packed, grid, scales, N, K);
+    if (s != TB_OK) return s;
+    if (!x) return TB_ERR_ARG;
+    if ((s = check_out(y, y_dtype)) != TB_OK) return s;
+    if (!aligned(x, 16)) return TB_ERR_ALIGN;
+    // the size rule is checked before any CUDA call
+    if (tb_workspace_bytes(1, N, K) > (size_t)TB_NOALLOC_SCRATCH_BYTES) return TB_ERR_UNSUPPORTED;
+    void* scratch = noalloc_scratch();
+    if (!scratch) return TB_ERR_CUDA;
+    Item it = make_item(packed, grid, scales, x, K, y, y_dtype, N, 1, N, K);
+    return launch_sk_items(&it, 1, scratch, TB_NOALLOC_SCRATCH_BYTES, false, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -19,6 +19,7 @@ TERNARY, INT2, INT3 = 0, 1, 2
 F32, BF16 = 0, 1
 MAX_LAYER_ITEMS = 16
 FLAG_OVERLAP_PREVIOUS = 1
+NOALLOC_SCRATCH_BYTES = 4 << 20  # TB_NOALLOC_SCRATCH_BYTES
 
 STATUS = {0: "TB_OK", 1: "TB_ERR_ARG", 2: "TB_ERR_SHAPE", 3: "TB_ERR_ALIGN", 4: "TB_ERR_UNSUPPORTED", 5: "TB_ERR_CUDA"}
 
@@ -37,6 +38,7 @@ SIGNATURES = {
     "tb_gemv": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I64, _P, _SZ, _P]),
     "tb_gemm": (_I32, [_P, _I32, _P, _P, _I64, _P, _I32, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "tb_layer_gemv": (_I32, [_P, _I32, ctypes.c_uint, _P, _SZ, _P]),
+    "tb_gemv_noalloc": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I64, _P]),
 }
 
 
@@ -168,6 +170,15 @@ def tb_gemv(packed: torch.Tensor, grid: int, scales: torch.Tensor, x: torch.Tens
         ws = workspace(workspace_bytes(1, N, K), x.device)
     _check(load().tb_gemv(_dev(packed, "packed"), grid, _bits(scales, "scales"), _bits(x, "x"), _dev(y, "y"),
                           _ydtype(y.dtype), N, K, _dev(ws, "workspace"), ws.numel(), _stream(x)), "tb_gemv")
+    return y
+
+
+def tb_gemv_noalloc(packed: torch.Tensor, grid: int, scales: torch.Tensor, x: torch.Tensor, N: int, K: int,
+                    y: torch.Tensor) -> torch.Tensor:
+    """tb_gemv over the library's fixed device scratch: no workspace, and
+    the caller provides y, so the call itself allocates nothing."""
+    _check(load().tb_gemv_noalloc(_dev(packed, "packed"), grid, _bits(scales, "scales"), _bits(x, "x"),
+                                  _dev(y, "y"), _ydtype(y.dtype), N, K, _stream(x)), "tb_gemv_noalloc")
     return y
 
 

@@ -211,6 +211,34 @@ TB_API size_t tb_layer_workspace_bytes(const tb_linear_t *items, int n_items);
 TB_API tb_status_t tb_layer_gemv(const tb_linear_t *items, int n_items, unsigned flags, void *workspace,
                                  size_t workspace_bytes, tb_stream_t stream);
 
+/* Size of the fixed device scratch behind tb_gemv_noalloc (4 MiB). */
+#define TB_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* tb_gemv without a workspace argument and without allocating anything.
+ * The ThinkBit pages have no counterpart: this is an interface variant of
+ * tb_gemv for callers that cannot hand over device scratch -- a plain C
+ * host with no device allocator of its own, or a decode loop that must not
+ * call cudaMalloc/cudaFree (or an allocator that may call them) because
+ * those calls can synchronize the device and stall other streams.
+ * Arguments and results are those of tb_gemv; x and y still belong to the
+ * caller.
+ *   scratch  one statically allocated device array of
+ *            TB_NOALLOC_SCRATCH_BYTES per device, inside this library.  A
+ *            problem whose tb_workspace_bytes(1, N, K) exceeds that size is
+ *            rejected with TB_ERR_UNSUPPORTED before any CUDA call (every
+ *            N <= 2^20 with K <= 2^19 fits).  Nothing has to be cleared by
+ *            the caller: the call itself zeroes what must start at zero.
+ *   setup    the first call on each device (with that device current) looks
+ *            up the array's address with cudaGetSymbolAddress and caches it;
+ *            make that first call before any stream capture.  A failed
+ *            lookup returns TB_ERR_CUDA and is retried on the next call.
+ *   sharing  every call on a device uses the same array: calls on one stream
+ *            are ordered and safe; calls that can overlap (other streams,
+ *            other host threads) race and give wrong results -- use tb_gemv
+ *            with separate workspaces for those. */
+TB_API tb_status_t tb_gemv_noalloc(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *x,
+                                   void *y, tb_dtype_t y_dtype, int64_t N, int64_t K, tb_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
