@@ -74,6 +74,9 @@ size_t sk_extra_workspace(int64_t tiles, int64_t tile_groups) {
     return align256((size_t)(tiles * 4)) + align256((size_t)(w * 2 * 32 * 4));
 }
 
+// batch sizes from which tb_gemm runs on the tcgen05 path
+constexpr int64_t kTCMinM = 32;
+
 int device_sms() {
     static int sms[64] = {0};
     int dev = 0;
@@ -234,6 +237,8 @@ extern "C" {
 
 int tb_version(void) { return 100; }
 
+unsigned int tb_wait_timeouts(void) { return take_wait_timeouts(); }
+
 const char* tb_status_string(tb_status_t s) {
     switch (s) {
         case TB_OK: return "ok";
@@ -288,6 +293,7 @@ size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K) {
         const int64_t tiles = (N + 31) / 32;
         return item_workspace(1, K) + sk_extra_workspace(tiles, tiles * (K / kGroup));
     }
+    if (M >= kTCMinM) return gemm_tc_workspace_bytes(M, N, K);
     return item_workspace(std::min<int64_t>(M, 16), K);
 }
 
@@ -331,6 +337,11 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if (M == 1) {
         Item it = make_item(packed, grid, scales, X, ldx, Y, y_dtype, N, 1, N, K);
         return launch_sk_items(&it, 1, workspace, workspace_bytes, false, st);
+    }
+    if (M >= kTCMinM) {
+        if (workspace_bytes < gemm_tc_workspace_bytes(M, N, K)) return TB_ERR_ARG;
+        if (K / kGroup * 64 > INT_MAX || (N + 127) / 128 > INT_MAX / 16) return TB_ERR_SHAPE;
+        return cuda_status(launch_gemm_tc(packed, grid, scales, X, ldx, Y, y_dtype, ldy, (int)M, N, K, workspace, st));
     }
     // column blocks of up to 16 batch rows per launch
     const size_t ysz = y_dtype == TB_F32 ? 4 : 2;

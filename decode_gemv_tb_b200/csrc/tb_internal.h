@@ -30,4 +30,14 @@ cudaError_t launch_gemv_sk(const Launch& P, int prep_warps, const SKLaunch& L, i
 // warps of the stream-K kernel resident at once on the current device (0 on error)
 int gemv_sk_resident_warps();
 
+// Small-batch GEMM on the tcgen05 tensor cores (2 <= M <= 64): preparation
+// kernel + main kernel.  Workspace: gemm_tc_workspace_bytes(M, N, K) bytes,
+// 256-byte aligned (device independent).
+size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemm_tc(const void* packed, int grid, const uint16_t* scales, const uint16_t* X, int64_t ldx,
+                           void* Y, int ydt, int64_t ldy, int M, int64_t N, int64_t K, void* ws, cudaStream_t st);
+// bounded device waits that gave up since the last call (clears the count;
+// synchronous); 0xFFFFFFFF if the count cannot be read
+unsigned int take_wait_timeouts();
+
 }  // namespace tb

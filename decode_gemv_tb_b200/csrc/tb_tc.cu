@@ -1,0 +1,571 @@
+// tb_tc.cu -- small-batch GEMM  Y = X W^T  on the fifth-generation tensor
+// cores (tcgen05), straight from the packed 2- and 3-bit codewords.
+//
+// ThinkBit page "ThinkBit은 2비트 양자화에서 추론 능력 보존을 추론 평가로
+// 검증한다" (onedev.kr/papers/1416), section 어떻게 동작하나: w = c * s with
+// one bf16 scale per 128 input weights; the product per output row n,
+// batch row m and 128-group g is
+//     Y[m][n] += s[n][g] * (sum_k u[n][k] X[m][k]  -  offset * sum_k X[m][k])
+// with u = c + offset the stored code.
+//
+// Data flow of one CTA (128 threads, one weight row per thread, a 128-row
+// tile of W and a contiguous range of its 128-groups):
+//   * every thread loads its row's packed words for the next group with
+//     128-bit loads and decodes them without arithmetic: masking one field
+//     at bit position p of each 16-bit half gives a bf16 pair u * 2^(p-133)
+//     (a bf16 pattern below 256 is exactly that multiple of 2^-133); the
+//     64 pairs of a group are written to tensor memory (tcgen05.st), one
+//     TMEM lane per row, k in natural order along the columns -- this is
+//     the A operand;
+//   * the preparation kernel has stored X per group as
+//         X[m][k] * 2^(133 - S_mg - p(k))       (exact: powers of two)
+//     in the K-major core-matrix layout the MMA reads from shared memory,
+//     followed by (offset * sum_k X[m][k], 2^S_mg); one thread brings each
+//     group in with a 1-D bulk copy, four groups ahead -- the B operand;
+//   * thread 0 issues the group's eight 128 x NP x 16 MMAs (bf16 in, fp32
+//     accumulate in tensor memory) and commits them to an mbarrier;
+//   * while they run, every thread reads its row of the previous group's
+//     accumulator back (tcgen05.ld) and applies the group scale:
+//         acc[m] += s * (2^S * D[m] - offset * sum X)
+//     A and D are double-buffered in tensor memory (2 x 64 + 2 x NP
+//     columns of the 256 a CTA allocates).
+// K-splits of one tile are combined by the last CTA to finish, in split
+// order (deterministic).  Every wait is bounded: a wait that gives up
+// counts itself in g_wait_timeouts, the CTA stops issuing work, waits
+// (bounded) for what it already issued, writes NaN outputs, frees its
+// tensor memory and exits.
+#include "tb_device.cuh"
+#include "tb_internal.h"
+
+#include <algorithm>
+
+namespace tb {
+
+// bounded waits that gave up since the last tb_wait_timeouts() call
+__device__ unsigned int g_wait_timeouts = 0;
+
+namespace {
+
+constexpr int kTCThreads = 128;   // one thread per row of the 128-row tile
+constexpr int kTCRows = 128;
+constexpr int kTCStages = 4;      // prepared X groups in shared memory
+constexpr uint32_t kTmemCols = 256;
+constexpr long long kWaitCycles = 4000000000LL;  // about 2 s at 2 GHz
+constexpr int kTCTargetCtas = 296;               // 2 CTAs on each of 148 SMs
+constexpr int kTCMaxSplits = 16;
+constexpr size_t kTCMinSmem = 80 * 1024;         // at most two CTAs (2 x 256 TMEM columns) per SM
+
+__host__ __device__ constexpr int tc_group_bytes(int np) { return np * 264; }  // NP x 128 bf16 + NP float2
+
+// field position (bit of its 16-bit half) of 3-bit field f after the decode below
+__host__ __device__ constexpr int pos3(int f) { return f < 12 ? f % 6 : (f & 1); }
+
+__device__ __forceinline__ uint32_t shr_fma(uint32_t x, int k) { return __umulhi(x, 1u << (32 - k)); }
+
+constexpr uint32_t bits_at(int first, int count, int shift) {
+    uint32_t m = 0;
+    for (int i = 0; i < count; ++i) m |= (1u << (first + 3 * i + shift)) | (1u << (16 + first + 3 * i + shift));
+    return m;
+}
+
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// ---- mbarrier --------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+// true once the phase with this parity has completed; false after about
+// kWaitCycles (counted in g_wait_timeouts)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_addr(bar);
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (clock64() - t0 > kWaitCycles) {
+            atomicAdd(&g_wait_timeouts, 1u);
+            return false;
+        }
+    }
+}
+
+// 1-D bulk copy global -> shared, completion counted on bar (no multicast)
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+// ---- tensor memory -----------------------------------------------------------
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 16 consecutive columns of this thread's lane, complete on return
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&d)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) d[i] = __uint_as_float(r[i]);
+}
+
+// D[tmem d] (+)= A[tmem a] x B[smem desc b]; one thread issues
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, bool accumulate) {
+    const uint32_t z = 0, acc = accumulate ? 1u : 0u;
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n}" ::"r"(d),
+        "r"(a), "l"(bdesc), "r"(idesc), "r"(acc), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand without swizzle: core
+// matrices of 8 rows x 16 bytes, the next 8 k (16 bytes) 128 bytes on
+// (leading byte offset), the next 8 rows 2048 bytes on (stride byte offset).
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(2048 >> 4) << 32) |
+           (1ull << 46);
+}
+
+// kind::f16 instruction descriptor: fp32 D, bf16 A and B, both K-major, M = 128, N = np
+__host__ __device__ constexpr uint32_t idesc_bf16(int np) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(np >> 3) << 17) | ((uint32_t)(kTCRows >> 4) << 24);
+}
+
+// ---- decode: one row's group into 64 bf16 pairs (TMEM columns) -----------------
+// 2-bit container: word i holds codes 16i .. 16i+15; field m (codes
+// 16i+2m, 16i+2m+1) masked in place for m < 4 (p = 2m) and after >> 8 for
+// m >= 4 (p = 2m - 8): column 8i + m.
+__device__ __forceinline__ void decode2_pair(uint32_t w0, uint32_t w1, uint32_t (&r)[16]) {
+    const uint32_t h0 = shr_fma(w0, 8), h1 = shr_fma(w1, 8);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const uint32_t mk = 0x00030003u << (2 * m);
+        r[m] = w0 & mk;
+        r[4 + m] = h0 & mk;
+        r[8 + m] = w1 & mk;
+        r[12 + m] = h1 & mk;
+    }
+}
+// 3-bit block: planes p0..p2 of codes 32j .. 32j+31; field f (codes 32j+2f,
+// 32j+2f+1) assembled from the planes at position pos3(f): column 16j + f.
+__device__ __forceinline__ void decode3_block(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t (&r)[16]) {
+    const uint32_t q1 = p1 << 1, q2 = p2 << 2;
+    const uint32_t zA = bit_mux(bit_mux(p0, q1, bits_at(0, 5, 1)), q2, bits_at(0, 5, 2));  // fields 0,3,6,9,12
+    const uint32_t zB = bit_mux(bit_mux(p0, q1, bits_at(1, 5, 1)), q2, bits_at(1, 5, 2));  // fields 1,4,7,10,13
+    const uint32_t zC = bit_mux(bit_mux(p0, q1, bits_at(2, 4, 1)), q2, bits_at(2, 4, 2));  // fields 2,5,8,11
+    const uint32_t a6 = shr_fma(zA, 6), b6 = shr_fma(zB, 6), c6 = shr_fma(zC, 6);
+    const uint32_t a12 = shr_fma(zA, 12), b12 = shr_fma(zB, 12);
+    // fields 14, 15 (plane bits 14/15 and 30/31): plane p realigned right by 14 - p
+    const uint32_t r0 = shr_fma(p0, 14), r1 = shr_fma(p1, 13), r2 = shr_fma(p2, 12);
+    const uint32_t z14 = bit_mux(bit_mux(r0, r1, 0x00020002u), r2, 0x00040004u);
+    const uint32_t z15 = bit_mux(bit_mux(r0, r1, 0x00040004u), r2, 0x00080008u);
+    r[0] = zA & 0x00070007u;
+    r[1] = zB & 0x000E000Eu;
+    r[2] = zC & 0x001C001Cu;
+    r[3] = zA & 0x00380038u;
+    r[4] = zB & 0x00700070u;
+    r[5] = zC & 0x00E000E0u;
+    r[6] = a6 & 0x00070007u;
+    r[7] = b6 & 0x000E000Eu;
+    r[8] = c6 & 0x001C001Cu;
+    r[9] = a6 & 0x00380038u;
+    r[10] = b6 & 0x00700070u;
+    r[11] = c6 & 0x00E000E0u;
+    r[12] = a12 & 0x00070007u;
+    r[13] = b12 & 0x000E000Eu;
+    r[14] = z14 & 0x00070007u;
+    r[15] = z15 & 0x000E000Eu;
+}
+
+}  // namespace
+
+struct TCArgs {
+    const uint8_t* packed;
+    const uint16_t* scales;
+    const uint16_t* X;  // [M][ldx] bf16
+    uint8_t* bprep;     // G prepared groups of tc_group_bytes(NP)
+    void* Y;            // [M][ldy]
+    float* partials;    // [tiles][splits][NP][128] when splits > 1
+    int32_t* counters;  // [tiles]
+    int64_t N, K, ldx, ldy;
+    int32_t M, NP, grid, ydt, G, tiles, splits;
+};
+
+namespace {
+
+// ---- preparation: one warp per (group g, batch row m < NP) -------------------
+__global__ void __launch_bounds__(256) k_prep_tc(const __grid_constant__ TCArgs A) {
+    for (int i = blockIdx.x * 256 + threadIdx.x; i < A.tiles; i += gridDim.x * 256) A.counters[i] = 0;
+    const int wi = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (wi >= A.G * A.NP) return;
+    const int g = wi / A.NP, m = wi - g * A.NP;
+    uint8_t* gb = A.bprep + (int64_t)g * tc_group_bytes(A.NP);
+    // elements k = 4 lane .. 4 lane + 3 of row m: core matrix (m / 8, k / 8), row m % 8, bytes 2 (k % 8)
+    uint8_t* dst = gb + ((m >> 3) * 16 + (lane >> 1)) * 128 + (m & 7) * 16 + 8 * (lane & 1);
+    if (m >= A.M) {  // padding rows of B: zero, and zero correction terms
+        *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+        if (lane == 0) *reinterpret_cast<float2*>(gb + A.NP * 256 + 8 * m) = make_float2(0.f, 0.f);
+        return;
+    }
+    const uint16_t* xg = A.X + (int64_t)m * A.ldx + (int64_t)g * kGroup;
+    const uint2 raw = *reinterpret_cast<const uint2*>(xg + 4 * lane);
+    const uint32_t hv[4] = {raw.x & 0xFFFFu, raw.x >> 16, raw.y & 0xFFFFu, raw.y >> 16};
+    int e = 0;
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        e = max(e, (int)((hv[j] >> 7) & 0xFFu));
+        sum += bf16_bits_to_float(hv[j]);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    // S = exponent of max |x| + 7 (a zero or subnormal group counts as 2^-126)
+    const int S = min(max(e, 1) - 127 + 7, 127);
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int k = 4 * lane + j;
+        const int p = A.grid == kInt3 ? pos3((k & 31) >> 1) : 2 * ((k >> 1) & 3);
+        const int sh = 133 - S - p;  // 1 .. 252: two exact power-of-two factors
+        const int s1 = sh >> 1, s2 = sh - s1;
+        const float v = bf16_bits_to_float(hv[j]) * __int_as_float((s1 + 127) << 23) * __int_as_float((s2 + 127) << 23);
+        out[j >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v)) << (16 * (j & 1));
+    }
+    *reinterpret_cast<uint2*>(dst) = make_uint2(out[0], out[1]);
+    if (lane == 0) {
+        const float off = A.grid == kInt3 ? 4.f : 2.f;
+        *reinterpret_cast<float2*>(gb + A.NP * 256 + 8 * m) = make_float2(off * sum, __int_as_float((S + 127) << 23));
+    }
+}
+
+// ---- main kernel -------------------------------------------------------------
+template <int NP, int KIND>
+__global__ void __launch_bounds__(kTCThreads, 1) k_gemm_tc(const __grid_constant__ TCArgs A) {
+    constexpr int GB = NP * 264;             // bytes of one prepared group (a multiple of 128)
+    constexpr int WQ = KIND ? 3 : 2;          // 16-byte packed words per row and group
+    constexpr uint32_t kIdesc = idesc_bf16(NP);
+    extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ __align__(8) uint64_t bar_full[kTCStages];
+    __shared__ __align__(8) uint64_t bar_mma[2];
+    __shared__ uint32_t tmem_sh;
+    __shared__ int last_sh;
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tile = blockIdx.x / A.splits, split = blockIdx.x - tile * A.splits;
+    const int g0 = (int)((int64_t)split * A.G / A.splits);
+    const int ng = (int)((int64_t)(split + 1) * A.G / A.splits) - g0;
+    const int64_t row = (int64_t)tile * kTCRows + tid;
+    const bool row_ok = row < A.N;
+    const int64_t rbytes = KIND ? 3 * A.K / 8 : A.K / 4;
+    const uint8_t* rowp = A.packed + (row_ok ? row : 0) * rbytes + (int64_t)g0 * (16 * WQ);
+    const uint16_t* srow = A.scales + (row_ok ? row : 0) * A.G + g0;
+
+    if (tid == 0) {
+        for (int s = 0; s < kTCStages; ++s) mbar_init(&bar_full[s], 1);
+        mbar_init(&bar_mma[0], 1);
+        mbar_init(&bar_mma[1], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&tmem_sh)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_sh;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // this warp's 32 TMEM lanes
+
+    int issued = 0;  // prepared groups whose copy thread 0 has issued
+    auto issue = [&](int i) {
+        const int s = i % kTCStages;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_expect_tx(&bar_full[s], GB);
+        bulk_g2s(smem + s * GB, A.bprep + (int64_t)(g0 + i) * GB, GB, &bar_full[s]);
+    };
+    if (tid == 0)
+        for (; issued < min(2, ng); ++issued) issue(issued);
+
+    uint4 nxt[WQ];
+    uint32_t s_nxt = 0;
+    auto load = [&](int i) {
+#pragma unroll
+        for (int q = 0; q < WQ; ++q) nxt[q] = row_ok ? ld_stream_u4(rowp + (int64_t)i * (16 * WQ) + 16 * q) : make_uint4(0, 0, 0, 0);
+        s_nxt = row_ok ? (uint32_t)__ldg(srow + i) : 0u;
+    };
+    if (ng > 0) load(0);
+
+    float acc[NP];
+#pragma unroll
+    for (int m = 0; m < NP; ++m) acc[m] = 0.f;
+
+    bool fail = false;      // this thread's bounded wait gave up
+    int committed = 0;      // groups whose MMAs thread 0 committed
+    uint32_t s_last = 0;    // scale of the group whose epilogue runs next
+    for (int i = 0; i <= ng; ++i) {
+        const bool have = i < ng;
+        const int b = i & 1;
+        uint32_t s_cur = 0;
+        if (have) {
+            uint4 cur[WQ];
+#pragma unroll
+            for (int q = 0; q < WQ; ++q) cur[q] = nxt[q];
+            s_cur = s_nxt;
+            if (i + 1 < ng) load(i + 1);
+            // A buffer b: its previous MMAs (group i - 2) completed before the
+            // epilogue of group i - 2, which this thread ran last iteration
+            const uint32_t acol = tmem + lane_base + (uint32_t)(b * 64);
+            if (KIND == 0) {
+                const uint32_t w[8] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[16];
+                    decode2_pair(w[2 * c], w[2 * c + 1], r);
+                    tmem_st16(acol + 16 * c, r);
+                }
+            } else {
+                const uint32_t w[12] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y,
+                                        cur[1].z, cur[1].w, cur[2].x, cur[2].y, cur[2].z, cur[2].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t r[16];
+                    decode3_block(w[3 * j], w[3 * j + 1], w[3 * j + 2], r);
+                    tmem_st16(acol + 16 * j, r);
+                }
+            }
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        if (__syncthreads_or(fail ? 1 : 0)) break;  // uniform: every thread leaves together
+        if (have && tid == 0) {
+            tc_fence_after();
+            const int s = i % kTCStages;
+            if (!mbar_wait(&bar_full[s], (uint32_t)(i / kTCStages) & 1u)) {
+                fail = true;
+            } else {
+                const uint32_t bbase = smem_addr(smem + s * GB);
+                const uint32_t dcol = tmem + 128u + (uint32_t)(b * NP);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    mma_ts(dcol, tmem + (uint32_t)(b * 64 + 8 * j), kmajor_desc(bbase + 256u * j), kIdesc, j > 0);
+                mma_commit(&bar_mma[b]);
+                committed = i + 1;
+                // stage (i + 2) % kTCStages last held group i - 2, whose MMAs
+                // and epilogue finished before this iteration's barrier
+                if (issued < ng && issued == i + 2) issue(issued++);
+            }
+        }
+        if (i >= 1) {  // epilogue of group i - 1 (warp-uniform: tcgen05.ld is a warp instruction)
+            const int bp = (i - 1) & 1;
+            bool ok = !__any_sync(0xffffffffu, fail);
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_mma[bp], (uint32_t)((i - 1) >> 1) & 1u));
+            if (!ok) {
+                fail = true;
+            } else {
+                tc_fence_after();
+                const float sc = bf16_bits_to_float(s_last);
+                const float2* cf = reinterpret_cast<const float2*>(smem + ((i - 1) % kTCStages) * GB + NP * 256);
+                const uint32_t dcol = tmem + lane_base + 128u + (uint32_t)(bp * NP);
+#pragma unroll
+                for (int c = 0; c < NP / 16; ++c) {
+                    float d[16];
+                    tmem_ld16(dcol + 16 * c, d);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const float2 v = cf[16 * c + q];
+                        acc[16 * c + q] = fmaf(sc, fmaf(v.y, d[q], -v.x), acc[16 * c + q]);
+                    }
+                }
+            }
+        }
+        s_last = s_cur;
+    }
+
+    const bool aborted = __syncthreads_or(fail ? 1 : 0) != 0;
+    if (aborted && tid == 0) {  // wait (bounded) for the copies and MMAs already issued
+        for (int i = 0; i < issued; ++i) mbar_wait(&bar_full[i % kTCStages], (uint32_t)(i / kTCStages) & 1u);
+        if (committed > 0) mbar_wait(&bar_mma[(committed - 1) & 1], (uint32_t)((committed - 1) >> 1) & 1u);
+    }
+    if (aborted) {
+#pragma unroll
+        for (int m = 0; m < NP; ++m) acc[m] = __int_as_float(0x7FC00000);
+    }
+
+    // ---- output ----
+    auto store = [&](int m, float v) {
+        if (A.ydt == kF32)
+            static_cast<float*>(A.Y)[(int64_t)m * A.ldy + row] = v;
+        else
+            static_cast<__nv_bfloat16*>(A.Y)[(int64_t)m * A.ldy + row] = __float2bfloat16_rn(v);
+    };
+    if (A.splits == 1) {
+        if (row_ok) {
+#pragma unroll
+            for (int m = 0; m < NP; ++m)
+                if (m < A.M) store(m, acc[m]);
+        }
+    } else {
+        float* slot = A.partials + ((int64_t)(tile * A.splits + split) * NP) * kTCRows;
+#pragma unroll
+        for (int m = 0; m < NP; ++m)
+            if (m < A.M) __stcg(slot + m * kTCRows + tid, acc[m]);
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) last_sh = atomicAdd(A.counters + tile, 1) == A.splits - 1;
+        __syncthreads();
+        if (last_sh) {
+            __threadfence();
+            if (row_ok) {
+                const float* base = A.partials + (int64_t)tile * A.splits * NP * kTCRows;
+                for (int m = 0; m < A.M; ++m) {
+                    float v = 0.f;
+                    for (int s = 0; s < A.splits; ++s) v += __ldcg(base + ((int64_t)s * NP + m) * kTCRows + tid);
+                    store(m, v);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+int tc_np(int M) { return (M + 15) / 16 * 16; }
+
+int tc_splits(int64_t N, int64_t K) {
+    const int64_t tiles = (N + kTCRows - 1) / kTCRows, G = K / kGroup;
+    int64_t s = (kTCTargetCtas + tiles / 2) / tiles;  // nearest to one wave of kTCTargetCtas
+    s = std::min<int64_t>(std::min<int64_t>(s, kTCMaxSplits), G);
+    return (int)std::max<int64_t>(s, 1);
+}
+
+size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+size_t tc_smem_bytes(int np) { return std::max(kTCMinSmem, (size_t)kTCStages * tc_group_bytes(np) + 1024); }
+
+template <int NP, int KIND>
+cudaError_t launch_tc_main(const TCArgs& A, cudaStream_t st) {
+    static bool ready[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const size_t smem = tc_smem_bytes(NP);
+    if (!ready[dev]) {
+        e = cudaFuncSetAttribute((const void*)k_gemm_tc<NP, KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        ready[dev] = true;
+    }
+    k_gemm_tc<NP, KIND><<<A.tiles * A.splits, kTCThreads, smem, st>>>(A);
+    return cudaGetLastError();
+}
+
+template <int KIND>
+cudaError_t launch_tc_np(const TCArgs& A, cudaStream_t st) {
+    switch (A.NP) {
+        case 16: return launch_tc_main<16, KIND>(A, st);
+        case 32: return launch_tc_main<32, KIND>(A, st);
+        case 48: return launch_tc_main<48, KIND>(A, st);
+        default: return launch_tc_main<64, KIND>(A, st);
+    }
+}
+
+}  // namespace
+
+size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    const int np = tc_np((int)M);
+    const int64_t tiles = (N + kTCRows - 1) / kTCRows, G = K / kGroup;
+    const int splits = tc_splits(N, K);
+    size_t b = align256((size_t)G * tc_group_bytes(np)) + align256((size_t)tiles * 4);
+    if (splits > 1) b += align256((size_t)tiles * splits * np * kTCRows * 4);
+    return b;
+}
+
+cudaError_t launch_gemm_tc(const void* packed, int grid, const uint16_t* scales, const uint16_t* X, int64_t ldx,
+                           void* Y, int ydt, int64_t ldy, int M, int64_t N, int64_t K, void* ws, cudaStream_t st) {
+    TCArgs A;
+    A.packed = static_cast<const uint8_t*>(packed);
+    A.scales = scales;
+    A.X = X;
+    A.Y = Y;
+    A.N = N;
+    A.K = K;
+    A.ldx = ldx;
+    A.ldy = ldy;
+    A.M = M;
+    A.NP = tc_np(M);
+    A.grid = grid;
+    A.ydt = ydt;
+    A.G = (int32_t)(K / kGroup);
+    A.tiles = (int32_t)((N + kTCRows - 1) / kTCRows);
+    A.splits = tc_splits(N, K);
+    char* w = static_cast<char*>(ws);
+    A.bprep = reinterpret_cast<uint8_t*>(w);
+    w += align256((size_t)A.G * tc_group_bytes(A.NP));
+    A.counters = reinterpret_cast<int32_t*>(w);
+    w += align256((size_t)A.tiles * 4);
+    A.partials = A.splits > 1 ? reinterpret_cast<float*>(w) : nullptr;
+    const int prep_warps = A.G * A.NP;
+    const int prep_ctas = std::max((prep_warps + 7) / 8, (A.tiles + 255) / 256);
+    k_prep_tc<<<prep_ctas, 256, 0, st>>>(A);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return grid == kInt3 ? launch_tc_np<1>(A, st) : launch_tc_np<0>(A, st);
+}
+
+unsigned int take_wait_timeouts() {
+    unsigned int v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_wait_timeouts, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+    if (cudaMemcpyToSymbol(g_wait_timeouts, &z, sizeof(z)) != cudaSuccess) return 0xFFFFFFFFu;
+    return v;
+}
+
+}  // namespace tb

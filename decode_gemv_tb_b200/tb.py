@@ -39,6 +39,7 @@ SIGNATURES = {
     "tb_gemm": (_I32, [_P, _I32, _P, _P, _I64, _P, _I32, _I64, _I64, _I64, _I64, _P, _SZ, _P]),
     "tb_layer_gemv": (_I32, [_P, _I32, ctypes.c_uint, _P, _SZ, _P]),
     "tb_gemv_noalloc": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I64, _P]),
+    "tb_wait_timeouts": (ctypes.c_uint, []),
 }
 
 
@@ -111,6 +112,11 @@ def _bits(t: torch.Tensor, name: str) -> int:
 
 
 # ---- sizes -----------------------------------------------------------------
+
+def wait_timeouts() -> int:
+    """Bounded device waits that gave up since the last call (synchronizes)."""
+    return int(load().tb_wait_timeouts())
+
 
 def version() -> int:
     return load().tb_version()

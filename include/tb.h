@@ -148,8 +148,12 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
 /* Scratch ("workspace") of the products below.  Each call first writes a
  * prepared copy of its activations (bf16, K per activation row, scaled by
  * powers of two) and per-128-group sums into the workspace, then reads them;
- * batch-1 calls also keep per-tile arrival counters and partial sums there
- * (tiles of K split between warps are combined in a fixed order).
+ * the calls also keep per-tile arrival counters and partial sums there
+ * (tiles whose K range is split are combined in a fixed order).  For
+ * M >= 32 (the tensor-core path) the size is exact and device independent:
+ *   ceil256(K/128 * NP * 264) + ceil256(4 * T) + [S > 1] ceil256(T * S * NP * 512)
+ * with NP = M rounded up to 16, T = ceil(N / 128) and S = the K split,
+ * max(1, min(floor((296 + T/2) / T), 16, K / 128)).
  *   - device memory, 256-byte aligned, at least the size returned here;
  *   - owned by the caller, written by every call: two calls that share a
  *     workspace must be ordered (e.g. the same stream);
@@ -174,6 +178,14 @@ TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *s
 TB_API tb_status_t tb_gemm(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *X,
                            int64_t ldx, void *Y, tb_dtype_t y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
                            void *workspace, size_t workspace_bytes, tb_stream_t stream);
+
+/* Diagnostic: how many bounded device-side waits gave up since the last
+ * call, on the current device (the count is then cleared).  The kernels
+ * that wait on the tensor-core pipeline give up after about two seconds,
+ * write NaN to their outputs and return; a nonzero count means such a
+ * launch produced no result.  Synchronizes with the device; returns
+ * 0xFFFFFFFF if the count cannot be read. */
+TB_API unsigned int tb_wait_timeouts(void);
 
 /* One linear layer of a grouped launch. */
 typedef struct {

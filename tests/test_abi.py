@@ -24,7 +24,8 @@ def lib():
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"^\s*TB_API\s+(?:const\s+)?[a-z_0-9]+\s*\*?\s*(tb_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    names = re.findall(r"^\s*TB_API\s+(?:(?:const|unsigned|signed)\s+)*[a-z_0-9]+\s*\*?\s*(tb_[a-z_0-9]+)\s*\(", src,
+                       flags=re.M)
     return sorted(set(names))
 
 
@@ -65,10 +66,18 @@ FAKE = 1 << 40  # a 256-byte-aligned address that is never dereferenced
 
 def test_workspace_sizes(lib):
     al = lambda b: (b + 255) // 256 * 256
-    for M, N, K in ((4, 100, 5120), (16, 17408, 17408), (64, 7, 1024)):
-        # prepared activations (2 bytes per element) + per-group pairs (8 bytes), each 256-byte aligned
+    for M, N, K in ((4, 100, 5120), (16, 17408, 17408), (17, 7, 1024)):
+        # M below the tensor-core threshold (32): prepared activations (2 bytes per element) + per-group
+        # pairs (8 bytes) of up to 16 batch rows, each 256-byte aligned
         Mb = min(M, 16)
         assert tb.workspace_bytes(M, N, K) == al(2 * Mb * K) + al(8 * Mb * (K // 128))
+    for M, N, K in ((32, 100, 5120), (33, 17408, 5120), (64, 7, 1024), (64, 40000, 4096)):
+        # tensor-core path: per group NP rows of prepared X (256 bytes) and NP pairs (8 bytes), NP = M
+        # rounded up to 16; a counter per 128-row tile; K-split partials of NP x 128 fp32 per tile and split
+        NP, tiles, G = (M + 15) // 16 * 16, (N + 127) // 128, K // 128
+        splits = max(1, min((296 + tiles // 2) // tiles, 16, G))
+        want = al(G * NP * 264) + al(4 * tiles) + (al(tiles * splits * NP * 128 * 4) if splits > 1 else 0)
+        assert tb.workspace_bytes(M, N, K) == want, (M, N, K)
     for N, K in ((1, 128), (256, 1024), (17408, 5120)):
         # batch 1 adds a counter per 32-row tile and two 32-float slots per warp
         tiles = (N + 31) // 32

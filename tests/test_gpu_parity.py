@@ -254,6 +254,50 @@ def test_gemm_strided_bf16_out(oracle):
     assert torch.all(Ybuf[:, N:] == 0)
 
 
+@pytest.mark.parametrize("grid", GRIDS)
+@pytest.mark.parametrize("M", [16, 33, 64])
+def test_gemm_multi_tile_split(oracle, grid, M):
+    """Several 128-row tiles, a ragged last tile and a 16-way K split."""
+    N, K = 300, 2048
+    W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=1100 + M + grid)
+    X = synth.activations(K, seed=1200 + M, M=M)
+    Y64, Yabs = oracle.gemm64(p_ref, grid, s_ref, u16(X), N, K)
+    Y = tb.tb_gemm(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), X.to(DEV), N, K)
+    assert_within(Y, Y64, Yabs, "f32", oracle, f"gemm tiles M={M}")
+    assert tb.wait_timeouts() == 0
+
+
+@pytest.mark.parametrize("grid", [tb.INT2, tb.INT3])
+def test_gemm_no_split(oracle, grid):
+    """Enough tiles that every CTA covers the whole K range (no K split)."""
+    N, K, M = 296 * 128, 256, 20
+    W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=1300 + grid)
+    X = synth.activations(K, seed=1301, M=M)
+    Y64, Yabs = oracle.gemm64(p_ref, grid, s_ref, u16(X), N, K)
+    Y = tb.tb_gemm(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), X.to(DEV), N, K, out_dtype=torch.bfloat16)
+    assert_within(Y, Y64, Yabs, "bf16", oracle, "gemm no split")
+    assert tb.wait_timeouts() == 0
+
+
+@pytest.mark.parametrize("grid", [tb.INT2, tb.INT3])
+@pytest.mark.parametrize("M", [4, 16, 64])
+def test_gemm_config4_gate_sampled(oracle, grid, M):
+    """Qwen3-14B-like gate projection (17408 x 5120) at full size, in the
+    launch configuration the benchmark times; 96 sampled rows per batch row
+    (tile and split boundaries included) against the oracle."""
+    N, K = 17408, 5120
+    W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=4000 + grid)
+    X = synth.activations(K, seed=4100 + M, M=M)
+    Y = tb.tb_gemm(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), X.to(DEV), N, K).cpu()
+    rng = np.random.default_rng(M + 10 * grid)
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 129, N - 128, N - 1], rng.integers(0, N, 90)]))
+    Xb = u16(X)
+    for m in range(M):
+        y64, yabs = oracle.gemv_rows64(p_ref, grid, s_ref, Xb[m], K, rows)
+        assert_within(Y[m, rows], y64, yabs, "f32", oracle, f"gate M={M} m={m}")
+    assert tb.wait_timeouts() == 0
+
+
 # ------------------------------------------------------------------ activations
 
 def _x_case(kind, K, seed):
