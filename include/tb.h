@@ -151,7 +151,8 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
  * the calls also keep per-tile arrival counters and partial sums there
  * (tiles whose K range is split are combined in a fixed order).  For
  * M >= 32 (the tensor-core path) the size is exact and device independent:
- *   ceil256(K/128 * NP * 264) + ceil256(4 * T) + [S > 1] ceil256(T * S * NP * 512)
+ *   ceil256(K/128 * NP * 264) + ceil256(T * K/128 * 256) + ceil256(4 * T)
+ *     + [S > 1] ceil256(T * S * NP * 512)
  * with NP = M rounded up to 16, T = ceil(N / 128) and S = the K split,
  * max(1, min(floor((296 + T/2) / T), 16, K / 128)).
  *   - device memory, 256-byte aligned, at least the size returned here;
