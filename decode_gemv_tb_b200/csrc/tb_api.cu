@@ -67,12 +67,8 @@ size_t item_workspace(int64_t M, int64_t K) {
 
 // Batch-1 launches additionally need one counter per 32-row tile and two
 // 32-float partial-sum slots per warp (at most kMaxSKWarps warps, and never
-// more warps than tile-groups).
+// more warps than chunks).
 constexpr int64_t kMaxSKWarps = 8192;
-size_t sk_extra_workspace(int64_t tiles, int64_t tile_groups) {
-    const int64_t w = std::min(kMaxSKWarps, std::max<int64_t>(tile_groups, 1));
-    return align256((size_t)(tiles * 4)) + align256((size_t)(w * 2 * 32 * 4));
-}
 
 // batch sizes from which tb_gemm runs on the tcgen05 path
 constexpr int64_t kTCMinM = 32;
@@ -150,13 +146,22 @@ tb_status_t launch_items(Item* items, int n, int nt, void* ws, size_t ws_bytes, 
     return cuda_status(launch_linear(L, nt, (int)ctas, (int)prep, overlap, st));
 }
 
-// Batch-1 (M == 1) launch: preparation kernel + stream-K kernel.  3-bit
-// items form the first partition, 2-bit items the second (each warp works
-// on one code width only); warps are split between them by cost.
-tb_status_t launch_sk_items(const Item* items, int n, void* ws, size_t ws_bytes, bool overlap, cudaStream_t st) {
+// Batch-1 (M == 1) launch: preparation kernel + k_gemv_tma.  Each item's
+// activations become G records of kRecBytes; 3-bit items form the first
+// partition, 2-bit items the second (each warp works on one code width
+// only); warps are split between them by cost.  Chunks are C = 2 (3-bit) or
+// 4 (2-bit) groups of one 32-row tile.
+int tm_chunk_groups(int grid) { return grid == TB_GRID_INT3 ? 2 : 4; }
+size_t tm_item_workspace(int64_t K) { return align256((size_t)(K / kGroup) * kRecBytes); }
+size_t tm_extra_workspace(int64_t tiles, int64_t chunks) {
+    const int64_t w = std::min(kMaxSKWarps, std::max<int64_t>(chunks, 1));
+    return align256((size_t)(tiles * 4)) + align256((size_t)(w * 2 * 32 * 4));
+}
+
+tb_status_t launch_tma_items(const Item* items, int n, void* ws, size_t ws_bytes, bool overlap, cudaStream_t st) {
     Launch P;
     std::memset(&P, 0, sizeof(P));
-    SKLaunch L;
+    TMLaunch L;
     std::memset(&L, 0, sizeof(L));
     int order[kMaxItems], n3 = 0;
     for (int i = 0; i < n; ++i)
@@ -165,70 +170,70 @@ tb_status_t launch_sk_items(const Item* items, int n, void* ws, size_t ws_bytes,
         if (items[i].grid != TB_GRID_INT3) order[k++] = i;
     char* w = static_cast<char*>(ws);
     size_t need = 0;
-    int64_t prep = 0, tiles = 0, tg_all = 0;
-    int64_t tg = 0, cost = 0, part_cost[2] = {0, 0};
+    int64_t prep = 0, tiles = 0, chunks_all = 0, chunk = 0, cost = 0, part_cost[2] = {0, 0};
     for (int j = 0; j < n; ++j) {
-        if (j == n3) tg = cost = 0;  // the 2-bit partition starts its positions again
+        if (j == n3) chunk = cost = 0;  // the 2-bit partition starts its positions again
         Item it = items[order[j]];
         it.prep_begin = (int32_t)prep;
-        it.xs = reinterpret_cast<uint16_t*>(w + need);
-        it.cf = reinterpret_cast<float2*>(w + need + align256((size_t)(it.K * 2)));
-        need += item_workspace(1, it.K);
+        it.rec = reinterpret_cast<uint8_t*>(w + need);
+        need += tm_item_workspace(it.K);
         prep += it.K / kGroup;
         P.it[j] = it;
 
-        SKItem& s = L.it[j];
-        s.packed = it.packed;
+        TMItem& s = L.it[j];
         s.scales = it.scales;
-        s.xs = it.xs;
-        s.cf = it.cf;
+        s.rec = it.rec;
         s.Y = it.Y;
         s.N = it.N;
-        s.K = it.K;
-        s.rbytes = row_bytes(it.grid, it.K);
         s.G = (int32_t)(it.K / kGroup);
         s.T = (int32_t)((it.N + 31) / 32);
+        s.C = tm_chunk_groups(it.grid);
+        s.cpt = (s.G + s.C - 1) / s.C;
+        s.unit_cost = it.grid == TB_GRID_INT3 ? 3 : 2;
         s.grid = it.grid;
         s.ydt = it.ydt;
-        s.unit_cost = it.grid == TB_GRID_INT3 ? 3 : 2;
-        s.tg_base = tg;
-        s.tg_count = (int64_t)s.T * s.G;
+        s.chunk_base = chunk;
         s.cost_base = cost;
         s.tile_base = (int32_t)tiles;
-        tg += s.tg_count;
-        tg_all += s.tg_count;
-        cost += s.tg_count * s.unit_cost;
+        chunk += (int64_t)s.T * s.cpt;
+        chunks_all += (int64_t)s.T * s.cpt;
+        cost += (int64_t)s.T * s.G * s.unit_cost;
         part_cost[j < n3 ? 0 : 1] = cost;
         tiles += s.T;
     }
     P.n_items = n;
     L.n_items = n;
-    if (part_cost[0] >= ((int64_t)1 << 31) || part_cost[1] >= ((int64_t)1 << 31))
+    if (part_cost[0] >= ((int64_t)1 << 31) || part_cost[1] >= ((int64_t)1 << 31) || chunks_all >= ((int64_t)1 << 31))
         return TB_ERR_UNSUPPORTED;  // partition arithmetic is 32-bit
     // layout with the device-independent bound on the warp count (the one
     // tb_workspace_bytes uses), checked before any CUDA call
     L.counters = reinterpret_cast<int32_t*>(w + need);
     L.partials = reinterpret_cast<float*>(w + need + align256((size_t)(tiles * 4)));
-    need += sk_extra_workspace(tiles, tg_all);
+    need += tm_extra_workspace(tiles, chunks_all);
     P.zero = L.counters;
     P.n_zero = (int32_t)tiles;
     if (!ws || ws_bytes < need) return TB_ERR_ARG;
     if (tiles > 0x7FFFFFFF || prep > 0x7FFFFFFF) return TB_ERR_SHAPE;
-    const int resident = gemv_sk_resident_warps();
+    for (int j = 0; j < n; ++j)
+        if (!encode_gemv_tma_map(&L.maps[j], P.it[j].packed, P.it[j].grid, P.it[j].N, P.it[j].K)) return TB_ERR_CUDA;
+    const int resident = gemv_tma_resident_warps();
     if (resident <= 0) return TB_ERR_CUDA;
-    // at most the resident warps; at least about four tile-groups per warp
-    const int64_t W = std::max<int64_t>(1, std::min<int64_t>({(int64_t)resident, (tg_all + 3) / 4, kMaxSKWarps}));
+    const int64_t W = std::max<int64_t>(1, std::min<int64_t>({(int64_t)resident, chunks_all, kMaxSKWarps}));
     const int64_t C = part_cost[0] + part_cost[1];
     int64_t W3 = part_cost[0] == 0 ? 0 : (part_cost[1] == 0 ? W : (W * part_cost[0] + C / 2) / C);
     if (part_cost[0] > 0) W3 = std::max<int64_t>(W3, 1);
     if (part_cost[1] > 0) W3 = std::min<int64_t>(W3, W - 1);
-    const int64_t W2 = W - W3;
-    L.W = (int32_t)W;
+    int64_t W2 = W - W3;
+    // each quota at least one chunk's cost (3-bit: 2 x 3, 2-bit: 4 x 2): then every warp between a
+    // tile's first and last owner owns a chunk of it, which the partial-sum combine relies on
+    if (W3 > 0) W3 = std::max<int64_t>(1, std::min<int64_t>(W3, part_cost[0] / 6));
+    if (W2 > 0) W2 = std::max<int64_t>(1, std::min<int64_t>(W2, part_cost[1] / 8));
+    L.W = (int32_t)(W3 + W2);
     L.part[0] = {0, n3, 0, (int32_t)W3, (uint32_t)part_cost[0],
                  (uint32_t)(W3 ? (part_cost[0] + W3 - 1) / W3 : 1)};
     L.part[1] = {n3, n - n3, (int32_t)W3, (int32_t)W2, (uint32_t)part_cost[1],
                  (uint32_t)(W2 ? (part_cost[1] + W2 - 1) / W2 : 1)};
-    return cuda_status(launch_gemv_sk(P, (int)prep, L, (int)((W + 7) / 8), overlap, st));
+    return cuda_status(launch_gemv_tma(P, (int)prep, L, (int)((L.W + 7) / 8), overlap, st));
 }
 
 }  // namespace
@@ -237,7 +242,10 @@ extern "C" {
 
 int tb_version(void) { return 100; }
 
-unsigned int tb_wait_timeouts(void) { return take_wait_timeouts(); }
+unsigned int tb_wait_timeouts(void) {
+    const unsigned int a = take_wait_timeouts(), b = take_gemv_timeouts();
+    return (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) ? 0xFFFFFFFFu : a + b;
+}
 
 const char* tb_status_string(tb_status_t s) {
     switch (s) {
@@ -289,9 +297,9 @@ tb_status_t tb_unpack(const void* packed, tb_grid_t grid, int64_t N, int64_t K, 
 
 size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (M < 1 || M > 64 || !shape_ok(N, K)) return 0;
-    if (M == 1) {
+    if (M == 1) {  // chunk count bounded with the smaller chunk (two groups)
         const int64_t tiles = (N + 31) / 32;
-        return item_workspace(1, K) + sk_extra_workspace(tiles, tiles * (K / kGroup));
+        return tm_item_workspace(K) + tm_extra_workspace(tiles, tiles * ((K / kGroup + 1) / 2));
     }
     if (M >= kTCMinM) return gemm_tc_workspace_bytes(M, N, K);
     return item_workspace(std::min<int64_t>(M, 16), K);
@@ -300,14 +308,15 @@ size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 size_t tb_layer_workspace_bytes(const tb_linear_t* items, int n_items) {
     if (!items || n_items < 1 || n_items > TB_MAX_LAYER_ITEMS) return 0;
     size_t b = 0;
-    int64_t tiles = 0, tgs = 0;
+    int64_t tiles = 0, chunks = 0;
     for (int i = 0; i < n_items; ++i) {
-        if (!shape_ok(items[i].N, items[i].K)) return 0;
-        b += item_workspace(1, items[i].K);
-        tiles += (items[i].N + 31) / 32;
-        tgs += (items[i].N + 31) / 32 * (items[i].K / kGroup);
+        if (!shape_ok(items[i].N, items[i].K) || !grid_ok(items[i].grid)) return 0;
+        const int64_t t = (items[i].N + 31) / 32, C = tm_chunk_groups(items[i].grid);
+        b += tm_item_workspace(items[i].K);
+        tiles += t;
+        chunks += t * ((items[i].K / kGroup + C - 1) / C);
     }
-    return b + sk_extra_workspace(tiles, tgs);
+    return b + tm_extra_workspace(tiles, chunks);
 }
 
 tb_status_t tb_gemv(const void* packed, tb_grid_t grid, const uint16_t* scales, const uint16_t* x, void* y,
@@ -320,7 +329,7 @@ tb_status_t tb_gemv(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if (!workspace) return TB_ERR_ARG;
     if (!aligned(x, 16) || !aligned(workspace, 256)) return TB_ERR_ALIGN;
     Item it = make_item(packed, grid, scales, x, K, y, y_dtype, N, 1, N, K);
-    return launch_sk_items(&it, 1, workspace, workspace_bytes, false, static_cast<cudaStream_t>(stream));
+    return launch_tma_items(&it, 1, workspace, workspace_bytes, false, static_cast<cudaStream_t>(stream));
 }
 
 tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, const uint16_t* X, int64_t ldx,
@@ -336,7 +345,7 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (M == 1) {
         Item it = make_item(packed, grid, scales, X, ldx, Y, y_dtype, N, 1, N, K);
-        return launch_sk_items(&it, 1, workspace, workspace_bytes, false, st);
+        return launch_tma_items(&it, 1, workspace, workspace_bytes, false, st);
     }
     if (M >= kTCMinM) {
         if (workspace_bytes < gemm_tc_workspace_bytes(M, N, K)) return TB_ERR_ARG;
@@ -369,7 +378,7 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
         if (!aligned(l.x, 16)) return TB_ERR_ALIGN;
         its[i] = make_item(l.packed, l.grid, l.scales, l.x, l.K, l.y, l.y_dtype, l.N, 1, l.N, l.K);
     }
-    return launch_sk_items(its, n_items, workspace, workspace_bytes, (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0,
+    return launch_tma_items(its, n_items, workspace, workspace_bytes, (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0,
                            static_cast<cudaStream_t>(stream));
 }
 
@@ -426,7 +435,7 @@ tb_status_t tb_gemv_noalloc(const void* packed, tb_grid_t grid, const uint16_t* 
     void* scratch = noalloc_scratch();
     if (!scratch) return TB_ERR_CUDA;
     Item it = make_item(packed, grid, scales, x, K, y, y_dtype, N, 1, N, K);
-    return launch_sk_items(&it, 1, scratch, TB_NOALLOC_SCRATCH_BYTES, false, static_cast<cudaStream_t>(stream));
+    return launch_tma_items(&it, 1, scratch, TB_NOALLOC_SCRATCH_BYTES, false, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

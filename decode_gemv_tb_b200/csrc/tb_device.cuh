@@ -7,6 +7,7 @@
 // onedev.kr/papers/1416, section 어떻게 동작하나).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -38,7 +39,15 @@ struct Item {
     int32_t cta_begin;   // first CTA of this item in the main launch
     int32_t prep_begin;  // first warp of this item in the preparation launch
     int32_t ksplit;      // warps sharing one 32-row tile (1, 2, 4 or 8)
+    uint8_t* rec;        // batch-1 TMA path: per-group records (see kRecBytes) instead of xs / cf
 };
+
+// Prepared activations of one 128-group for the batch-1 TMA kernel, one
+// contiguous record: the 128 scaled activations in MMA order, first half at
+// bytes 0..127, (offset * sum x, 2^S) at 128..135, zero at 136..143, second
+// half at 144..271 (the 16-byte gap keeps the fragment loads free of bank
+// conflicts).  A chunk of consecutive groups is one bulk copy.
+constexpr int kRecBytes = 272;
 
 struct Launch {
     Item it[kMaxItems];
@@ -77,6 +86,27 @@ struct SKLaunch {
     SKPart part[2];       // [0]: 3-bit items, [1]: 2-bit items
     int32_t* counters;    // one per 32-row tile, zeroed by the preparation kernel
     float* partials;      // [W][2][32]
+};
+
+// Batch-1 TMA kernel (tb_linear.cu): items read in chunks of C groups x 32
+// rows through one 2-D tensor map each (see tb_partition.h, ChunkItem).
+struct TMItem {
+    const uint16_t* scales;
+    const uint8_t* rec;  // G records of kRecBytes
+    void* Y;
+    int64_t N;
+    int64_t chunk_base, cost_base;  // ChunkItem fields
+    int32_t T, G, C, cpt, unit_cost;
+    int32_t grid, ydt, tile_base;
+};
+
+struct TMLaunch {
+    CUtensorMap maps[kMaxItems];  // packed weights of item i: bytes x rows, box (C group bytes) x 32
+    TMItem it[kMaxItems];
+    int32_t n_items, W;
+    SKPart part[2];  // 3-bit items first, then the 2-bit container
+    int32_t* counters;
+    float* partials;
 };
 
 // ---- cache-controlled loads ----------------------------------------------

@@ -1,6 +1,7 @@
 // tb_internal.h -- launchers behind the C interface (host side).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -29,6 +30,18 @@ cudaError_t launch_gemv_sk(const Launch& P, int prep_warps, const SKLaunch& L, i
                            cudaStream_t st);
 // warps of the stream-K kernel resident at once on the current device (0 on error)
 int gemv_sk_resident_warps();
+
+struct TMLaunch;
+// Batch-1 path with TMA staging: preparation kernel (writes records, clears
+// P.zero) + k_gemv_tma.  The tensor map of each item comes from
+// encode_gemv_tma_map (false if the driver cannot encode it).
+cudaError_t launch_gemv_tma(const Launch& P, int prep_warps, const TMLaunch& L, int ctas, bool overlap,
+                            cudaStream_t st);
+bool encode_gemv_tma_map(CUtensorMap* map, const void* packed, int grid, int64_t N, int64_t K);
+// warps of k_gemv_tma resident at once on the current device (0 on error)
+int gemv_tma_resident_warps();
+// bounded waits of k_gemv_tma that gave up since the last call (clears)
+unsigned int take_gemv_timeouts();
 
 // Small-batch GEMM on the tcgen05 tensor cores (2 <= M <= 64): preparation
 // kernel + main kernel.  Workspace: gemm_tc_workspace_bytes(M, N, K) bytes,

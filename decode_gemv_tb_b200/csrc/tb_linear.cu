@@ -167,11 +167,16 @@ __global__ void __launch_bounds__(kThreads) k_prep(const __grid_constant__ Launc
         const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(v));  // exact: 8 significant bits
         out[j >> 1] |= b << (16 * (j & 1));
     }
-    *reinterpret_cast<uint2*>(I.xs + (int64_t)m * K + grp * kGroup + 4 * lane) = make_uint2(out[0], out[1]);
-    if (lane == 0) {
-        const float off = grid == kInt3 ? 4.f : 2.f;
-        I.cf[grp * M + m] = make_float2(off * sum, __int_as_float((S + 127) << 23));
+    const float off = grid == kInt3 ? 4.f : 2.f;
+    if (I.rec) {  // batch-1 record (M == 1)
+        uint8_t* rec = I.rec + grp * kRecBytes;
+        *reinterpret_cast<uint2*>(rec + 8 * lane + (lane >= 16 ? 16 : 0)) = make_uint2(out[0], out[1]);
+        if (lane == 0)
+            *reinterpret_cast<float4*>(rec + 128) = make_float4(off * sum, __int_as_float((S + 127) << 23), 0.f, 0.f);
+        return;
     }
+    *reinterpret_cast<uint2*>(I.xs + (int64_t)m * K + grp * kGroup + 4 * lane) = make_uint2(out[0], out[1]);
+    if (lane == 0) I.cf[grp * M + m] = make_float2(off * sum, __int_as_float((S + 127) << 23));
 }
 
 // ---------------------------------------------------------------------------
@@ -843,6 +848,369 @@ __global__ void __launch_bounds__(kThreads, 2) k_gemv_sk(const __grid_constant__
 
 size_t gemv_sk_smem_bytes() { return (size_t)kWarps * kSKWarpB; }
 
+// ---------------------------------------------------------------------------
+// Batch-1 kernel with TMA staging (k_gemv_tma).
+//
+// Reading 32 rows x 32 bytes per warp with per-lane 16-byte copies leaves
+// each load instruction touching 32 cache lines for 16 to 32 bytes apiece:
+// on B200 that access pattern tops out near 4.5 TB/s however it is issued
+// from the SM.  Here lane 0 of each warp instead issues one 2-D tensor copy
+// per chunk -- 32 rows x 128 bytes (four 2-bit groups, 128-byte swizzled) or
+// 32 rows x 96 bytes (two 3-bit groups) -- plus one bulk copy of the chunk's
+// prepared activation records, into a two-stage ring; both complete on the
+// stage's mbarrier.  The per-group arithmetic is that of k_gemv_sk.
+constexpr int kTMStageB = 6144;                // weights box (<= 4 KB) + records (<= 4 x 272 B)
+constexpr int kTMRec = 4096;                   // offset of the records in a stage
+constexpr int kTMWarpB = 2 * kTMStageB;        // two stages per warp
+constexpr int kTMSmem = kWarps * kTMWarpB + 1024;  // + alignment slack (swizzled boxes need 1 KB alignment)
+constexpr long long kTMWaitCycles = 4000000000LL;  // about 2 s
+
+__device__ unsigned int g_tm_timeouts = 0;  // bounded waits of k_gemv_tma that gave up
+
+__device__ __forceinline__ void tm_bar_init(uint32_t bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tm_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// all lanes wait; true when the phase completed, false (counted) after about kTMWaitCycles
+__device__ __forceinline__ bool tm_wait(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (clock64() - t0 > kTMWaitCycles) {
+            atomicAdd(&g_tm_timeouts, 1u);
+            return false;
+        }
+    }
+}
+// 2-D tiled tensor copy (no multicast): box at (x bytes, y rows) of map -> dst
+__device__ __forceinline__ void tm_load_box(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+// 1-D bulk copy (no multicast)
+__device__ __forceinline__ void tm_load_bulk(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+// One group gi of a chunk held in stage: 32 rows x 128 codes, two 16-row MMA
+// tiles, as sk_step.  Weights: 2-bit rows are 128 bytes, 128-byte swizzled
+// (16-byte unit u of row r at unit u ^ (r & 7)); 3-bit rows are 96 bytes.
+template <int KIND>
+__device__ __forceinline__ void tm_step(const uint8_t* stage, int gi, uint32_t srow, int g, int t, float (&acc)[4]) {
+    float d[2][4];
+    bool first = true;  // the first MMA of each chain starts from zero
+    auto mma = [&](int rt, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+        if (first) mma16816_z(d[rt], a0, a1, a2, a3, b0, b1);
+        else mma16816(d[rt], a0, a1, a2, a3, b0, b1);
+    };
+    const uint8_t* rec = stage + kTMRec + gi * kRecBytes;
+    auto xfrag = [&](int q) {  // B fragment: codes 32 t + 8 q .. + 7 of the group
+        const int c = 4 * t + q;
+        return *reinterpret_cast<const uint4*>(rec + 16 * c + (c >= 8 ? 16 : 0));
+    };
+    if (KIND == 0) {
+        uint2 wv[4];
+        // row g + 8 q, bytes 32 gi + 8 t .. + 7: 16-byte unit 2 gi + t / 2, swizzled by (g + 8 q) & 7 = g
+        const int off = (((2 * gi + (t >> 1)) ^ g) << 4) + 8 * (t & 1);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) wv[q] = *reinterpret_cast<const uint2*>(stage + (g + 8 * q) * 128 + off);
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            const uint4 xv0 = xfrag(2 * w), xv1 = xfrag(2 * w + 1);
+            uint32_t W[4], H[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                W[q] = w ? wv[q].y : wv[q].x;
+                H[q] = shr_fma(W[q], 8);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t m0 = 0x00030003u << (4 * (r & 1)), m1 = 0x000C000Cu << (4 * (r & 1));
+                const uint4 v = (r >> 1) ? xv1 : xv0;
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt) {
+                    const uint32_t A = r < 2 ? W[2 * rt] : H[2 * rt], B = r < 2 ? W[2 * rt + 1] : H[2 * rt + 1];
+                    mma(rt, A & m0, B & m0, A & m1, B & m1, (r & 1) ? v.z : v.x, (r & 1) ? v.w : v.y);
+                }
+                first = false;
+            }
+        }
+    } else {
+        uint4 xv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xv[q] = xfrag(q);
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt) {
+            uint32_t P[2][3];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int p = 0; p < 3; ++p)
+                    P[h][p] = *reinterpret_cast<const uint32_t*>(stage + (g + 8 * (2 * rt + h)) * 96 + 48 * gi + 12 * t +
+                                                                 4 * p);
+            uint32_t q1[2], q2[2], zA[2], zB[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                q1[h] = P[h][1] << 1;
+                q2[h] = P[h][2] << 2;
+                zA[h] = bit_mux(bit_mux(P[h][0], q1[h], bits_at(0, 5, 1)), q2[h], bits_at(0, 5, 2));
+                zB[h] = bit_mux(bit_mux(P[h][0], q1[h], bits_at(1, 5, 1)), q2[h], bits_at(1, 5, 2));
+            }
+            bool first3 = true;
+            auto emit = [&](int r, const uint32_t (&fa)[2], uint32_t ma, const uint32_t (&fb)[2], uint32_t mb) {
+                const uint4 v = xv[r >> 1];
+                if (first3) mma16816_z(d[rt], fa[0] & ma, fa[1] & ma, fb[0] & mb, fb[1] & mb, (r & 1) ? v.z : v.x,
+                                       (r & 1) ? v.w : v.y);
+                else mma16816(d[rt], fa[0] & ma, fa[1] & ma, fb[0] & mb, fb[1] & mb, (r & 1) ? v.z : v.x,
+                              (r & 1) ? v.w : v.y);
+                first3 = false;
+            };
+            emit(0, zA, 0x00070007u, zB, 0x000E000Eu);
+            emit(1, zA, 0x00380038u, zB, 0x00700070u);
+            uint32_t sA[2], sB[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                sA[h] = shr_fma(zA[h], 6);
+                sB[h] = shr_fma(zB[h], 6);
+            }
+            emit(2, sA, 0x00070007u, sB, 0x000E000Eu);
+            emit(3, sA, 0x00380038u, sB, 0x00700070u);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                sA[h] = shr_fma(zA[h], 12);
+                sB[h] = shr_fma(zB[h], 12);
+            }
+            emit(4, sA, 0x00070007u, sB, 0x000E000Eu);
+            uint32_t zC[2], zC6[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                zC[h] = bit_mux(bit_mux(P[h][0], q1[h], bits_at(2, 4, 1)), q2[h], bits_at(2, 4, 2));
+                zC6[h] = shr_fma(zC[h], 6);
+            }
+            emit(5, zC, 0x001C001Cu, zC, 0x00E000E0u);
+            emit(6, zC6, 0x001C001Cu, zC6, 0x00E000E0u);
+            uint32_t z14[2], z15[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t r0 = shr_fma(P[h][0], 14), r1 = shr_fma(P[h][1], 13), r2 = shr_fma(P[h][2], 12);
+                z14[h] = bit_mux(bit_mux(r0, r1, 0x00020002u), r2, 0x00040004u);
+                z15[h] = bit_mux(bit_mux(r0, r1, 0x00040004u), r2, 0x00080008u);
+            }
+            emit(7, z14, 0x00070007u, z15, 0x000E000Eu);
+        }
+    }
+    const float2 c = *reinterpret_cast<const float2*>(rec + 128);
+    float sc[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) sc[q] = bf16_bits_to_float(__shfl_sync(0xffffffffu, srow, g + 8 * q));
+#pragma unroll
+    for (int rt = 0; rt < 2; ++rt) {
+        acc[2 * rt] = fmaf(sc[2 * rt], fmaf(c.y, d[rt][0], -c.x), acc[2 * rt]);
+        acc[2 * rt + 1] = fmaf(sc[2 * rt + 1], fmaf(c.y, d[rt][2], -c.x), acc[2 * rt + 1]);
+    }
+}
+
+// End of a warp's segment of a tile: write y, or hand the partial sums over
+// and combine them if this warp arrives last (as sk_flush; the contributors
+// are the owners of the tile's first and last chunk start -- every warp in
+// between owns at least one chunk start because the launcher keeps the
+// quota at least one chunk's cost).
+__device__ __noinline__ void tm_flush(const TMLaunch& L, int part, int64_t wg, int item, uint32_t tile, bool whole,
+                                      bool first_seg, float v0, float v1, float v2, float v3) {
+    const TMItem& I = L.it[item];
+    const SKPart& P = L.part[part];
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int64_t row0 = (int64_t)tile * kRows;
+    const float v[4] = {v0, v1, v2, v3};
+    if (whole) {
+        if (t == 0) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int64_t row = row0 + g + 8 * q;
+                if (row < I.N) {
+                    if (I.ydt == kF32) static_cast<float*>(I.Y)[row] = v[q];
+                    else static_cast<__nv_bfloat16*>(I.Y)[row] = __float2bfloat16_rn(v[q]);
+                }
+            }
+        }
+        return;
+    }
+    float* mine = L.partials + (wg * 2 + (first_seg ? 0 : 1)) * kRows;
+    if (t == 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) __stcg(mine + g + 8 * q, v[q]);
+    }
+    __threadfence();
+    __syncwarp();
+    const uint32_t uc = (uint32_t)I.unit_cost;
+    const uint32_t pA = (uint32_t)I.cost_base + tile * (uint32_t)I.G * uc;
+    const uint32_t pZ = pA + (uint32_t)(I.cpt - 1) * (uint32_t)I.C * uc;
+    const uint32_t w0 = part_owner(pA, P.Q), w1 = part_owner(pZ, P.Q);
+    int last = 0;
+    if (lane == 0) last = atomicAdd(L.counters + I.tile_base + tile, 1) == (int)(w1 - w0);
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
+    __threadfence();
+    const uint32_t cA = (uint32_t)I.chunk_base + tile * (uint32_t)I.cpt;
+    float sum = 0.f;
+    for (uint32_t w = w0; w <= w1; ++w) {
+        // a warp that starts inside this tile has it as its first segment (slot 0), an earlier one
+        // as its last (slot 1)
+        const uint32_t wb = part_first_chunk(L.it + P.first, P.count, w * P.Q);
+        sum += __ldcg(L.partials + ((int64_t)(P.W0 + w) * 2 + (wb >= cA ? 0 : 1)) * kRows + lane);
+    }
+    const int64_t row = row0 + lane;
+    if (row < I.N) {
+        if (I.ydt == kF32) static_cast<float*>(I.Y)[row] = sum;
+        else static_cast<__nv_bfloat16*>(I.Y)[row] = __float2bfloat16_rn(sum);
+    }
+}
+
+// One warp of k_gemv_tma for code width KIND (0: 2-bit container, 1: 3-bit).
+template <int KIND>
+__device__ __forceinline__ void tm_warp(const TMLaunch& L, int part, uint32_t w, int64_t wg, uint8_t* base,
+                                        uint64_t* bars) {
+    constexpr int C = KIND ? 2 : 4;         // groups per chunk
+    constexpr int WB = C * (KIND ? 48 : 32);  // box width in bytes: 96 or 128
+    const SKPart& P = L.part[part];
+    const TMItem* items = L.it + P.first;
+    const CUtensorMap* maps = L.maps + P.first;
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    uint32_t cb, ce;
+    part_chunk_range(items, P.count, w, P.Q, P.C, &cb, &ce);
+    if (cb >= ce) return;
+    const int32_t n = (int32_t)(ce - cb);
+    const uint32_t base_s = smem_u32(base);
+    const uint32_t bar0 = smem_u32(bars), bar1 = bar0 + 8;
+
+    // ---- locate the first chunk
+    int c_item = 0;
+    for (int i = 1; i < P.count; ++i)
+        if (cb >= (uint32_t)items[i].chunk_base) c_item = i;
+    uint32_t c_tile;
+    int32_t c_j;
+    {
+        const uint32_t local = cb - (uint32_t)items[c_item].chunk_base, cpt = (uint32_t)items[c_item].cpt;
+        c_tile = local / cpt;
+        c_j = (int32_t)(local - c_tile * cpt);
+    }
+
+    // ---- issue cursor: lane 0 copies, every lane loads its row's scales
+    int i_item = c_item;
+    uint32_t i_tile = c_tile;
+    int32_t i_j = c_j;
+    auto issue = [&](uint32_t st, uint32_t bar, bool box, bool recs, uint32_t (&sc)[C]) {
+        const TMItem& I = items[i_item];
+        const int geff = min(C, I.G - i_j * C);
+        if (lane == 0) {
+            if (box) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tm_expect(bar, (uint32_t)(32 * WB + geff * kRecBytes));
+                tm_load_box(st, &maps[i_item], i_j * WB, (int)(i_tile * kRows), bar);
+            }
+            if (recs) tm_load_bulk(st + kTMRec, I.rec + (int64_t)i_j * C * kRecBytes, (uint32_t)(geff * kRecBytes), bar);
+        }
+        if (box) {
+            const int64_t row = min((int64_t)i_tile * kRows + lane, I.N - 1);
+            const uint16_t* sp = I.scales + row * I.G + i_j * C;
+#pragma unroll
+            for (int k = 0; k < C; ++k) sc[k] = k < geff ? (uint32_t)__ldg(sp + k) : 0u;
+        }
+    };
+    auto advance = [&]() {
+        if (++i_j == items[i_item].cpt) {
+            i_j = 0;
+            if (++i_tile == (uint32_t)items[i_item].T) {
+                i_tile = 0;
+                ++i_item;
+            }
+        }
+    };
+
+    uint32_t sc[2][C];
+    // first chunk: weights and scales before the preparation kernel is waited for, records after
+    issue(base_s, bar0, true, false, sc[0]);
+    pdl_wait();  // prepared records and zeroed tile counters are ready past this point
+    issue(base_s, bar0, false, true, sc[0]);
+    advance();
+
+    int32_t seg_j = c_j;
+    bool first_seg = true;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int32_t k0 = 0; k0 < n; k0 += 2) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int32_t k = k0 + u;
+            if (k < n) {
+                // stage 1 - u held chunk k - 1, which every lane finished (syncwarp below)
+                if (k + 1 < n) {
+                    issue(base_s + (1 - u) * kTMStageB, u ? bar0 : bar1, true, true, sc[1 - u]);
+                    advance();
+                }
+                if (!__all_sync(0xffffffffu, tm_wait(u ? bar1 : bar0, (uint32_t)(k >> 1) & 1u))) {
+                    // give up: let the other stage's copy land (bounded) before leaving
+                    if (k + 1 < n) tm_wait(u ? bar0 : bar1, (uint32_t)((k + 1) >> 1) & 1u);
+                    return;
+                }
+                const uint8_t* stage = base + u * kTMStageB;
+                const TMItem& I = items[c_item];
+                const int geff = min(C, I.G - c_j * C);
+#pragma unroll
+                for (int gi = 0; gi < C; ++gi)
+                    if (gi < geff) tm_step<KIND>(stage, gi, sc[u][gi], g, t, acc);
+                ++c_j;
+                const bool more = k + 1 < n;
+                if (c_j == I.cpt || !more) {
+                    tm_flush(L, part, wg, P.first + c_item, c_tile, seg_j == 0 && c_j == I.cpt, first_seg, acc[0],
+                             acc[1], acc[2], acc[3]);
+                    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+                    first_seg = false;
+                    seg_j = c_j = 0;
+                    if (more && ++c_tile == (uint32_t)I.T) {
+                        c_tile = 0;
+                        ++c_item;
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 2) k_gemv_tma(const __grid_constant__ TMLaunch L) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[kWarps][2];
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5;
+    const int64_t wg = (int64_t)blockIdx.x * kWarps + warp;
+    if (wg >= L.W) return;  // whole warps; the kernel has no CTA-wide barrier
+    // stages start on 1 KB boundaries (the 128-byte swizzle pattern repeats every 1 KB)
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw) + warp * kTMWarpB;
+    if ((threadIdx.x & 31) == 0) {
+        tm_bar_init(smem_u32(&bars[warp][0]));
+        tm_bar_init(smem_u32(&bars[warp][1]));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    if (wg < L.part[0].W0 + L.part[0].W) tm_warp<1>(L, 0, (uint32_t)(wg - L.part[0].W0), wg, base, bars[warp]);
+    else tm_warp<0>(L, 1, (uint32_t)(wg - L.part[1].W0), wg, base, bars[warp]);
+}
+
 bool sk_prepare_device(int dev) {
     static bool ready[64] = {false};
     if (dev < 0 || dev >= 64) return false;
@@ -888,7 +1256,95 @@ cudaError_t launch_main(const Launch& L, int ctas, size_t smem, cudaStream_t st)
     return launch_pdl(fn, args, (unsigned)ctas, smem, st, true);
 }
 
+
+// ---- batch-1 TMA kernel: host side -------------------------------------------
+
+typedef CUresult (*TMEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// the driver's tensor-map encoder, looked up once through the runtime
+TMEncodeFn tm_encoder() {
+    static TMEncodeFn fn = []() -> TMEncodeFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<TMEncodeFn>(p);
+    }();
+    return fn;
+}
+
+bool tm_prepare_device(int dev) {
+    static bool ready[64] = {false};
+    if (dev < 0 || dev >= 64) return false;
+    if (!ready[dev]) {
+        if (cudaFuncSetAttribute((const void*)k_gemv_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, kTMSmem) !=
+            cudaSuccess)
+            return false;
+        ready[dev] = true;
+    }
+    return true;
+}
+
 }  // namespace
+
+// Tensor map of one packed matrix for k_gemv_tma: bytes x rows, box of one
+// chunk (128 bytes = four 2-bit groups, 128-byte swizzled; 96 bytes = two
+// 3-bit groups) x 32 rows; rows and bytes past the end read as zero.
+bool encode_gemv_tma_map(CUtensorMap* map, const void* packed, int grid, int64_t N, int64_t K) {
+    TMEncodeFn enc = tm_encoder();
+    if (!enc) return false;
+    const bool three = grid == kInt3;
+    const cuuint64_t dims[2] = {(cuuint64_t)row_bytes(grid, K), (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_bytes(grid, K)};
+    const cuuint32_t box[2] = {three ? 96u : 128u, (cuuint32_t)kRows};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(packed), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, three ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemv_tma(const Launch& P, int prep_warps, const TMLaunch& L, int ctas, bool overlap,
+                            cudaStream_t st) {
+    {
+        void* args[] = {const_cast<Launch*>(&P), &prep_warps};
+        cudaError_t e = launch_pdl((const void*)k_prep, args,
+                                   (unsigned)std::max((prep_warps + kWarps - 1) / kWarps, 1), 0, st, overlap);
+        if (e != cudaSuccess) return e;
+    }
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!tm_prepare_device(dev)) return cudaErrorInvalidDevice;
+    void* args[] = {const_cast<TMLaunch*>(&L)};
+    return launch_pdl((const void*)k_gemv_tma, args, (unsigned)ctas, kTMSmem, st, true);
+}
+
+// Warps of k_gemv_tma resident at once on the current device.
+int gemv_tma_resident_warps() {
+    static int warps[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (warps[dev] == 0) {
+        int sms = 0, per_sm = 0;
+        if (!tm_prepare_device(dev)) return 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv_tma, kThreads, kTMSmem) != cudaSuccess ||
+            per_sm < 1)
+            return 0;
+        warps[dev] = sms * per_sm * kWarps;
+    }
+    return warps[dev];
+}
+
+unsigned int take_gemv_timeouts() {
+    unsigned int v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tm_timeouts, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
+    if (cudaMemcpyToSymbol(g_tm_timeouts, &z, sizeof(z)) != cudaSuccess) return 0xFFFFFFFFu;
+    return v;
+}
 
 cudaError_t launch_gemv_sk(const Launch& P, int prep_warps, const SKLaunch& L, int ctas, bool overlap,
                            cudaStream_t st) {

@@ -58,4 +58,48 @@ TB_HD void part_range(const Item* it, int n, uint32_t w, uint32_t Q, uint32_t C,
     *end = part_first_tg(it, n, hi);
 }
 
+// Chunked variant.  The work of item i is T_i tiles x G_i groups, read in
+// chunks of C_i consecutive groups of one tile (a tile's last chunk may be
+// shorter; chunks per tile cpt_i = ceil(G_i / C_i)), numbered item by item,
+// tile by tile from chunk_base_i.  Chunk j of tile t starts at the cost
+// position
+//     pos = cost_base_i + (t G_i + j C_i) c_i,
+// and a warp owns the chunks whose start position lies in its quota range
+// [w Q, (w + 1) Q): whole chunks only, so no chunk is read by two warps.
+struct ChunkItem {
+    int64_t chunk_base, cost_base;
+    int32_t T, G, C, cpt, unit_cost;
+};
+
+// first chunk whose start position is >= L (Item: any type with the
+// ChunkItem fields)
+template <class Item>
+TB_HD uint32_t part_first_chunk(const Item* it, int n, uint32_t L) {
+    for (int i = 0; i < n; ++i) {
+        const uint32_t cb = (uint32_t)it[i].cost_base, uc = (uint32_t)it[i].unit_cost;
+        const uint32_t tcost = (uint32_t)it[i].G * uc, end = cb + (uint32_t)it[i].T * tcost;
+        if (L < end) {
+            const uint32_t d = L > cb ? L - cb : 0, ccost = (uint32_t)it[i].C * uc;
+            uint32_t t = d / tcost;
+            const uint32_t r = d - t * tcost;
+            uint32_t j = (r + ccost - 1) / ccost;
+            if (j >= (uint32_t)it[i].cpt) {
+                ++t;
+                j = 0;
+            }
+            return (uint32_t)it[i].chunk_base + t * (uint32_t)it[i].cpt + j;
+        }
+    }
+    return n ? (uint32_t)(it[n - 1].chunk_base + (int64_t)it[n - 1].T * it[n - 1].cpt) : 0;
+}
+
+// [begin, end) chunks of warp w (empty when w Q >= C)
+template <class Item>
+TB_HD void part_chunk_range(const Item* it, int n, uint32_t w, uint32_t Q, uint32_t C, uint32_t* begin,
+                            uint32_t* end) {
+    const uint32_t lo = w * Q < C ? w * Q : C, hi = (w + 1) * Q < C ? (w + 1) * Q : C;
+    *begin = part_first_chunk(it, n, lo);
+    *end = part_first_chunk(it, n, hi);
+}
+
 }  // namespace tb

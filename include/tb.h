@@ -149,7 +149,9 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
  * prepared copy of its activations (bf16, K per activation row, scaled by
  * powers of two) and per-128-group sums into the workspace, then reads them;
  * the calls also keep per-tile arrival counters and partial sums there
- * (tiles whose K range is split are combined in a fixed order).  For
+ * (tiles whose K range is split are combined in a fixed order).  For M = 1
+ * the size is ceil256(K/128 * 272) + ceil256(4 * ceil(N/32))
+ * + ceil256(256 * min(8192, ceil(N/32) * ceil(K/256))).  For
  * M >= 32 (the tensor-core path) the size is exact and device independent:
  *   ceil256(K/128 * NP * 264) + ceil256(T * K/128 * 256) + ceil256(4 * T)
  *     + [S > 1] ceil256(T * S * NP * 512)

@@ -79,20 +79,23 @@ def test_workspace_sizes(lib):
         want = (al(G * NP * 264) + al(tiles * G * 128 * 2) + al(4 * tiles) +
                 (al(tiles * splits * NP * 128 * 4) if splits > 1 else 0))
         assert tb.workspace_bytes(M, N, K) == want, (M, N, K)
-    for N, K in ((1, 128), (256, 1024), (17408, 5120)):
-        # batch 1 adds a counter per 32-row tile and two 32-float slots per warp
+    for N, K in ((1, 128), (256, 1024), (17408, 5120), (100, 1408)):
+        # batch 1: one 272-byte record per 128-group of x, a counter per 32-row tile and two 32-float
+        # slots per warp (at most one warp per chunk of two groups, the smaller chunk)
         tiles = (N + 31) // 32
-        warps = min(8192, tiles * (K // 128))
-        assert tb.workspace_bytes(1, N, K) == al(2 * K) + al(8 * (K // 128)) + al(4 * tiles) + al(256 * warps)
+        warps = min(8192, tiles * ((K // 128 + 1) // 2))
+        assert tb.workspace_bytes(1, N, K) == al(272 * (K // 128)) + al(4 * tiles) + al(256 * warps)
     assert tb.workspace_bytes(0, 8, 128) == 0 and tb.workspace_bytes(1, 8, 100) == 0
     assert tb.workspace_bytes(65, 8, 128) == 0 and tb.workspace_bytes(1, 0, 128) == 0
     items = (tb.Linear * 3)()
-    for i, (N, K) in enumerate(((4096, 4096), (1024, 4096), (4096, 12288))):
-        items[i] = tb.Linear(FAKE, FAKE, FAKE, FAKE, N, K, 1, 0)
-    tiles = sum((N + 31) // 32 for N in (4096, 1024, 4096))
-    tgs = sum((N + 31) // 32 * (K // 128) for N, K in ((4096, 4096), (1024, 4096), (4096, 12288)))
-    per = sum(al(2 * K) + al(8 * (K // 128)) for K in (4096, 4096, 12288))
-    assert tb.layer_workspace_bytes(items) == per + al(4 * tiles) + al(256 * min(8192, tgs))
+    shapes = ((4096, 4096, 2), (1024, 4096, 1), (4096, 12288, 0))  # (N, K, grid)
+    for i, (N, K, grid) in enumerate(shapes):
+        items[i] = tb.Linear(FAKE, FAKE, FAKE, FAKE, N, K, grid, 0)
+    tiles = sum((N + 31) // 32 for N, _, _ in shapes)
+    # chunks of two 3-bit groups or four 2-bit groups per 32-row tile
+    chunks = sum((N + 31) // 32 * -(-(K // 128) // (2 if grid == 2 else 4)) for N, K, grid in shapes)
+    per = sum(al(272 * (K // 128)) for _, K, _ in shapes)
+    assert tb.layer_workspace_bytes(items) == per + al(4 * tiles) + al(256 * min(8192, chunks))
 
 
 def test_argument_errors_before_launch(lib):
