@@ -46,11 +46,11 @@ def algo_bytes(N, K, grid, M=1, ybytes=4):
 
 
 def traffic_per_launch(algorithmic_bytes):
-    """DRAM bytes per k_gemv_sk launch from the committed ncu capture: its
+    """DRAM bytes per k_gemv_tma launch from the committed ncu capture: its
     measured traffic / algorithmic ratio times this launch's algorithmic
     bytes; None when the kernel's sources changed after the capture."""
     import hashlib
-    p = os.path.join(ROOT, "profiles", "k_gemv_sk_traffic.json")
+    p = os.path.join(ROOT, "profiles", "k_gemv_tma_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -504,7 +504,7 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": profile_traffic,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
-                         else "fallback 6.65 TB/s", "kernel": "k_gemv_sk (per tb_layer_gemv call; duration includes its k_prep)"},
+                         else "fallback 6.65 TB/s", "kernel": "k_gemv_tma (per tb_layer_gemv call; duration includes its k_prep)"},
             "e2e": {"value": e2e_value, "unit": "GB/s",
                     "h2d_bytes_per_step": S.x_all.numel() * 2, "d2h_bytes_per_step": S.y_all.numel() * 4},
             "gpu_launches": 2 * n_layers * args.steps,
