@@ -58,18 +58,6 @@ struct Launch {
 };
 
 // ---- stream-K batch-1 launch (see tb_linear.cu) ----------------------------
-struct SKItem {
-    const uint8_t* packed;
-    const uint16_t* scales;
-    const uint16_t* xs;  // prepared activations [K]
-    const float2* cf;    // [K/128] (offset * sum x, 2^S)
-    void* Y;
-    int64_t N, K, rbytes;
-    int64_t tg_base, tg_count, cost_base;  // partition (tb_partition.h)
-    int32_t unit_cost, G, T, grid, ydt;
-    int32_t tile_base;   // first tile counter of this item
-};
-
 // Two partitions side by side: the 3-bit items (it[0 .. n3)) on warps
 // [0, W3), the 2-bit items (it[n3 .. n_items)) on warps [W3, W); tile-group
 // and cost positions of the 2-bit items start again at 0.
@@ -77,15 +65,6 @@ struct SKPart {
     int32_t first, count;  // items
     int32_t W0, W;         // first warp, warps
     uint32_t C, Q;         // total cost, cost quota per warp (tb_partition.h)
-};
-
-struct SKLaunch {
-    SKItem it[kMaxItems];
-    int32_t n_items;
-    int32_t W;            // warps in the launch
-    SKPart part[2];       // [0]: 3-bit items, [1]: 2-bit items
-    int32_t* counters;    // one per 32-row tile, zeroed by the preparation kernel
-    float* partials;      // [W][2][32]
 };
 
 // Batch-1 TMA kernel (tb_linear.cu): items read in chunks of C groups x 32

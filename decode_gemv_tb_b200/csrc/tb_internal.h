@@ -24,13 +24,6 @@ cudaError_t launch_linear(const Launch& L, int nt, int ctas, int prep_warps, boo
 // dynamic shared memory of the main kernel
 size_t linear_smem_bytes(int nt, int scl_stride);
 
-struct SKLaunch;
-// Batch-1 path: preparation kernel (also clears P.zero) + stream-K kernel.
-cudaError_t launch_gemv_sk(const Launch& P, int prep_warps, const SKLaunch& L, int ctas, bool overlap,
-                           cudaStream_t st);
-// warps of the stream-K kernel resident at once on the current device (0 on error)
-int gemv_sk_resident_warps();
-
 struct TMLaunch;
 // Batch-1 path with TMA staging: preparation kernel (writes records, clears
 // P.zero) + k_gemv_tma.  The tensor map of each item comes from

@@ -485,371 +485,14 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 3 : 2) k_linear(const __gr
 }
 
 // ---------------------------------------------------------------------------
-// Stream-K batch-1 kernel.
+// Batch-1 kernel (k_gemv_tma): stream-K over TMA-staged chunks.
 //
-// Persistent warps, one contiguous equal-cost range of tile-groups each
-// (tb_partition.h), across tile and item boundaries: the cp.async ring never
+// Persistent warps, one contiguous equal-cost range of chunks each
+// (tb_partition.h), across tile and item boundaries, so the copy ring never
 // drains at a tile boundary.  A tile whose K the warp covers entirely is
 // written directly; a tile shared by several warps is combined by the last
 // of them to finish (per-tile arrival counter), which adds the partial sums
 // in warp order, so the result does not depend on timing.
-#ifndef TB_SK_STAGES
-#define TB_SK_STAGES 4
-#endif
-constexpr int kSKStages = TB_SK_STAGES;  // ring depth: kSKStages - 1 groups in flight per warp
-
-// Per-warp shared memory: kSKStages stages, each the weights of one
-// tile-group (32 rows x 32 or 48 bytes), its prepared activations (128 bf16,
-// stored as two 128-byte halves 16 bytes apart so the four t-lanes of an
-// LDS.128 hit distinct banks) and the 16-byte chunk holding its
-// (offset * sum x, 2^S) pair.
-constexpr int kSKW = 1536;               // weights
-constexpr int kSKX = kSKW;               // activations: 272 bytes
-constexpr int kSKC = kSKX + 272;         // (sum, 2^S) chunk: 16 bytes
-constexpr int kSKStageB = kSKC + 16;     // 1824
-constexpr int kSKWarpB = kSKStages * kSKStageB;
-
-// ---- per-step helpers -----------------------------------------------------------
-__device__ __forceinline__ uint32_t sk_xs_dst(int c) { return 16 * c + (c >= 8 ? 16 : 0); }
-
-// One 128-group of the 32-row tile from a stage: decode, MMAs, scale, accumulate
-// (batch 1: the prepared activations and the (sum, 2^S) pair come from the stage).
-// cofs: byte offset of this group's (sum, 2^S) pair inside the 16-byte chunk (8 for odd groups);
-// srow: bf16 scale of row `lane` (shuffled to rows g, g+8, g+16, g+24 only at the end, so the load
-// behind it has the whole step to land)
-template <int KIND>
-__device__ __forceinline__ void sk_step(const uint8_t* stage, uint32_t srow, int cofs, int g, int t,
-                                        float (&acc)[4]) {
-    float d[2][4];
-    bool first = true;  // the first MMA of each chain starts from zero
-    auto mma = [&](int rt, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
-        if (first) mma16816_z(d[rt], a0, a1, a2, a3, b0, b1);
-        else mma16816(d[rt], a0, a1, a2, a3, b0, b1);
-    };
-    // B fragment for codes 32 t + 8 q .. + 7 of the group
-    auto xfrag = [&](int q) {
-        const int c = 4 * t + q;  // 16-byte chunk of the 256-byte activation slice
-        return *reinterpret_cast<const uint4*>(stage + kSKX + sk_xs_dst(c));
-    };
-    if (KIND == 0) {
-        uint2 wv[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) wv[q] = *reinterpret_cast<const uint2*>(stage + (g + 8 * q) * 32 + 8 * t);
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            const uint4 xv0 = xfrag(2 * w), xv1 = xfrag(2 * w + 1);
-            uint32_t W[4], H[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                W[q] = w ? wv[q].y : wv[q].x;
-                H[q] = shr_fma(W[q], 8);
-            }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const uint32_t m0 = 0x00030003u << (4 * (r & 1)), m1 = 0x000C000Cu << (4 * (r & 1));
-                const uint4 v = (r >> 1) ? xv1 : xv0;
-#pragma unroll
-                for (int rt = 0; rt < 2; ++rt) {
-                    const uint32_t A = r < 2 ? W[2 * rt] : H[2 * rt], B = r < 2 ? W[2 * rt + 1] : H[2 * rt + 1];
-                    mma(rt, A & m0, B & m0, A & m1, B & m1, (r & 1) ? v.z : v.x, (r & 1) ? v.w : v.y);
-                }
-                first = false;
-            }
-        }
-    } else {
-        uint4 xv[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) xv[q] = xfrag(q);
-        // the two 16-row MMA tiles one after the other (keeps the live decode state small)
-#pragma unroll
-        for (int rt = 0; rt < 2; ++rt) {
-            uint32_t P[2][3];
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int p = 0; p < 3; ++p)
-                    P[h][p] = *reinterpret_cast<const uint32_t*>(stage + (g + 8 * (2 * rt + h)) * 48 + 12 * t + 4 * p);
-            uint32_t q1[2], q2[2], zA[2], zB[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                q1[h] = P[h][1] << 1;
-                q2[h] = P[h][2] << 2;
-                zA[h] = bit_mux(bit_mux(P[h][0], q1[h], bits_at(0, 5, 1)), q2[h], bits_at(0, 5, 2));
-                zB[h] = bit_mux(bit_mux(P[h][0], q1[h], bits_at(1, 5, 1)), q2[h], bits_at(1, 5, 2));
-            }
-            bool first3 = true;
-            auto emit = [&](int r, const uint32_t (&fa)[2], uint32_t ma, const uint32_t (&fb)[2], uint32_t mb) {
-                const uint4 v = xv[r >> 1];
-                if (first3) mma16816_z(d[rt], fa[0] & ma, fa[1] & ma, fb[0] & mb, fb[1] & mb, (r & 1) ? v.z : v.x,
-                                       (r & 1) ? v.w : v.y);
-                else mma16816(d[rt], fa[0] & ma, fa[1] & ma, fb[0] & mb, fb[1] & mb, (r & 1) ? v.z : v.x,
-                              (r & 1) ? v.w : v.y);
-                first3 = false;
-            };
-            emit(0, zA, 0x00070007u, zB, 0x000E000Eu);
-            emit(1, zA, 0x00380038u, zB, 0x00700070u);
-            uint32_t sA[2], sB[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                sA[h] = shr_fma(zA[h], 6);
-                sB[h] = shr_fma(zB[h], 6);
-            }
-            emit(2, sA, 0x00070007u, sB, 0x000E000Eu);
-            emit(3, sA, 0x00380038u, sB, 0x00700070u);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                sA[h] = shr_fma(zA[h], 12);
-                sB[h] = shr_fma(zB[h], 12);
-            }
-            emit(4, sA, 0x00070007u, sB, 0x000E000Eu);
-            uint32_t zC[2], zC6[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                zC[h] = bit_mux(bit_mux(P[h][0], q1[h], bits_at(2, 4, 1)), q2[h], bits_at(2, 4, 2));
-                zC6[h] = shr_fma(zC[h], 6);
-            }
-            emit(5, zC, 0x001C001Cu, zC, 0x00E000E0u);
-            emit(6, zC6, 0x001C001Cu, zC6, 0x00E000E0u);
-            // fields 14, 15 (plane bits 14/15, 30/31) from the raw planes, plane p realigned right
-            // by 14 - p: plane p of field 14 lands at bit p (16 + p), of field 15 at bit p + 1
-            uint32_t z14[2], z15[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t r0 = shr_fma(P[h][0], 14), r1 = shr_fma(P[h][1], 13), r2 = shr_fma(P[h][2], 12);
-                z14[h] = bit_mux(bit_mux(r0, r1, 0x00020002u), r2, 0x00040004u);
-                z15[h] = bit_mux(bit_mux(r0, r1, 0x00040004u), r2, 0x00080008u);
-            }
-            emit(7, z14, 0x00070007u, z15, 0x000E000Eu);
-        }
-    }
-    const float2 c = *reinterpret_cast<const float2*>(stage + kSKC + cofs);
-    float sc[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) sc[q] = bf16_bits_to_float(__shfl_sync(0xffffffffu, srow, g + 8 * q));
-#pragma unroll
-    for (int rt = 0; rt < 2; ++rt) {
-        acc[2 * rt] = fmaf(sc[2 * rt], fmaf(c.y, d[rt][0], -c.x), acc[2 * rt]);
-        acc[2 * rt + 1] = fmaf(sc[2 * rt + 1], fmaf(c.y, d[rt][2], -c.x), acc[2 * rt + 1]);
-    }
-}
-
-__device__ __forceinline__ void cp_async16_if(uint32_t dst, const void* src, bool p) {
-    asm volatile(
-        "{\n .reg .pred q;\n setp.ne.b32 q, %2, 0;\n @q cp.async.cg.shared.global [%0], [%1], 16;\n}" ::"r"(dst),
-        "l"(src), "r"((int)p)
-        : "memory");
-}
-
-// End of a segment [seg_grp, end_grp) of a tile: write y, or hand the
-// partial sums over and combine them if this warp arrives last.
-//   item: index into L.it; part: the partition the item belongs to;
-//   wg: this warp's index in the launch.
-__device__ __noinline__ void sk_flush(const SKLaunch& L, int part, int64_t wg, int item, uint32_t tile,
-                                      int32_t seg_grp, int32_t end_grp, bool first_seg, float v0, float v1, float v2,
-                                      float v3) {
-    const SKItem& I = L.it[item];
-    const SKPart& P = L.part[part];
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const int64_t row0 = (int64_t)tile * kRows;
-    const float v[4] = {v0, v1, v2, v3};
-    if (seg_grp == 0 && end_grp == I.G) {
-        if (t == 0) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int64_t row = row0 + g + 8 * q;
-                if (row < I.N) {
-                    if (I.ydt == kF32) static_cast<float*>(I.Y)[row] = v[q];
-                    else static_cast<__nv_bfloat16*>(I.Y)[row] = __float2bfloat16_rn(v[q]);
-                }
-            }
-        }
-        return;
-    }
-    float* mine = L.partials + (wg * 2 + (first_seg ? 0 : 1)) * kRows;
-    if (t == 0) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) __stcg(mine + g + 8 * q, v[q]);
-    }
-    __threadfence();
-    __syncwarp();
-    // contributors of this tile: the owners of its first and last tile-group (within the partition)
-    const uint32_t A = (uint32_t)I.tg_base + tile * (uint32_t)I.G;
-    const uint32_t pA = (uint32_t)I.cost_base + (A - (uint32_t)I.tg_base) * (uint32_t)I.unit_cost;
-    const uint32_t w0 = part_owner(pA, P.Q), w1 = part_owner(pA + (uint32_t)(I.G - 1) * I.unit_cost, P.Q);
-    int last = 0;
-    if (lane == 0) last = atomicAdd(L.counters + I.tile_base + tile, 1) == (int)(w1 - w0);
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (!last) return;
-    __threadfence();
-    float sum = 0.f;
-    for (uint32_t w = w0; w <= w1; ++w) {
-        // a warp that starts inside this tile has it as its first segment (slot 0), an earlier one
-        // as its last (slot 1)
-        const uint32_t wb = part_first_tg(L.it + P.first, P.count, w * P.Q);
-        sum += __ldcg(L.partials + ((int64_t)(P.W0 + w) * 2 + (wb >= A ? 0 : 1)) * kRows + lane);
-    }
-    const int64_t row = row0 + lane;
-    if (row < I.N) {
-        if (I.ydt == kF32) static_cast<float*>(I.Y)[row] = sum;
-        else static_cast<__nv_bfloat16*>(I.Y)[row] = __float2bfloat16_rn(sum);
-    }
-}
-
-// One warp of the stream-K kernel for code width KIND (0: 2-bit, 1: 3-bit).
-template <int KIND>
-__device__ __forceinline__ void sk_warp(const SKLaunch& L, int part, uint32_t w, int64_t wg, uint8_t* base) {
-    constexpr int RB = KIND ? 48 : 32;  // bytes of one row in one group
-    constexpr int NCH = KIND ? 3 : 2;   // 16-byte chunks per lane per stage
-    const SKPart& P = L.part[part];
-    const SKItem* items = L.it + P.first;
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    uint32_t tb, te;
-    part_range(items, P.count, w, P.Q, P.C, &tb, &te);
-    if (tb >= te) return;
-    const int32_t nsteps = (int32_t)(te - tb);
-
-    const uint32_t base_s = smem_u32(base);
-
-    // ---- locate the first tile-group
-    int c_item = 0;
-    for (int i = 1; i < P.count; ++i)
-        if (tb >= (uint32_t)items[i].tg_base) c_item = i;
-    uint32_t c_tile;
-    int32_t c_grp;
-    {
-        const uint32_t local = tb - (uint32_t)items[c_item].tg_base, G = (uint32_t)items[c_item].G;
-        c_tile = local / G;
-        c_grp = (int32_t)(local - c_tile * G);
-    }
-
-    // ---- issue cursor and this lane's copy sources
-    int i_item = c_item;
-    uint32_t i_tile = c_tile;
-    int32_t i_grp = c_grp, i_G = items[c_item].G;
-    const uint8_t* wsrc[NCH];
-    const uint16_t* i_sp;
-    const uint16_t* i_xs;
-    const float2* i_cf;
-    auto set_tile = [&](int item, uint32_t tile, int32_t grp) {
-        const SKItem& I = items[item];
-        const int64_t row0 = (int64_t)tile * kRows, nm1 = I.N - 1;
-#pragma unroll
-        for (int i = 0; i < NCH; ++i) {
-            const int c = lane + 32 * i, r = KIND ? c / 3 : c >> 1, pp = KIND ? c - 3 * r : c & 1;
-            wsrc[i] = I.packed + min(row0 + r, nm1) * I.rbytes + (int64_t)grp * RB + 16 * pp;
-        }
-        i_sp = I.scales + min(row0 + lane, nm1) * I.G + grp;
-        i_xs = I.xs + (int64_t)grp * kGroup + 8 * (lane & 15);
-        i_cf = I.cf + (grp & ~1);
-        i_G = I.G;
-    };
-    set_tile(i_item, i_tile, i_grp);
-    auto advance_issue = [&]() {
-#pragma unroll
-        for (int i = 0; i < NCH; ++i) wsrc[i] += RB;
-        ++i_sp;
-        i_xs += kGroup;
-        i_cf += (i_grp & 1) ? 2 : 0;
-        if (++i_grp == i_G) {
-            i_grp = 0;
-            if (++i_tile == (uint32_t)items[i_item].T) {
-                i_tile = 0;
-                ++i_item;
-            }
-            if (i_item < P.count) set_tile(i_item, i_tile, 0);
-        }
-    };
-    auto issue_weights = [&](uint32_t st) {
-#pragma unroll
-        for (int i = 0; i < NCH; ++i) cp_async16(st + 512 * i + 16 * lane, wsrc[i]);
-    };
-    auto issue_acts = [&](uint32_t st, const uint16_t* xs, const float2* cf) {
-        cp_async16_if(st + kSKX + sk_xs_dst(lane & 15), xs, lane < 16);
-        cp_async16_if(st + kSKC, cf, lane == 16);
-    };
-
-    // ---- prologue: weights and scales of the first steps before waiting for the preparation
-    //      kernel, their activation copies after it (one commit group per step).  Scales ride in
-    //      a register ring, one per stage: this lane's row, loaded kSKStages - 1 steps ahead.
-    uint32_t sring[kSKStages];
-    const uint16_t* pro_xs[kSKStages - 1];
-    const float2* pro_cf[kSKStages - 1];
-#pragma unroll
-    for (int k = 0; k < kSKStages - 1; ++k) {
-        if (k < nsteps) {
-            issue_weights(base_s + k * kSKStageB);
-            sring[k] = __ldg(i_sp);
-            pro_xs[k] = i_xs;
-            pro_cf[k] = i_cf;
-            advance_issue();
-        }
-    }
-    pdl_wait();  // prepared activations and zeroed tile counters are ready past this point
-#pragma unroll
-    for (int k = 0; k < kSKStages - 1; ++k) {
-        if (k < nsteps) issue_acts(base_s + k * kSKStageB, pro_xs[k], pro_cf[k]);
-        cp_commit();
-    }
-
-    // ---- main loop, unrolled by the ring size so every stage offset is a constant
-    int32_t c_G = items[c_item].G, seg_grp = c_grp;
-    bool first_seg = true;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-    for (int32_t j0 = 0; j0 < nsteps; j0 += kSKStages) {
-#pragma unroll
-        for (int u = 0; u < kSKStages; ++u) {
-            const int32_t j = j0 + u;
-            if (j < nsteps) {
-                cp_wait<kSKStages - 2>();
-                __syncwarp();  // stage u (every lane's copies) is visible
-                const uint32_t srow = sring[u];
-                if (j + kSKStages - 1 < nsteps) {
-                    const uint32_t st = base_s + ((u + kSKStages - 1) % kSKStages) * kSKStageB;
-                    issue_weights(st);
-                    issue_acts(st, i_xs, i_cf);
-                    sring[(u + kSKStages - 1) % kSKStages] = __ldg(i_sp);
-                    advance_issue();
-                }
-                cp_commit();
-                sk_step<KIND>(base + u * kSKStageB, srow, (c_grp & 1) * 8, g, t, acc);
-                ++c_grp;
-                const bool more = j + 1 < nsteps;
-                if (c_grp == c_G || !more) {
-                    sk_flush(L, part, wg, P.first + c_item, c_tile, seg_grp, c_grp, first_seg, acc[0], acc[1], acc[2],
-                             acc[3]);
-                    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-                    first_seg = false;
-                    seg_grp = c_grp = 0;
-                    if (more) {
-                        if (++c_tile == (uint32_t)items[c_item].T) {
-                            c_tile = 0;
-                            ++c_item;
-                        }
-                        c_G = items[c_item].G;
-                    }
-                }
-            }
-        }
-    }
-    cp_wait<0>();
-}
-
-__global__ void __launch_bounds__(kThreads, 2) k_gemv_sk(const __grid_constant__ SKLaunch L) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    pdl_trigger();
-    const int warp = threadIdx.x >> 5;
-    const int64_t wg = (int64_t)blockIdx.x * kWarps + warp;
-    if (wg >= L.W) return;  // whole warps; the kernel has no CTA-wide barrier
-    uint8_t* base = smem + warp * kSKWarpB;
-    if (wg < L.part[0].W0 + L.part[0].W) sk_warp<1>(L, 0, (uint32_t)(wg - L.part[0].W0), wg, base);
-    else sk_warp<0>(L, 1, (uint32_t)(wg - L.part[1].W0), wg, base);
-}
-
-size_t gemv_sk_smem_bytes() { return (size_t)kWarps * kSKWarpB; }
-
-// ---------------------------------------------------------------------------
-// Batch-1 kernel with TMA staging (k_gemv_tma).
 //
 // Reading 32 rows x 32 bytes per warp with per-lane 16-byte copies leaves
 // each load instruction touching 32 cache lines for 16 to 32 bytes apiece:
@@ -858,7 +501,8 @@ size_t gemv_sk_smem_bytes() { return (size_t)kWarps * kSKWarpB; }
 // per chunk -- 32 rows x 128 bytes (four 2-bit groups, 128-byte swizzled) or
 // 32 rows x 96 bytes (two 3-bit groups) -- plus one bulk copy of the chunk's
 // prepared activation records, into a two-stage ring; both complete on the
-// stage's mbarrier.  The per-group arithmetic is that of k_gemv_sk.
+// stage's mbarrier.  Per group, the warp decodes its two 16-row MMA tiles
+// with LOP3 masks and runs sixteen mma.sync m16n8k16 (bf16, fp32 accumulate).
 constexpr int kTMStageB = 6144;                // weights box (<= 4 KB) + records (<= 4 x 272 B)
 constexpr int kTMRec = 4096;                   // offset of the records in a stage
 constexpr int kTMWarpB = 2 * kTMStageB;        // two stages per warp
@@ -906,7 +550,7 @@ __device__ __forceinline__ void tm_load_bulk(uint32_t dst, const void* src, uint
 }
 
 // One group gi of a chunk held in stage: 32 rows x 128 codes, two 16-row MMA
-// tiles, as sk_step.  Weights: 2-bit rows are 128 bytes, 128-byte swizzled
+// tiles.  Weights: 2-bit rows are 128 bytes, 128-byte swizzled
 // (16-byte unit u of row r at unit u ^ (r & 7)); 3-bit rows are 96 bytes.
 template <int KIND>
 __device__ __forceinline__ void tm_step(const uint8_t* stage, int gi, uint32_t srow, int g, int t, float (&acc)[4]) {
@@ -1024,7 +668,7 @@ __device__ __forceinline__ void tm_step(const uint8_t* stage, int gi, uint32_t s
 }
 
 // End of a warp's segment of a tile: write y, or hand the partial sums over
-// and combine them if this warp arrives last (as sk_flush; the contributors
+// and combine them if this warp arrives last (the contributors
 // are the owners of the tile's first and last chunk start -- every warp in
 // between owns at least one chunk start because the launcher keeps the
 // quota at least one chunk's cost).
@@ -1211,18 +855,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_gemv_tma(const __grid_constant_
     else tm_warp<0>(L, 1, (uint32_t)(wg - L.part[1].W0), wg, base, bars[warp]);
 }
 
-bool sk_prepare_device(int dev) {
-    static bool ready[64] = {false};
-    if (dev < 0 || dev >= 64) return false;
-    if (!ready[dev]) {
-        if (cudaFuncSetAttribute((const void*)k_gemv_sk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gemv_sk_smem_bytes()) != cudaSuccess)
-            return false;
-        ready[dev] = true;
-    }
-    return true;
-}
-
 cudaError_t launch_pdl(const void* fn, void** args, unsigned grid, size_t smem, cudaStream_t st, bool pdl) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
@@ -1344,42 +976,6 @@ unsigned int take_gemv_timeouts() {
     if (cudaMemcpyFromSymbol(&v, g_tm_timeouts, sizeof(v)) != cudaSuccess) return 0xFFFFFFFFu;
     if (cudaMemcpyToSymbol(g_tm_timeouts, &z, sizeof(z)) != cudaSuccess) return 0xFFFFFFFFu;
     return v;
-}
-
-cudaError_t launch_gemv_sk(const Launch& P, int prep_warps, const SKLaunch& L, int ctas, bool overlap,
-                           cudaStream_t st) {
-    {
-        void* args[] = {const_cast<Launch*>(&P), &prep_warps};
-        cudaError_t e = launch_pdl((const void*)k_prep, args,
-                                   (unsigned)std::max((prep_warps + kWarps - 1) / kWarps, 1), 0, st, overlap);
-        if (e != cudaSuccess) return e;
-    }
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (!sk_prepare_device(dev)) return cudaErrorInvalidDevice;
-    void* args[] = {const_cast<SKLaunch*>(&L)};
-    return launch_pdl((const void*)k_gemv_sk, args, (unsigned)ctas, gemv_sk_smem_bytes(), st, true);
-}
-
-// Warps of the stream-K kernel that are resident at once on the current
-// device (its grid is sized to exactly this, so every warp runs from the
-// start: the partition is only balanced if no warp waits for a slot).
-int gemv_sk_resident_warps() {
-    static int warps[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (warps[dev] == 0) {
-        int sms = 0, per_sm = 0;
-        if (!sk_prepare_device(dev)) return 0;
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv_sk, kThreads, gemv_sk_smem_bytes()) !=
-                cudaSuccess ||
-            per_sm < 1)
-            return 0;
-        warps[dev] = sms * per_sm * kWarps;
-    }
-    return warps[dev];
 }
 
 size_t linear_smem_bytes(int nt, int scl_stride) {
