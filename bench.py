@@ -64,6 +64,18 @@ def traffic_per_launch(algorithmic_bytes):
     return algorithmic_bytes * d["traffic_over_algorithmic"]
 
 
+def workload_config(stack, world):
+    """The `config` object of the JSON line (both arms): the decode stack's
+    shape, grid mix and bytes."""
+    packed = sum(m.N * m.K * (3 if m.grid == synth.INT3 else 2) // 8 for mats in stack for m in mats)
+    step_bytes = sum(algo_bytes(m.N, m.K, m.grid) for mats in stack for m in mats)
+    return {"workload": f"qwen3_8b_like_decode_stack_{len(stack)}L_mixed_grids", "batch": 1, "layers": len(stack),
+            "hidden": 4096, "mlp": 12288, "kv_dim": 1024,
+            "grid_mix": {synth.GRID_NAMES[g]: round(v, 4) for g, v in synth.grid_fractions(stack).items()},
+            "packed_GB": packed / 1e9, "step_algorithmic_bytes": step_bytes,
+            "l2": "working set larger than L2 (no flush)", "parallelism": f"replicas{world}", "prewarm_s": PREWARM_S}
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -400,11 +412,10 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "qwen3_8b_like_decode_stack_36L_mixed_grids (sample: layer-0 k+v GEMV)",
-                       "batch": 1},
+            "config": workload_config(synth.config3_stack(), 1),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": "fp64 single-threaded oracle GEMV of layer-0 k and v (1024x4096, 2-bit) "
-                                       "per step"},
+                             "sample": "each step: fp64 single-threaded oracle GEMV of layer-0 k and v (1024x4096, "
+                                       "2-bit) of this workload; value = their algorithmic bytes / time"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -491,12 +502,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"qwen3_8b_like_decode_stack_{n_layers}L_mixed_grids", "batch": 1,
-                       "layers": n_layers, "hidden": 4096, "mlp": 12288, "kv_dim": 1024,
-                       "grid_mix": {synth.GRID_NAMES[g]: round(v, 4) for g, v in synth.grid_fractions(S.stack).items()},
-                       "packed_GB": S.packed_bytes / 1e9, "step_algorithmic_bytes": S.step_bytes,
-                       "l2": "working set larger than L2 (no flush)", "parallelism": f"replicas{world}",
-                       "prewarm_s": PREWARM_S},
+            "config": workload_config(S.stack, world),
             "decoder_layer_us_per_token": us_layer,
             "decoder_layer_us_per_token_overlap_flag": ms_ovl * 1e3 / n_layers,
             "tokens_per_s_equivalent": 1e6 / (us_layer * n_layers),
