@@ -347,6 +347,81 @@ def rows_section(dev, stream):
     out["gemm_gate_17408x5120"] = g
     del bufs, Ws
     torch.cuda.empty_cache()
+
+    # hot L2 (repeated calls on the same buffers) and cold L2 (a 256 MB write
+    # before every call, its own time subtracted)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    t_flush = med(lambda: flush.fill_(1))
+
+    def hot_cold(fn):
+        hot = med(fn)
+        cold = med(lambda: (flush.fill_(1), fn())) - t_flush
+        return hot, max(cold, 1e-6)
+
+    def gemv_row(N, K, grid, p, s, x):
+        y = torch.empty(N, dtype=torch.float32, device=dev)
+        ws = tb.workspace(tb.workspace_bytes(1, N, K), dev)
+        hot, cold = hot_cold(lambda: tb.tb_gemv(p, grid, s, x, N, K, y=y, ws=ws))
+        by = algo_bytes(N, K, grid)
+        return {"hot_us": hot * 1e3, "hot_GB_s": by / hot / 1e6, "cold_us": cold * 1e3, "cold_GB_s": by / cold / 1e6}
+
+    # config 1: 256 x 1024 2-bit, W = c s exactly
+    c1 = synth.CONFIG1
+    codes = synth.uniform_codes(c1["N"], c1["K"], -2, 1, seed=c1["seed"])
+    s1 = synth.config1_scales(c1["N"], c1["K"], seed=c1["seed"])
+    W1 = (codes.float() * s1.float().repeat_interleave(128, dim=1)).to(dev)
+    s1 = s1.to(dev)
+    p1 = tb.tb_pack(W1, synth.INT2, s1)
+    out["gemv_config1_256x1024_int2"] = gemv_row(c1["N"], c1["K"], synth.INT2, p1, s1,
+                                                 synth.activations(c1["K"], seed=c1["seed"], device=dev))
+    # config 2: Qwen3-1.7B-like shapes over the three grids
+    c2 = {}
+    for m in synth.config2_cases():
+        W = synth.gaussian_weights(m.N, m.K, seed=m.seed, device=dev)
+        s2 = tb.tb_scales_absmax(W, m.grid)
+        p2 = tb.tb_pack(W, m.grid, s2)
+        c2[m.name] = gemv_row(m.N, m.K, m.grid, p2, s2, synth.activations(m.K, seed=m.seed, device=dev))
+        del W
+    out["gemv_config2"] = c2
+
+    # one isolated 8B-like layer (q, o 3-bit; k, v 2-bit; MLP ternary), one tb_layer_gemv per launch
+    items = []
+    for m in synth.isolated_layer():
+        W = synth.gaussian_weights(m.N, m.K, seed=m.seed, device=dev, dtype=torch.bfloat16)
+        si = tb.tb_scales_absmax(W, m.grid)
+        items.append((tb.tb_pack(W, m.grid, si), m.grid, si, synth.activations(m.K, seed=m.seed, device=dev),
+                      torch.empty(m.N, dtype=torch.float32, device=dev), m.N, m.K))
+        del W
+    arr = tb.linear_items(items)
+    wsl = tb.workspace(tb.layer_workspace_bytes(arr), dev)
+    hot, cold = hot_cold(lambda: tb.tb_layer_gemv(arr, wsl, 0))
+    by = sum(algo_bytes(n, k, gr) for _, gr, _, _, _, n, k in items)
+    out["isolated_layer_8b_q3_k2_v2_o3_mlp_ternary"] = {"hot_us_per_launch": hot * 1e3, "cold_us_per_launch": cold * 1e3,
+                                                        "cold_GB_s": by / cold / 1e6, "algorithmic_bytes": by}
+    del items, arr, wsl, flush
+    torch.cuda.empty_cache()
+
+    # config 5: batch-1 GEMV over all 280 matrices of a 40-layer 14B-like stack
+    # (outlier weights, mixed grids), packed by the library; one pass = 40 layer calls
+    layers, packed5, by5 = [], 0, 0
+    for mats in synth.config5_stack():
+        its = []
+        for m in mats:
+            W = synth.outlier_weights(m.N, m.K, seed=m.seed, device=dev)
+            s5 = tb.tb_scales_absmax(W, m.grid)
+            p5 = tb.tb_pack(W, m.grid, s5)
+            del W
+            its.append((p5, m.grid, s5, synth.activations(m.K, seed=m.seed, device=dev),
+                        torch.empty(m.N, dtype=torch.float32, device=dev), m.N, m.K))
+            packed5 += p5.numel()
+            by5 += algo_bytes(m.N, m.K, m.grid)
+        layers.append((its, tb.linear_items(its)))
+    ws5 = tb.workspace(max(tb.layer_workspace_bytes(a) for _, a in layers), dev)
+    ms5 = med(lambda: [tb.tb_layer_gemv(a, ws5, 0) for _, a in layers], reps=5, inner=1)
+    out["config5_stack_14b_40L_gemv"] = {"ms_per_pass": ms5, "GB_s": by5 / ms5 / 1e6, "packed_GB": packed5 / 1e9,
+                                         "algorithmic_GB": by5 / 1e9, "matrices": 280}
+    del layers, ws5
+    torch.cuda.empty_cache()
     return out
 
 

@@ -104,6 +104,14 @@ def config3_stack():
     return mixed_grid_stack(CONFIG3_LAYERS, 7, 14, CONFIG3_HIDDEN, CONFIG3_MLP, 3000)
 
 
+def isolated_layer():
+    """One Qwen3-8B-like layer timed on its own: q and o at 3 bits, k and v
+    at 2 bits, the MLP ternary."""
+    grids = {"q": INT3, "k": INT2, "v": INT2, "o": INT3, "gate": TERNARY, "up": TERNARY, "down": TERNARY}
+    return [Matrix(f"iso.{name}", N, K, grids[name], 3900 * 16 + pi)
+            for pi, (name, N, K) in enumerate(qwen3_layer_shapes(CONFIG3_HIDDEN, CONFIG3_MLP))]
+
+
 def config5_stack():
     """40 Qwen3-14B-like layers: 18.73% 3-bit, 5.95% 2-bit, 75.32% ternary."""
     return mixed_grid_stack(CONFIG5_LAYERS, 14, 16, CONFIG4_HIDDEN, CONFIG4_MLP, 5000)
