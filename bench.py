@@ -274,13 +274,25 @@ def time_region(fn, steps, warmup, stream, dist=None, clocks=None):
     torch.cuda.synchronize()
     if clocks:
         clocks.end()
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(e0.elapsed_time(e1), dist)
     if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     return ms
+
+
+def max_over_ranks(ms, dist=None):
+    """The slowest rank's time (every rank calls this at the same step)."""
+    if not dist:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, step_bytes, ms_per_step):
+    """Whole-job GB/s: each of the `world` replicas processes one step's
+    bytes in the slowest rank's step time."""
+    return world * step_bytes / (ms_per_step * 1e-3) / 1e9
 
 
 def rows_section(dev, stream):
@@ -538,7 +550,7 @@ def main():
         ms = time_region(g_step.replay, args.steps, args.warmup, cur, dist, clk)
     clocks = clk.summary()
     ms_step = ms / args.steps
-    value = world * S.step_bytes / (ms_step * 1e-3) / 1e9
+    value = job_throughput(world, S.step_bytes, ms_step)
     us_layer = ms_step * 1e3 / n_layers
     # dominant kernel: the stream-K GEMV of each tb_layer_gemv call; its
     # duration is taken as the whole call's (preparation kernel included),
@@ -563,7 +575,7 @@ def main():
 
     g_e2e = capture(e2e_step)
     ms_e2e = time_region(g_e2e.replay, args.steps, args.warmup, cur, dist)
-    e2e_value = world * S.step_bytes / (ms_e2e / args.steps * 1e-3) / 1e9
+    e2e_value = job_throughput(world, S.step_bytes, ms_e2e / args.steps)
     del g_e2e, g_step
 
     rows = None if args.no_rows else rows_section(dev, torch.cuda.current_stream(dev))

@@ -370,3 +370,10 @@ def test_layer_overlap_flag_and_shared_workspace(oracle):
         for L, it in enumerate(layers):
             for i, (p, grid, s, x, y, N, K) in enumerate(it):
                 assert torch.equal(y, alone[L][i]), (flags, L, i)
+
+
+def test_zz_no_bounded_wait_gave_up():
+    """After every test above: no device-side bounded wait (TMA copies,
+    tensor-core hand-offs) timed out, so every result above is a real one."""
+    torch.cuda.synchronize()
+    assert tb.wait_timeouts() == 0
