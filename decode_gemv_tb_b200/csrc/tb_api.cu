@@ -349,7 +349,9 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     }
     if (M >= kTCMinM) {
         if (workspace_bytes < gemm_tc_workspace_bytes(M, N, K)) return TB_ERR_ARG;
-        if (K / kGroup * 64 > INT_MAX || (N + 127) / 128 > INT_MAX / 16) return TB_ERR_SHAPE;
+        if (K / kGroup * 64 > INT_MAX || (N + 127) / 128 > INT_MAX / 16 ||
+            (N + 127) / 128 * (K / kGroup) >= ((int64_t)1 << 32))
+            return TB_ERR_SHAPE;
         return cuda_status(launch_gemm_tc(packed, grid, scales, X, ldx, Y, y_dtype, ldy, (int)M, N, K, workspace, st));
     }
     // column blocks of up to 16 batch rows per launch

@@ -18,19 +18,23 @@
 //     that multiple of 2^-133); the pairs go to tensor memory (tcgen05.st),
 //     one TMEM lane per row, k in natural order along the columns -- the A
 //     operand;
-//   * the preparation kernel has stored X per group as
-//         X[m][k] * 2^(133 - S_mg - p(k))       (exact: powers of two)
+//   * the preparation kernel has stored X per group, with one exponent S_g
+//     for all batch rows, as
+//         X[m][k] * 2^(133 - S_g - p(k))       (exact: powers of two)
 //     in the K-major core-matrix layout the MMA reads from shared memory,
-//     followed by (offset * sum_k X[m][k], 2^S_mg), and the group scales
+//     each row followed by a 16-wide correction slice (sum_k X[m][k] *
+//     2^(120 - S_g) as three bf16 terms), then 2^S_g; and the group scales
 //     transposed per tile; the producer brings a group's X and the tile's
 //     128 scales in with two bulk copies, two groups ahead -- the B operand;
 //   * the producer warp issues the group's eight 128 x NP x 16 MMAs (bf16
 //     in, fp32 accumulate in tensor memory; one elected lane of the
-//     converged warp, so the operands stay warp-uniform) and commits them
-//     to an mbarrier;
+//     converged warp, so the operands stay warp-uniform), a ninth with A a
+//     constant shared-memory tile (-offset * 2^-120 in three k slots) and B
+//     the correction slices, which subtracts offset * sum X, and commits
+//     them to an mbarrier;
 //   * while they run, each decoder reads its half of the previous group's
 //     accumulator row back (tcgen05.ld) and applies the group scale:
-//         acc[m] += s * (2^S * D[m] - offset * sum X)
+//         acc[m] += (s * 2^S_g) * D[m]
 //     A and D are double-buffered in tensor memory (2 x 64 + 2 x NP
 //     columns of the 256 a CTA allocates; two CTAs per SM).
 // K-splits of one tile are combined by the last CTA to finish, in split
@@ -58,7 +62,11 @@ constexpr int kTCTargetCtas = 296;               // 2 CTAs on each of 148 SMs
 constexpr int kTCMaxSplits = 16;
 constexpr size_t kTCMinSmem = 80 * 1024;         // at most two CTAs (2 x 256 TMEM columns) per SM
 
-__host__ __device__ constexpr int tc_group_bytes(int np) { return np * 264; }  // NP x 128 bf16 + NP float2
+// one prepared group: NP rows x 144 bf16 (128 activations + a 16-wide
+// correction slice) in the K-major core-matrix layout (18 chunks of 8 k per
+// 8 rows: 2304 bytes per 8 rows), then 2^S_g as a float and 12 zero bytes
+__host__ __device__ constexpr int tc_group_bytes(int np) { return np * 288 + 16; }
+constexpr int kTCBRowGroupB = 18 * 128;  // stride between 8-row core-matrix groups of B
 
 // field position (bit of its 16-bit half) of 3-bit field f after the decode below
 __host__ __device__ constexpr int pos3(int f) { return f < 12 ? f % 6 : (f & 1); }
@@ -153,6 +161,14 @@ __device__ __forceinline__ void mma_ts_warp(uint32_t d, uint32_t a, uint64_t bde
         "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u)
         : "memory");
 }
+// D[tmem d] += A[smem desc a] x B[smem desc b], same warp-level issue
+__device__ __forceinline__ void mma_ss_warp(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
+    asm volatile(
+        "{\n .reg .pred e, p;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}" ::"r"(d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(1u), "r"(0u)
+        : "memory");
+}
 // commit by the same elected lane (the lowest active one) that issued the MMAs
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
     asm volatile(
@@ -163,9 +179,9 @@ __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
 
 // Shared-memory descriptor of a K-major operand without swizzle: core
 // matrices of 8 rows x 16 bytes, the next 8 k (16 bytes) 128 bytes on
-// (leading byte offset), the next 8 rows 2048 bytes on (stride byte offset).
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) {
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(2048 >> 4) << 32) |
+// (leading byte offset), the next 8 rows sbo bytes on (stride byte offset).
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr, uint32_t sbo) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(sbo >> 4) << 32) |
            (1ull << 46);
 }
 
@@ -237,59 +253,97 @@ struct TCArgs {
 
 namespace {
 
-// ---- preparation: one warp per (group g, batch row m < NP) -------------------
+// ---- preparation: one CTA per group g -----------------------------------------
+// Rows m < M of X for group g become X[m][k] * 2^(133 - S_g - p(k)), with one
+// exponent S_g = (largest exponent of the group over all batch rows) + 7, in
+// the K-major core-matrix layout; rows M .. NP - 1 are zero.  The 16-wide
+// correction slice of row m holds Sum_k X[m][k] * 2^(120 - S_g) split exactly
+// into three bf16 terms: against the constant A slice (-offset * 2^-120 in
+// three k slots) the MMA then adds -offset * Sum_k X[m][k] * 2^-S_g to
+// D[.][m], so that D = 2^-S_g * (Sum_k u X - offset Sum_k X) and the epilogue
+// is acc += (s * 2^S_g) * D.  The CTAs also clear the tile counters and
+// transpose the group scales per 128-row tile.
+__device__ __forceinline__ float pow2_scale(float v, int sh) {  // v * 2^sh, sh within +-252, exact
+    const int s1 = sh >> 1, s2 = sh - s1;
+    return v * __int_as_float((s1 + 127) << 23) * __int_as_float((s2 + 127) << 23);
+}
+
 __global__ void __launch_bounds__(256) k_prep_tc(const __grid_constant__ TCArgs A) {
+    __shared__ int wmax[8];
+    __shared__ float sums[64];
     for (int i = blockIdx.x * 256 + threadIdx.x; i < A.tiles; i += gridDim.x * 256) A.counters[i] = 0;
     // scales transposed per 128-row tile, so that one bulk copy brings a tile's 128 scales of a group
+    // (element i: tile-group pair i / 128 = t * G + g, row t * 128 + i % 128)
     const int64_t n_sprep = (int64_t)A.tiles * A.G * kTCRows;
     for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n_sprep; i += (int64_t)gridDim.x * 256) {
-        const int64_t t = i / ((int64_t)A.G * kTCRows), rem = i - t * A.G * kTCRows;
-        const int64_t g = rem / kTCRows, row = t * kTCRows + (rem - g * kTCRows);
+        const uint32_t tg = (uint32_t)(i >> 7), t = tg / (uint32_t)A.G, g = tg - t * (uint32_t)A.G;
+        const int64_t row = (int64_t)t * kTCRows + (i & (kTCRows - 1));
         A.sprep[i] = row < A.N ? A.scales[row * A.G + g] : (uint16_t)0;
     }
-    const int wi = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (wi >= A.G * A.NP) return;
-    const int g = wi / A.NP, m = wi - g * A.NP;
+    const int g = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (g >= A.G) return;  // uniform over the CTA
     uint8_t* gb = A.bprep + (int64_t)g * tc_group_bytes(A.NP);
-    // elements k = 4 lane .. 4 lane + 3 of row m: core matrix (m / 8, k / 8), row m % 8, bytes 2 (k % 8)
-    uint8_t* dst = gb + ((m >> 3) * 16 + (lane >> 1)) * 128 + (m & 7) * 16 + 8 * (lane & 1);
-    if (m >= A.M) {  // padding rows of B: zero, and zero correction terms
-        *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
-        if (lane == 0) *reinterpret_cast<float2*>(gb + A.NP * 256 + 8 * m) = make_float2(0.f, 0.f);
-        return;
-    }
-    const uint16_t* xg = A.X + (int64_t)m * A.ldx + (int64_t)g * kGroup;
-    const uint2 raw = *reinterpret_cast<const uint2*>(xg + 4 * lane);
-    const uint32_t hv[4] = {raw.x & 0xFFFFu, raw.x >> 16, raw.y & 0xFFFFu, raw.y >> 16};
+    // pass 1: largest exponent over every row, and each row's sum
     int e = 0;
-    float sum = 0.f;
+    for (int m = warp; m < A.M; m += 8) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(A.X + (int64_t)m * A.ldx + (int64_t)g * kGroup + 4 * lane);
+        const uint32_t hv[4] = {raw.x & 0xFFFFu, raw.x >> 16, raw.y & 0xFFFFu, raw.y >> 16};
+        float sum = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        e = max(e, (int)((hv[j] >> 7) & 0xFFu));
-        sum += bf16_bits_to_float(hv[j]);
+        for (int j = 0; j < 4; ++j) {
+            e = max(e, (int)((hv[j] >> 7) & 0xFFu));
+            sum += bf16_bits_to_float(hv[j]);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) sums[m] = sum;
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
-        sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    }
+    for (int o = 16; o; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
+    if (lane == 0) wmax[warp] = e;
+    __syncthreads();
+    e = wmax[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) e = max(e, wmax[w]);
     // S = exponent of max |x| + 7 (a zero or subnormal group counts as 2^-126)
     const int S = min(max(e, 1) - 127 + 7, 127);
-    uint32_t out[2] = {0u, 0u};
+    // pass 2: the scaled rows and their correction slices
+    for (int m = warp; m < A.NP; m += 8) {
+        uint8_t* rowb = gb + (m >> 3) * kTCBRowGroupB + (m & 7) * 16;  // chunk c of row m at rowb + 128 c
+        uint2 outv = make_uint2(0u, 0u);
+        uint4 corr = make_uint4(0u, 0u, 0u, 0u);
+        if (m < A.M) {
+            const uint2 raw =
+                *reinterpret_cast<const uint2*>(A.X + (int64_t)m * A.ldx + (int64_t)g * kGroup + 4 * lane);
+            const uint32_t hv[4] = {raw.x & 0xFFFFu, raw.x >> 16, raw.y & 0xFFFFu, raw.y >> 16};
+            uint32_t out[2] = {0u, 0u};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int k = 4 * lane + j;
-        const int p = A.grid == kInt3 ? pos3((k & 31) >> 1) : 2 * ((k >> 1) & 3);
-        const int sh = 133 - S - p;  // 1 .. 252: two exact power-of-two factors
-        const int s1 = sh >> 1, s2 = sh - s1;
-        const float v = bf16_bits_to_float(hv[j]) * __int_as_float((s1 + 127) << 23) * __int_as_float((s2 + 127) << 23);
-        out[j >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v)) << (16 * (j & 1));
+            for (int j = 0; j < 4; ++j) {
+                const int k = 4 * lane + j;
+                const int p = A.grid == kInt3 ? pos3((k & 31) >> 1) : 2 * ((k >> 1) & 3);
+                const float v = pow2_scale(bf16_bits_to_float(hv[j]), 133 - S - p);  // exact: 8 significant bits
+                out[j >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v)) << (16 * (j & 1));
+            }
+            outv = make_uint2(out[0], out[1]);
+            if (lane == 0) {
+                const float v = pow2_scale(sums[m], 120 - S);
+                const __nv_bfloat16 h1 = __float2bfloat16_rn(v);
+                const float r1 = v - __bfloat162float(h1);
+                const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
+                const __nv_bfloat16 h3 = __float2bfloat16_rn(r1 - __bfloat162float(h2));
+                corr.x = (uint32_t)__bfloat16_as_ushort(h1) | ((uint32_t)__bfloat16_as_ushort(h2) << 16);
+                corr.y = (uint32_t)__bfloat16_as_ushort(h3);
+            }
+        }
+        // elements k = 4 lane .. 4 lane + 3: chunk lane / 2, bytes 8 (lane % 2)
+        *reinterpret_cast<uint2*>(rowb + (lane >> 1) * 128 + 8 * (lane & 1)) = outv;
+        if (lane == 0) {
+            *reinterpret_cast<uint4*>(rowb + 16 * 128) = corr;                       // k 128 .. 135
+            *reinterpret_cast<uint4*>(rowb + 17 * 128) = make_uint4(0u, 0u, 0u, 0u);  // k 136 .. 143
+        }
     }
-    *reinterpret_cast<uint2*>(dst) = make_uint2(out[0], out[1]);
-    if (lane == 0) {
-        const float off = A.grid == kInt3 ? 4.f : 2.f;
-        *reinterpret_cast<float2*>(gb + A.NP * 256 + 8 * m) = make_float2(off * sum, __int_as_float((S + 127) << 23));
-    }
+    if (threadIdx.x == 0)
+        *reinterpret_cast<float4*>(gb + A.NP * 288) = make_float4(__int_as_float((S + 127) << 23), 0.f, 0.f, 0.f);
 }
 
 // ---- main kernel -------------------------------------------------------------
@@ -390,7 +444,7 @@ __device__ __forceinline__ void decode_half(const uint4* src, uint32_t acol) {
 
 template <int NP, int KIND>
 __global__ void __launch_bounds__(kTCBlock, 2) k_gemm_tc(const __grid_constant__ TCArgs A) {
-    constexpr int GB = NP * 264;      // prepared X of one group (a multiple of 128 bytes)
+    constexpr int GB = tc_group_bytes(NP);  // prepared X of one group (a multiple of 16 bytes)
     constexpr int SB = GB + 256;      // + the tile's 128 scales of that group
     constexpr int WQ = KIND ? 3 : 2;  // 16-byte packed chunks per row and group
     constexpr int WH = KIND ? 2 : 1;  // chunks one half-row thread loads (chunks h .. h + WH - 1)
@@ -398,6 +452,8 @@ __global__ void __launch_bounds__(kTCBlock, 2) k_gemm_tc(const __grid_constant__
     constexpr uint32_t kIdesc = idesc_bf16(NP);
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* const wring = smem + kTCStages * SB;  // [kTCWStages][256][kTCWStride]
+    // constant A of the correction slice: 128 rows x 16 k, -offset * 2^-120 in k = 0, 1, 2
+    uint8_t* const aconst = wring + kTCWStages * kTCDecoders * kTCWStride;
     __shared__ __align__(8) uint64_t bar_full[kTCStages];
     __shared__ __align__(8) uint64_t bar_afull[2], bar_dfree[2], bar_mma[2];
     __shared__ uint32_t tmem_sh;
@@ -411,6 +467,13 @@ __global__ void __launch_bounds__(kTCBlock, 2) k_gemm_tc(const __grid_constant__
     const int64_t row = (int64_t)tile * kTCRows + r;
     const bool row_ok = tid < kTCDecoders && row < A.N;
 
+    if (tid < kTCRows) {  // row tid of the constant slice: chunk 0 (k 0 .. 7) and chunk 1 (k 8 .. 15)
+        const uint32_t c = KIND ? 0x8480u : 0x8400u;  // bf16 -4 * 2^-120 / -2 * 2^-120
+        uint8_t* rowa = aconst + (tid >> 3) * 256 + (tid & 7) * 16;
+        *reinterpret_cast<uint4*>(rowa) = make_uint4(c | (c << 16), c, 0u, 0u);
+        *reinterpret_cast<uint4*>(rowa + 128) = make_uint4(0u, 0u, 0u, 0u);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // read by the tensor cores
+    }
     if (tid == 0) {
         for (int s = 0; s < kTCStages; ++s) mbar_init(&bar_full[s], 1);
         for (int b = 0; b < 2; ++b) {
@@ -459,11 +522,13 @@ __global__ void __launch_bounds__(kTCBlock, 2) k_gemm_tc(const __grid_constant__
             if (!mbar_wait_warp(&bar_afull[b], (uint32_t)(i >> 1) & 1u)) { fail = true; break; }
             if (!mbar_wait_warp(&bar_full[s], (uint32_t)(i / kTCStages) & 1u)) { fail = true; break; }
             tc_fence_after();
-            const uint64_t bdesc = kmajor_desc(smem_addr(smem + s * SB));
+            const uint64_t bdesc = kmajor_desc(smem_addr(smem + s * SB), kTCBRowGroupB);
             const uint32_t dcol = tmem + 128u + (uint32_t)(b * NP), acol = tmem + (uint32_t)(b * 64);
 #pragma unroll
             for (int j = 0; j < 8; ++j)  // K slice j: 8 TMEM columns of A, 256 bytes (16 descriptor units) of B
                 mma_ts_warp(dcol, acol + 8u * j, bdesc + 16u * j, kIdesc, j > 0 ? 1u : 0u);
+            // correction slice: constant A (shared memory) x chunks 16, 17 of B
+            mma_ss_warp(dcol, kmajor_desc(smem_addr(aconst), 256), bdesc + 16u * 8, kIdesc);
             mma_commit_warp(&bar_mma[b]);
             committed = i + 1;
             // the next stage to fill, (i + kTCStages - 1) % kTCStages, last held group i - 1
@@ -516,18 +581,14 @@ __global__ void __launch_bounds__(kTCBlock, 2) k_gemm_tc(const __grid_constant__
                 }
                 tc_fence_after();
                 const uint8_t* st = smem + sp * SB;
-                const float sc = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + GB + 2 * r));
-                // correction pairs (offset * sum x, 2^S) of this half's columns, two per float4
-                const float4* cf = reinterpret_cast<const float4*>(st + NP * 256) + h * (NH / 2);
+                // D = 2^-S (sum u x - offset sum x): one factor s * 2^S per row and group
+                const float f = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + GB + 2 * r)) *
+                                *reinterpret_cast<const float*>(st + NP * 288);
                 float d[NH];
                 tmem_ld_cols<NH>(tmem + lane_base + 128u + (uint32_t)(bp * NP + h * NH), d);
 #pragma unroll
-                for (int q = 0; q < NH / 2; ++q) {
-                    const float4 v = cf[q];
-                    acc[2 * q] = fmaf(sc, fmaf(v.y, d[2 * q], -v.x), acc[2 * q]);
-                    acc[2 * q + 1] = fmaf(sc, fmaf(v.w, d[2 * q + 1], -v.z), acc[2 * q + 1]);
-                }
-                // D buffer read and the stage's scale and pairs consumed
+                for (int q = 0; q < NH; ++q) acc[q] = fmaf(f, d[q], acc[q]);
+                // D buffer read and the stage's scale and exponent consumed
                 tc_fence_before();
                 mbar_arrive(&bar_dfree[bp]);
             }
@@ -608,7 +669,7 @@ size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 size_t tc_smem_bytes(int np) {
     return std::max(kTCMinSmem, (size_t)kTCStages * (tc_group_bytes(np) + 256) +
-                                    (size_t)kTCWStages * kTCDecoders * kTCWStride + 1024);
+                                    (size_t)kTCWStages * kTCDecoders * kTCWStride + 4096 + 1024);
 }
 
 template <int NP, int KIND>
@@ -677,8 +738,10 @@ cudaError_t launch_gemm_tc(const void* packed, int grid, const uint16_t* scales,
     A.counters = reinterpret_cast<int32_t*>(w);
     w += align256((size_t)A.tiles * 4);
     A.partials = A.splits > 1 ? reinterpret_cast<float*>(w) : nullptr;
-    const int prep_warps = A.G * A.NP;
-    const int prep_ctas = std::max((prep_warps + 7) / 8, (A.tiles + 255) / 256);
+    // one CTA per group at least, and about 8 transposed scales per thread
+    const int64_t n_sprep = (int64_t)A.tiles * A.G * kTCRows;
+    const int prep_ctas = (int)std::max<int64_t>(
+        std::max<int64_t>(A.G, (A.tiles + 255) / 256), std::min<int64_t>((n_sprep + 2047) / 2048, 1184));
     k_prep_tc<<<prep_ctas, 256, 0, st>>>(A);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -153,7 +153,7 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
  * the size is ceil256(K/128 * 272) + ceil256(4 * ceil(N/32))
  * + ceil256(256 * min(8192, ceil(N/32) * ceil(K/256))).  For
  * M >= 32 (the tensor-core path) the size is exact and device independent:
- *   ceil256(K/128 * NP * 264) + ceil256(T * K/128 * 256) + ceil256(4 * T)
+ *   ceil256(K/128 * (NP * 288 + 16)) + ceil256(T * K/128 * 256) + ceil256(4 * T)
  *     + [S > 1] ceil256(T * S * NP * 512)
  * with NP = M rounded up to 16, T = ceil(N / 128) and S = the K split,
  * max(1, min(floor((296 + T/2) / T), 16, K / 128)).
@@ -175,7 +175,11 @@ TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *s
                            tb_stream_t stream);
 
 /* Small-batch GEMM Y = X W^T, 1 <= M <= 64.
- *   X          [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device.
+ *   X          [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device; finite, |x| < 2^120.
+ *              From M = 32 the activations of one 128-group share one
+ *              power-of-two exponent over all M rows: an element more than
+ *              about 2^110 below the group's largest |X[.][k]| over the batch
+ *              may count as zero.
  *   Y          [M][ldy] fp32 or bf16, ldy >= N, device; Y[m][n] for n < N written.
  *   workspace  tb_workspace_bytes(M, N, K) bytes. */
 TB_API tb_status_t tb_gemm(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *X,

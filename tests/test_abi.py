@@ -72,11 +72,12 @@ def test_workspace_sizes(lib):
         Mb = min(M, 16)
         assert tb.workspace_bytes(M, N, K) == al(2 * Mb * K) + al(8 * Mb * (K // 128))
     for M, N, K in ((32, 100, 5120), (33, 17408, 5120), (64, 7, 1024), (64, 40000, 4096)):
-        # tensor-core path: per group NP rows of prepared X (256 bytes) and NP pairs (8 bytes), NP = M
-        # rounded up to 16; the scales transposed per 128-row tile; a counter per tile; K-split partials of NP x 128 fp32 per tile and split
+        # tensor-core path: per group NP rows of prepared X and correction slice (288 bytes) and the
+        # group exponent (16 bytes), NP = M rounded up to 16; the scales transposed per 128-row tile;
+        # a counter per tile; K-split partials of NP x 128 fp32 per tile and split
         NP, tiles, G = (M + 15) // 16 * 16, (N + 127) // 128, K // 128
         splits = max(1, min((296 + tiles // 2) // tiles, 16, G))
-        want = (al(G * NP * 264) + al(tiles * G * 128 * 2) + al(4 * tiles) +
+        want = (al(G * (NP * 288 + 16)) + al(tiles * G * 128 * 2) + al(4 * tiles) +
                 (al(tiles * splits * NP * 128 * 4) if splits > 1 else 0))
         assert tb.workspace_bytes(M, N, K) == want, (M, N, K)
     for N, K in ((1, 128), (256, 1024), (17408, 5120), (100, 1408)):

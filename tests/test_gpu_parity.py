@@ -236,6 +236,22 @@ def test_gemm_parity(oracle, grid, M):
     assert_within(Y, Y64, Yabs, "f32", oracle, f"gemm M={M}")
 
 
+@pytest.mark.parametrize("grid", GRIDS)
+@pytest.mark.parametrize("M", [17, 32, 64])
+def test_gemm_row_magnitudes(oracle, grid, M):
+    """Batch rows 2^-45 .. 2^45 apart.  From M = 32 a group's activations share
+    one power-of-two exponent over the batch rows; every row must still be
+    within the tolerance of its own exact sum."""
+    N, K = 200, 1024
+    W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=1500 + M)
+    g = torch.Generator().manual_seed(1600 + M)
+    e = torch.randint(-45, 46, (M, 1), generator=g).float()
+    X = (torch.randn(M, K, generator=g) * torch.exp2(e)).to(torch.bfloat16)
+    Y64, Yabs = oracle.gemm64(p_ref, grid, s_ref, u16(X), N, K)
+    Y = tb.tb_gemm(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), X.to(DEV), N, K)
+    assert_within(Y, Y64, Yabs, "f32", oracle, f"row magnitudes M={M}")
+
+
 def test_gemm_strided_bf16_out(oracle):
     N, K, M = 40, 512, 12
     W, _, s_ref, p_ref = oracle_problem(oracle, tb.INT2, N, K, seed=900)
