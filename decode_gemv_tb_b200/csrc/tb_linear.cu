@@ -752,34 +752,48 @@ __device__ __forceinline__ void tm_warp(const TMLaunch& L, int part, uint32_t w,
         c_j = (int32_t)(local - c_tile * cpt);
     }
 
+    // The fields of the item under each cursor live in registers and are
+    // re-read (from the kernel parameters, through a dynamic index) only when
+    // the cursor moves on to another item.
+    struct Cur {
+        const uint16_t* scales;
+        const uint8_t* rec;
+        int64_t N;
+        int32_t G, cpt, T;
+    };
+    auto cur_of = [&](int i) {
+        const TMItem& I = items[i];
+        return Cur{I.scales, I.rec, I.N, I.G, I.cpt, I.T};
+    };
+
     // ---- issue cursor: lane 0 copies, every lane loads its row's scales
     int i_item = c_item;
     uint32_t i_tile = c_tile;
     int32_t i_j = c_j;
+    Cur ic = cur_of(i_item);
     auto issue = [&](uint32_t st, uint32_t bar, bool box, bool recs, uint32_t (&sc)[C]) {
-        const TMItem& I = items[i_item];
-        const int geff = min(C, I.G - i_j * C);
+        const int geff = min(C, ic.G - i_j * C);
         if (lane == 0) {
             if (box) {
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 tm_expect(bar, (uint32_t)(32 * WB + geff * kRecBytes));
                 tm_load_box(st, &maps[i_item], i_j * WB, (int)(i_tile * kRows), bar);
             }
-            if (recs) tm_load_bulk(st + kTMRec, I.rec + (int64_t)i_j * C * kRecBytes, (uint32_t)(geff * kRecBytes), bar);
+            if (recs) tm_load_bulk(st + kTMRec, ic.rec + (int64_t)i_j * C * kRecBytes, (uint32_t)(geff * kRecBytes), bar);
         }
         if (box) {
-            const int64_t row = min((int64_t)i_tile * kRows + lane, I.N - 1);
-            const uint16_t* sp = I.scales + row * I.G + i_j * C;
+            const int64_t row = min((int64_t)i_tile * kRows + lane, ic.N - 1);
+            const uint16_t* sp = ic.scales + row * ic.G + i_j * C;
 #pragma unroll
             for (int k = 0; k < C; ++k) sc[k] = k < geff ? (uint32_t)__ldg(sp + k) : 0u;
         }
     };
     auto advance = [&]() {
-        if (++i_j == items[i_item].cpt) {
+        if (++i_j == ic.cpt) {
             i_j = 0;
-            if (++i_tile == (uint32_t)items[i_item].T) {
+            if (++i_tile == (uint32_t)ic.T) {
                 i_tile = 0;
-                ++i_item;
+                if (++i_item < P.count) ic = cur_of(i_item);
             }
         }
     };
@@ -793,6 +807,7 @@ __device__ __forceinline__ void tm_warp(const TMLaunch& L, int part, uint32_t w,
 
     int32_t seg_j = c_j;
     bool first_seg = true;
+    Cur cc = cur_of(c_item);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
     for (int32_t k0 = 0; k0 < n; k0 += 2) {
@@ -811,22 +826,21 @@ __device__ __forceinline__ void tm_warp(const TMLaunch& L, int part, uint32_t w,
                     return;
                 }
                 const uint8_t* stage = base + u * kTMStageB;
-                const TMItem& I = items[c_item];
-                const int geff = min(C, I.G - c_j * C);
+                const int geff = min(C, cc.G - c_j * C);
 #pragma unroll
                 for (int gi = 0; gi < C; ++gi)
                     if (gi < geff) tm_step<KIND>(stage, gi, sc[u][gi], g, t, acc);
                 ++c_j;
                 const bool more = k + 1 < n;
-                if (c_j == I.cpt || !more) {
-                    tm_flush(L, part, wg, P.first + c_item, c_tile, seg_j == 0 && c_j == I.cpt, first_seg, acc[0],
+                if (c_j == cc.cpt || !more) {
+                    tm_flush(L, part, wg, P.first + c_item, c_tile, seg_j == 0 && c_j == cc.cpt, first_seg, acc[0],
                              acc[1], acc[2], acc[3]);
                     acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
                     first_seg = false;
                     seg_j = c_j = 0;
-                    if (more && ++c_tile == (uint32_t)I.T) {
+                    if (more && ++c_tile == (uint32_t)cc.T) {
                         c_tile = 0;
-                        ++c_item;
+                        cc = cur_of(++c_item);  // more chunks follow, so the next item exists
                     }
                 }
                 __syncwarp();
