@@ -49,6 +49,18 @@
  *               k = 32j .. 32j+31.  In plane p, bit m holds bit p of code
  *               32j+2m and bit 16+m holds bit p of code 32j+2m+1
  *               (m = 0..15).
+ *        ternary, 5 trits per byte ("b3", grid id 3; the 2-bit container is
+ *               the default ternary layout, this one is the optional denser
+ *               variant): digit d = c + 1 in {0,1,2}.  Row n is RB =
+ *               16 * ceil(26 G / 16) bytes (G = K/128); group j takes the
+ *               26 bytes from byte 26 j.  Group byte b < 25 holds codes
+ *               128 j + 5 b + i (i = 0..4) as sum_i d_i 3^i; byte 25 holds
+ *               codes 128 j + 125 + i (i = 0..2) the same way; bytes from
+ *               26 G on are zero.  Any byte value v decodes digit i as
+ *               floor(v / 3^i) mod 3, so the values 243..255 (never
+ *               written) still decode to ternary codes.  Byte a of a row is
+ *               bits [8 (a mod 4), 8 (a mod 4) + 7] of uint32 word a / 4
+ *               (the bytes' memory order).
  *  R7  W is [N out][K in] row-major, y = W x, no bias.
  *  R8  products are summed in k order in fp64; fp32 output is the RNE
  *      rounding of that sum; bf16 output is the RNE rounding of the fp32.
@@ -71,15 +83,15 @@
 #define TBO_GROUP 128
 
 /* grid ids, same numbering the public interface uses */
-enum { TBO_TERNARY = 0, TBO_INT2 = 1, TBO_INT3 = 2 };
+enum { TBO_TERNARY = 0, TBO_INT2 = 1, TBO_INT3 = 2, TBO_TERNARY_B3 = 3 };
 
-static int grid_ok(int g) { return g == TBO_TERNARY || g == TBO_INT2 || g == TBO_INT3; }
+static int grid_ok(int g) { return g == TBO_TERNARY || g == TBO_INT2 || g == TBO_INT3 || g == TBO_TERNARY_B3; }
 
-/* [TB-how]: the three grids */
-static int grid_qmin(int g) { return g == TBO_TERNARY ? -1 : (g == TBO_INT2 ? -2 : -4); }
-static int grid_qmax(int g) { return g == TBO_TERNARY ? 1 : (g == TBO_INT2 ? 1 : 3); }
-/* R5 */
-static int grid_offset(int g) { return g == TBO_INT3 ? 4 : 2; }
+/* [TB-how]: the three grids (the 5-trits-per-byte layout stores the ternary grid) */
+static int grid_qmin(int g) { return (g == TBO_TERNARY || g == TBO_TERNARY_B3) ? -1 : (g == TBO_INT2 ? -2 : -4); }
+static int grid_qmax(int g) { return g == TBO_INT3 ? 3 : 1; }
+/* R5; R6 for the base-3 digit */
+static int grid_offset(int g) { return g == TBO_INT3 ? 4 : (g == TBO_TERNARY_B3 ? 1 : 2); }
 /* R1: divisor d = |qmin| */
 static int grid_scale_div(int g) { return -grid_qmin(g); }
 
@@ -156,11 +168,40 @@ int tbo_quantize(float w, uint16_t scale_bf16, int grid, int *bad)
 
 /* ---- bit layout (R6) ----------------------------------------------------- */
 
-int64_t tbo_row_words(int grid, int64_t K) { return grid == TBO_INT3 ? 3 * (K / 32) : K / 16; }
+/* R6, 5-trits-per-byte layout: bytes per group and per row */
+#define TBO_B3_GROUP_BYTES 26
+static int64_t b3_row_bytes(int64_t K) { return 16 * ((TBO_B3_GROUP_BYTES * (K / TBO_GROUP) + 15) / 16); }
+
+int64_t tbo_row_words(int grid, int64_t K)
+{
+    if (grid == TBO_TERNARY_B3) return b3_row_bytes(K) / 4;
+    return grid == TBO_INT3 ? 3 * (K / 32) : K / 16;
+}
+
+/* byte of row position k and its base-3 digit index */
+static void b3_place(int64_t k, int64_t *byte, int *digit)
+{
+    int64_t j = k / TBO_GROUP, r = k % TBO_GROUP;
+    *byte = TBO_B3_GROUP_BYTES * j + r / 5;
+    *digit = (int)(r % 5);
+}
+
+static unsigned pow3(int i)
+{
+    unsigned p = 1;
+    while (i-- > 0) p *= 3;
+    return p;
+}
 
 static void put_code(uint32_t *row, int grid, int64_t k, unsigned u)
 {
-    if (grid == TBO_INT3) {
+    if (grid == TBO_TERNARY_B3) {
+        int64_t a;
+        int i;
+        b3_place(k, &a, &i);
+        /* the row starts zeroed and a byte's digits never exceed 242 in total: no carry */
+        row[a / 4] += (uint32_t)(u * pow3(i)) << (8 * (a % 4));
+    } else if (grid == TBO_INT3) {
         int64_t block = k / 32;
         int i = (int)(k % 32);
         int bitpos = (i % 2 == 0) ? i / 2 : 16 + i / 2;
@@ -176,7 +217,13 @@ static void put_code(uint32_t *row, int grid, int64_t k, unsigned u)
 
 static unsigned get_code(const uint32_t *row, int grid, int64_t k)
 {
-    if (grid == TBO_INT3) {
+    if (grid == TBO_TERNARY_B3) {
+        int64_t a;
+        int i;
+        b3_place(k, &a, &i);
+        unsigned v = (row[a / 4] >> (8 * (a % 4))) & 0xFFu;
+        return (v / pow3(i)) % 3u;
+    } else if (grid == TBO_INT3) {
         int64_t block = k / 32;
         int i = (int)(k % 32);
         int bitpos = (i % 2 == 0) ? i / 2 : 16 + i / 2;

@@ -29,9 +29,11 @@ LIB = os.path.join(HERE, "libtb_oracle.so")
 
 TERNARY, INT2, INT3 = 0, 1, 2
 GRIDS = (TERNARY, INT2, INT3)
-GRID_NAMES = {TERNARY: "ternary", INT2: "int2", INT3: "int3"}
+# the ternary grid in the optional 5-trits-per-byte layout
+TERNARY_B3 = 3
+GRID_NAMES = {TERNARY: "ternary", INT2: "int2", INT3: "int3", TERNARY_B3: "ternary_b3"}
 # [how it works]: the three codeword grids
-GRID_RANGE = {TERNARY: (-1, 1), INT2: (-2, 1), INT3: (-4, 3)}
+GRID_RANGE = {TERNARY: (-1, 1), INT2: (-2, 1), INT3: (-4, 3), TERNARY_B3: (-1, 1)}
 GROUP = 128
 
 CFLAGS = ["-O2", "-fno-fast-math", "-ffp-contract=off", "-std=c11", "-shared", "-fPIC"]

@@ -15,6 +15,8 @@ from decode_gemv_tb_b200 import synth
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 GRIDS = (0, 1, 2)
 NAME2GRID = {"ternary": 0, "int2": 1, "int3": 2}
+B3 = 3                # the ternary grid in the optional 5-trits-per-byte layout
+LAYOUTS = GRIDS + (B3,)
 
 
 def page_facts():
@@ -229,6 +231,128 @@ def test_every_2bit_word_pattern_roundtrips(oracle):
                 assert diff[0] // (3 if grid == 2 else 1) == pos // per
 
 
+# ---------------------------------------------------------------- 5 trits per byte
+
+def _parse_segments(field: str):
+    out = []
+    for seg in field.split("|"):
+        seg = seg.strip()
+        if "*" in seg:
+            v, cnt = seg.split("*")
+            out += [int(v)] * int(cnt)
+        else:
+            out += [int(v) for v in seg.split(",")]
+    return out
+
+
+def test_b3_golden_examples(oracle):
+    n_lines = 0
+    with open(os.path.join(GOLDEN, "format_b3_examples.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            codes, words, _why = [p.strip() for p in line.split(";", 2)]
+            c = _parse_segments(codes)
+            K = len(c)
+            assert K in (128, 256)
+            packed, bad = oracle.pack(np.array(c, np.float32)[None, :], B3,
+                                      np.full((1, K // 128), bf16_of(1.0), np.uint16))
+            assert bad == 0
+            assert [int(v) for v in packed[0]] == [int(w, 16) for w in words.split(",")], line
+            assert list(oracle.unpack(packed, B3, 1, K)[0]) == c
+            n_lines += 1
+    assert n_lines >= 12
+
+
+def test_b3_every_byte_value_decodes_base3(oracle):
+    """Each byte value 0..255 written straight into the packed row decodes,
+    digit by digit, to Python's floor(v / 3^i) mod 3, minus 1; the other
+    bytes (zero) decode to -1 and the row padding is never read."""
+    K = 128
+    rw = oracle.row_words(B3, K)
+    assert rw == 8  # 26 bytes padded to 32
+    for b, ndig in ((0, 5), (3, 5), (7, 5), (24, 5), (25, 3)):
+        rows = np.zeros((256, rw), np.uint32)
+        for v in range(256):
+            rows[v, b // 4] = v << (8 * (b % 4))
+        rows[:, 7] = 0xFFFFFFFF  # padding bytes 28..31
+        codes = oracle.unpack(rows, B3, 256, K)
+        for v in range(256):
+            assert list(codes[v, 5 * b: 5 * b + ndig]) == [(v // 3 ** i) % 3 - 1 for i in range(ndig)]
+            assert np.all(np.delete(codes[v], range(5 * b, 5 * b + ndig)) == -1)
+
+
+def test_b3_pack_is_a_bijection_on_digit_patterns(oracle):
+    """All 3^5 patterns of a full byte pack to the distinct values 0..242,
+    each the base-3 number of its digits c + 1; all 3^3 patterns of the
+    last byte to 0..26."""
+    import itertools
+    ones = None
+    for first, n, byte in ((10, 5, 2), (125, 3, 25)):
+        pats = list(itertools.product((-1, 0, 1), repeat=n))
+        rows = np.full((len(pats), 128), -1.0, np.float32)
+        for r, pat in enumerate(pats):
+            rows[r, first:first + n] = pat
+        ones = np.full((len(pats), 1), bf16_of(1.0), np.uint16)
+        packed, bad = oracle.pack(rows, B3, ones)
+        assert bad == 0
+        vals = [(int(packed[r, byte // 4]) >> (8 * (byte % 4))) & 0xFF for r in range(len(pats))]
+        assert sorted(vals) == list(range(3 ** n))
+        for pat, v in zip(pats, vals):
+            assert v == sum((d + 1) * 3 ** i for i, d in enumerate(pat))
+
+
+def test_b3_bytes_closed_form(oracle):
+    facts = page_facts()
+    g, sbits = int(facts["group_size"]), int(facts["scale_bits"])
+    assert 25 * 5 + 3 == g           # 25 full bytes and one of three trits hold a group
+    assert 8 / 5 >= math.log2(3)     # 5 trits fit a byte: 3^5 = 243 <= 256
+    assert 3 ** 5 <= 256 < 3 ** 6
+    for N, K in ((1, 128), (3, 256), (5, 640), (256, 1024), (2048, 6144), (17408, 5120)):
+        G = K // g
+        assert oracle.packed_bytes(B3, N, K) == N * 16 * math.ceil(26 * G / 16)
+        bits = (8 * oracle.packed_bytes(B3, N, K) + sbits * N * G) / (N * K)
+        assert bits <= 2 + sbits / g      # never above the 2-bit container
+        if G % 8 == 0:                   # 8 groups = 208 bytes = 13 x 16: no padding
+            assert bits == 26 * 8 / g + sbits / g == 1.75
+
+
+def test_b3_quantizes_and_scales_like_ternary(oracle):
+    rng = np.random.default_rng(90)
+    for _ in range(2000):
+        s = bf16_of(float(abs(rng.standard_normal()) * 10 ** rng.uniform(-6, 3)) + 1e-30)
+        w = float(np.float32(rng.standard_normal() * bf16_value(s) * 3))
+        assert oracle.quantize(w, s, B3) == (_exact_code(w, s, 0), 0)
+    one = bf16_of(1.0)
+    assert oracle.quantize(float("nan"), one, B3) == (0, 1)
+    assert oracle.quantize(float("inf"), one, B3) == (1, 1)
+    assert oracle.quantize(float("-inf"), one, B3) == (-1, 1)
+    for bad_s in (0x0000, 0x8000, bf16_of(-1.0), 0x7F80, 0x7FC0):
+        assert oracle.quantize(0.7, bad_s, B3) == (0, 1)
+    W = (rng.standard_normal((6, 384)) * 0.02).astype(np.float32)
+    t = torch.from_numpy(W).view(6, 3, 128).abs().amax(-1)  # ternary divisor |qmin| = 1
+    assert np.array_equal(oracle.scales_absmax(W, B3), t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+
+
+@pytest.mark.parametrize("K", [128, 384, 640, 1024])
+def test_b3_exact_reconstruction_roundtrip(oracle, K):
+    rng = np.random.default_rng(100 + K)
+    N = 7
+    c = rng.integers(-1, 2, size=(N, K)).astype(np.int64)
+    sb = np.array([[bf16_of(float(abs(rng.standard_normal()) * 0.02 + 1e-3)) for _ in range(K // 128)]
+                   for _ in range(N)], dtype=np.uint16)
+    svals = np.vectorize(bf16_value)(sb).astype(np.float64)
+    W = (c * np.repeat(svals, 128, axis=1)).astype(np.float32)
+    packed, bad = oracle.pack(W, B3, sb)
+    assert bad == 0
+    assert packed.shape == (N, 4 * math.ceil(26 * (K // 128) / 16))
+    assert np.array_equal(oracle.unpack(packed, B3, N, K).astype(np.int64), c)
+    # the padding words past 26 G bytes stay zero
+    tail = packed.view(np.uint8).reshape(N, -1)[:, 26 * (K // 128):]
+    assert not tail.any()
+
+
 # ---------------------------------------------------------------- scales
 
 @pytest.mark.parametrize("grid", GRIDS)
@@ -283,7 +407,7 @@ def _random_problem(oracle, grid, N, K, seed):
     return c, sb, W64, packed, xb
 
 
-@pytest.mark.parametrize("grid", GRIDS)
+@pytest.mark.parametrize("grid", LAYOUTS)
 def test_gemv_equals_dense_matmul(oracle, grid):
     """Textbook reduction: y equals numpy's matmul of the dequantized
     matrix (built here directly as c*s, not by the oracle) with x."""
@@ -300,7 +424,7 @@ def test_gemv_integer_exact(oracle):
     """Integer x and power-of-two scales: y is an exact integer multiple of
     the scale, equal to an int64 matmul."""
     rng = np.random.default_rng(40)
-    for grid in GRIDS:
+    for grid in LAYOUTS:
         lo, hi = oracle.GRID_RANGE[grid]
         N, K = 19, 1024
         c = rng.integers(lo, hi + 1, size=(N, K)).astype(np.int64)
@@ -318,7 +442,7 @@ def test_gemv_permutation_rows(oracle):
     entries of x: y[n] = x[p(n)].  Non-square, so a transposed operand or
     a wrong row stride fails."""
     rng = np.random.default_rng(50)
-    for grid in GRIDS:
+    for grid in LAYOUTS:
         N, K = 24, 384
         p = rng.permutation(K)[:N]
         c = np.zeros((N, K))
