@@ -41,8 +41,11 @@ SPEC_HBM_GBS = 8000.0
 
 def algo_bytes(N, K, grid, M=1, ybytes=4):
     """packed codes + bf16 scales + activations + outputs of one product."""
-    bits = 3 if grid == synth.INT3 else 2
-    return N * K * bits // 8 + N * (K // 128) * 2 + M * K * 2 + M * N * ybytes
+    if grid == tb.TERNARY_B3:  # 26 bytes per 128-group, rows padded to 16 bytes
+        codes = N * 16 * ((26 * (K // 128) + 15) // 16)
+    else:
+        codes = N * K * (3 if grid == synth.INT3 else 2) // 8
+    return codes + N * (K // 128) * 2 + M * K * 2 + M * N * ybytes
 
 
 def traffic_per_launch(algorithmic_bytes):
@@ -395,6 +398,17 @@ def rows_section(dev, stream):
         c2[m.name] = gemv_row(m.N, m.K, m.grid, p2, s2, synth.activations(m.K, seed=m.seed, device=dev))
         del W
     out["gemv_config2"] = c2
+    # the same ternary cases in the optional 5-trits-per-byte layout
+    c2b = {}
+    for m in synth.config2_cases():
+        if m.grid != synth.TERNARY:
+            continue
+        W = synth.gaussian_weights(m.N, m.K, seed=m.seed, device=dev)
+        s2 = tb.tb_scales_absmax(W, tb.TERNARY_B3)
+        p2 = tb.tb_pack(W, tb.TERNARY_B3, s2)
+        c2b[m.name] = gemv_row(m.N, m.K, tb.TERNARY_B3, p2, s2, synth.activations(m.K, seed=m.seed, device=dev))
+        del W
+    out["gemv_config2_ternary_5trit"] = c2b
 
     # one isolated 8B-like layer (q, o 3-bit; k, v 2-bit; MLP ternary), one tb_layer_gemv per launch
     items = []

@@ -14,7 +14,10 @@ using namespace tb;
 
 namespace {
 
-bool grid_ok(int g) { return g == TB_GRID_TERNARY || g == TB_GRID_INT2 || g == TB_GRID_INT3; }
+bool grid_ok(int g) {
+    return g == TB_GRID_TERNARY || g == TB_GRID_INT2 || g == TB_GRID_INT3 || g == TB_GRID_TERNARY_B3;
+}
+bool is_b3(int g) { return g == TB_GRID_TERNARY_B3; }
 bool dtype_ok(int d) { return d == TB_F32 || d == TB_BF16; }
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool shape_ok(int64_t N, int64_t K) { return N >= 1 && K >= kGroup && K % kGroup == 0; }
@@ -261,7 +264,7 @@ const char* tb_status_string(tb_status_t s) {
 
 size_t tb_packed_bytes(tb_grid_t grid, int64_t N, int64_t K) {
     if (!grid_ok(grid) || !shape_ok(N, K)) return 0;
-    return (size_t)(N * row_bytes(grid, K));
+    return (size_t)(N * (is_b3(grid) ? b3_row_bytes(K) : row_bytes(grid, K)));
 }
 
 size_t tb_scale_bytes(int64_t N, int64_t K) {
@@ -274,7 +277,9 @@ tb_status_t tb_scales_absmax(const void* W, tb_dtype_t w_dtype, int64_t N, int64
     if (!W || !scales || !dtype_ok(w_dtype) || !grid_ok(grid)) return TB_ERR_ARG;
     if (!shape_ok(N, K)) return TB_ERR_SHAPE;
     if (!aligned(W, 16) || !aligned(scales, 2)) return TB_ERR_ALIGN;
-    return cuda_status(launch_scales(W, w_dtype, N, K, grid, scales, static_cast<cudaStream_t>(stream)));
+    // the 5-trits-per-byte layout stores the ternary grid: same scale rule
+    return cuda_status(launch_scales(W, w_dtype, N, K, is_b3(grid) ? (int)TB_GRID_TERNARY : (int)grid, scales,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 tb_status_t tb_pack(const void* W, tb_dtype_t w_dtype, int64_t N, int64_t K, tb_grid_t grid,
@@ -311,6 +316,7 @@ size_t tb_layer_workspace_bytes(const tb_linear_t* items, int n_items) {
     int64_t tiles = 0, chunks = 0;
     for (int i = 0; i < n_items; ++i) {
         if (!shape_ok(items[i].N, items[i].K) || !grid_ok(items[i].grid)) return 0;
+        if (is_b3(items[i].grid)) continue;  // launched on their own, without workspace
         const int64_t t = (items[i].N + 31) / 32, C = tm_chunk_groups(items[i].grid);
         b += tm_item_workspace(items[i].K);
         tiles += t;
@@ -328,6 +334,10 @@ tb_status_t tb_gemv(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if ((s = check_out(y, y_dtype)) != TB_OK) return s;
     if (!workspace) return TB_ERR_ARG;
     if (!aligned(x, 16) || !aligned(workspace, 256)) return TB_ERR_ALIGN;
+    if (is_b3(grid)) {
+        if (!gemv_b3_supported(K)) return TB_ERR_UNSUPPORTED;
+        return cuda_status(launch_gemv_b3(packed, scales, x, y, y_dtype, N, K, static_cast<cudaStream_t>(stream)));
+    }
     Item it = make_item(packed, grid, scales, x, K, y, y_dtype, N, 1, N, K);
     return launch_tma_items(&it, 1, workspace, workspace_bytes, false, static_cast<cudaStream_t>(stream));
 }
@@ -343,6 +353,16 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if (!workspace) return TB_ERR_ARG;
     if (!aligned(X, 16) || ldx % 8 != 0 || !aligned(workspace, 256)) return TB_ERR_ALIGN;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (is_b3(grid)) {  // one GEMV launch per batch row
+        if (!gemv_b3_supported(K)) return TB_ERR_UNSUPPORTED;
+        const size_t ysz = y_dtype == TB_F32 ? 4 : 2;
+        for (int64_t m = 0; m < M; ++m) {
+            const cudaError_t e = launch_gemv_b3(packed, scales, X + m * ldx, static_cast<char*>(Y) + m * ldy * ysz,
+                                                 y_dtype, N, K, st);
+            if (e != cudaSuccess) return TB_ERR_CUDA;
+        }
+        return TB_OK;
+    }
     if (M == 1) {
         Item it = make_item(packed, grid, scales, X, ldx, Y, y_dtype, N, 1, N, K);
         return launch_tma_items(&it, 1, workspace, workspace_bytes, false, st);
@@ -371,6 +391,7 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
     if ((flags & ~(unsigned)TB_FLAG_OVERLAP_PREVIOUS) != 0 || !workspace) return TB_ERR_ARG;
     if (!aligned(workspace, 256)) return TB_ERR_ALIGN;
     Item its[kMaxItems];
+    int n_main = 0;
     for (int i = 0; i < n_items; ++i) {
         const tb_linear_t& l = items[i];
         tb_status_t s = check_weights(l.packed, l.grid, l.scales, l.N, l.K);
@@ -378,10 +399,25 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
         if (!l.x) return TB_ERR_ARG;
         if ((s = check_out(l.y, l.y_dtype)) != TB_OK) return s;
         if (!aligned(l.x, 16)) return TB_ERR_ALIGN;
-        its[i] = make_item(l.packed, l.grid, l.scales, l.x, l.K, l.y, l.y_dtype, l.N, 1, l.N, l.K);
+        if (is_b3(l.grid)) {
+            if (!gemv_b3_supported(l.K)) return TB_ERR_UNSUPPORTED;
+            continue;
+        }
+        its[n_main++] = make_item(l.packed, l.grid, l.scales, l.x, l.K, l.y, l.y_dtype, l.N, 1, l.N, l.K);
     }
-    return launch_tma_items(its, n_items, workspace, workspace_bytes, (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0,
-                           static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (n_main > 0) {
+        const tb_status_t s = launch_tma_items(its, n_main, workspace, workspace_bytes,
+                                               (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0, st);
+        if (s != TB_OK) return s;
+    }
+    // items in the 5-trits-per-byte layout: one launch each, after the grouped launch
+    for (int i = 0; i < n_items; ++i) {
+        const tb_linear_t& l = items[i];
+        if (!is_b3(l.grid)) continue;
+        if (launch_gemv_b3(l.packed, l.scales, l.x, l.y, l.y_dtype, l.N, l.K, st) != cudaSuccess) return TB_ERR_CUDA;
+    }
+    return TB_OK;
 }
 
 }  // extern "C"
@@ -432,6 +468,10 @@ tb_status_t tb_gemv_noalloc(const void* packed, tb_grid_t grid, const uint16_t* 
     if (!x) return TB_ERR_ARG;
     if ((s = check_out(y, y_dtype)) != TB_OK) return s;
     if (!aligned(x, 16)) return TB_ERR_ALIGN;
+    if (is_b3(grid)) {  // needs no scratch
+        if (!gemv_b3_supported(K)) return TB_ERR_UNSUPPORTED;
+        return cuda_status(launch_gemv_b3(packed, scales, x, y, y_dtype, N, K, static_cast<cudaStream_t>(stream)));
+    }
     // the size rule is checked before any CUDA call
     if (tb_workspace_bytes(1, N, K) > (size_t)TB_NOALLOC_SCRATCH_BYTES) return TB_ERR_UNSUPPORTED;
     void* scratch = noalloc_scratch();

@@ -9,6 +9,12 @@ namespace tb {
 
 struct Launch;
 
+// The ternary grid in the optional 5-trits-per-byte layout (include/tb.h):
+// 26 bytes per 128-group, rows padded to 16 bytes.
+constexpr int kTernaryB3 = 3;
+constexpr int64_t kB3GroupBytes = 26;
+__host__ __device__ inline int64_t b3_row_bytes(int64_t K) { return 16 * ((kB3GroupBytes * (K / 128) + 15) / 16); }
+
 cudaError_t launch_scales(const void* W, int w_dtype, int64_t N, int64_t K, int grid, uint16_t* scales,
                           cudaStream_t st);
 cudaError_t launch_pack(const void* W, int w_dtype, int64_t N, int64_t K, int grid, const uint16_t* scales,
@@ -35,6 +41,13 @@ bool encode_gemv_tma_map(CUtensorMap* map, const void* packed, int grid, int64_t
 int gemv_tma_resident_warps();
 // bounded waits of k_gemv_tma that gave up since the last call (clears)
 unsigned int take_gemv_timeouts();
+
+// Batch-1 GEMV over the 5-trits-per-byte layout: one launch, no workspace.
+// The activations are staged in shared memory, which bounds K
+// (gemv_b3_supported).
+bool gemv_b3_supported(int64_t K);
+cudaError_t launch_gemv_b3(const void* packed, const uint16_t* scales, const uint16_t* x, void* y, int ydt,
+                           int64_t N, int64_t K, cudaStream_t st);
 
 // Small-batch GEMM on the tcgen05 tensor cores (2 <= M <= 64): preparation
 // kernel + main kernel.  Workspace: gemm_tc_workspace_bytes(M, N, K) bytes,

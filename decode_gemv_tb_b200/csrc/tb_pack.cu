@@ -6,7 +6,8 @@
 // 다른가: codewords are produced by rounding.  Tie rule, scale rule and the
 // bit layout are the library's (include/tb.h).
 //
-// All three kernels are HBM-bound streams: scales read the weights once,
+// The 5-trits-per-byte ternary layout has its own pack and unpack kernels.
+// All of them are HBM-bound streams: scales read the weights once,
 // pack reads weights + scales and writes the packed codes, unpack reads
 // the codes and writes one int8 per weight.
 #include "tb_device.cuh"
@@ -25,6 +26,9 @@ struct WLoad<kF32> {
         float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx));
         v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
     }
+    static __device__ __forceinline__ float one(const void* base, int64_t idx) {
+        return __ldg(static_cast<const float*>(base) + idx);
+    }
 };
 template <>
 struct WLoad<kBF16> {
@@ -34,6 +38,9 @@ struct WLoad<kBF16> {
         v[1] = __uint_as_float(h.x & 0xFFFF0000u);
         v[2] = __uint_as_float(h.y << 16);
         v[3] = __uint_as_float(h.y & 0xFFFF0000u);
+    }
+    static __device__ __forceinline__ float one(const void* base, int64_t idx) {
+        return __uint_as_float((uint32_t)__ldg(static_cast<const uint16_t*>(base) + idx) << 16);
     }
 };
 
@@ -186,6 +193,38 @@ __global__ void __launch_bounds__(256) k_pack3(const void* __restrict__ W, int64
     warp_count(bad, bad_count);
 }
 
+// 5 trits per byte (ternary): one thread per byte of the padded row.  Group
+// byte b < 25 holds codes 5b .. 5b+4 of its group, byte 25 codes 125..127,
+// as sum_i (c_i + 1) 3^i; padding bytes are written as zero.
+template <int WT>
+__global__ void __launch_bounds__(256) k_pack_b3(const void* __restrict__ W, int64_t N, int64_t K,
+                                                 const uint16_t* __restrict__ S, uint8_t* __restrict__ P,
+                                                 int32_t* __restrict__ bad_count) {
+    const int64_t G = K / kGroup, RB = b3_row_bytes(K);
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    int bad = 0;
+    if (t < N * RB) {
+        const int64_t n = t / RB, a = t - n * RB;
+        uint32_t v = 0;
+        if (a < kB3GroupBytes * G) {
+            const int64_t j = a / kB3GroupBytes;
+            const int b = (int)(a - j * kB3GroupBytes);
+            const QScale q = make_qscale(S[n * G + j]);
+            const int64_t k0 = n * K + j * kGroup + 5 * b;
+            uint32_t p3 = 1;
+#pragma unroll
+            for (int i = 0; i < 5; ++i) {
+                if (i < 3 || b < 25) {
+                    v += (uint32_t)(quant_code(WLoad<WT>::one(W, k0 + i), q, -1, 1, bad) + 1) * p3;
+                    p3 *= 3u;
+                }
+            }
+        }
+        P[t] = (uint8_t)v;
+    }
+    warp_count(bad, bad_count);
+}
+
 // ---- unpack -------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_unpack2(const uint32_t* __restrict__ P, int64_t nwords,
                                                  int8_t* __restrict__ C) {
@@ -231,6 +270,27 @@ __global__ void __launch_bounds__(256) k_unpack3(const uint32_t* __restrict__ P,
     dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
+// 5 trits per byte: one thread per group byte; digit i of byte value v is
+// floor(v / 3^i) mod 3, the code that digit minus 1.
+__global__ void __launch_bounds__(256) k_unpack_b3(const uint8_t* __restrict__ P, int64_t N, int64_t K,
+                                                   int8_t* __restrict__ C) {
+    const int64_t G = K / kGroup, RB = b3_row_bytes(K), per_row = kB3GroupBytes * G;
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= N * per_row) return;
+    const int64_t n = t / per_row, a = t - n * per_row;
+    const int64_t j = a / kB3GroupBytes;
+    const int b = (int)(a - j * kB3GroupBytes);
+    uint32_t v = __ldg(P + n * RB + a);
+    int8_t* out = C + n * K + j * kGroup + 5 * b;
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        if (i < 3 || b < 25) {
+            out[i] = (int8_t)((int)(v % 3u) - 1);
+            v /= 3u;
+        }
+    }
+}
+
 inline unsigned nblk(int64_t threads) { return (unsigned)((threads + 255) / 256); }
 
 }  // namespace
@@ -250,7 +310,12 @@ cudaError_t launch_pack(const void* W, int wt, int64_t N, int64_t K, int grid, c
         if (e != cudaSuccess) return e;
     }
     uint32_t* out = static_cast<uint32_t*>(P);
-    if (grid == kInt3) {
+    if (grid == kTernaryB3) {
+        const int64_t n = N * b3_row_bytes(K);
+        uint8_t* bytes = static_cast<uint8_t*>(P);
+        if (wt == kF32) k_pack_b3<kF32><<<nblk(n), 256, 0, st>>>(W, N, K, S, bytes, bad_count);
+        else k_pack_b3<kBF16><<<nblk(n), 256, 0, st>>>(W, N, K, S, bytes, bad_count);
+    } else if (grid == kInt3) {
         const int64_t n = N * (K / 32);
         if (wt == kF32) k_pack3<kF32><<<nblk(n), 256, 0, st>>>(W, N, K, S, out, bad_count);
         else k_pack3<kBF16><<<nblk(n), 256, 0, st>>>(W, N, K, S, out, bad_count);
@@ -264,7 +329,10 @@ cudaError_t launch_pack(const void* W, int wt, int64_t N, int64_t K, int grid, c
 
 cudaError_t launch_unpack(const void* P, int grid, int64_t N, int64_t K, int8_t* C, cudaStream_t st) {
     const uint32_t* in = static_cast<const uint32_t*>(P);
-    if (grid == kInt3) {
+    if (grid == kTernaryB3) {
+        const int64_t n = N * kB3GroupBytes * (K / kGroup);
+        k_unpack_b3<<<nblk(n), 256, 0, st>>>(static_cast<const uint8_t*>(P), N, K, C);
+    } else if (grid == kInt3) {
         const int64_t n = N * (K / 32);
         k_unpack3<<<nblk(n), 256, 0, st>>>(in, n, C);
     } else {

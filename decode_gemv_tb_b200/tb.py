@@ -16,6 +16,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libtb_b200.so")
 
 TERNARY, INT2, INT3 = 0, 1, 2
+TERNARY_B3 = 3  # the ternary grid, 5 codes per byte
 F32, BF16 = 0, 1
 MAX_LAYER_ITEMS = 16
 FLAG_OVERLAP_PREVIOUS = 1

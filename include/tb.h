@@ -39,8 +39,16 @@
  *     k = 32j .. 32j+31 in planes p = 0, 1, 2 (consecutive words); bit m of
  *     plane p is bit p of u for code 32j+2m, bit 16+m of plane p is bit p of
  *     u for code 32j+2m+1, m = 0..15.
- *   Bytes per weight including the scales: 2.125 / 8 (ternary, 2-bit) and
- *   3.125 / 8 (3-bit).
+ *   TB_GRID_TERNARY_B3 -- the ternary grid, 5 codes per byte: digit
+ *     d = c + 1 in {0,1,2}; row n is 16 * ceil(26 K/128 / 16) bytes; group j
+ *     takes the 26 bytes from byte 26 j: group byte b < 25 is
+ *     sum_{i<5} d(128 j + 5 b + i) 3^i, byte 25 is sum_{i<3} d(128 j + 125 +
+ *     i) 3^i; the row's remaining bytes are zero.  Any byte value v decodes
+ *     digit i as floor(v / 3^i) mod 3 (243..255 are never written).  No byte
+ *     holds codes of two groups.
+ *   Bytes per weight including the scales: 2.125 / 8 (ternary, 2-bit),
+ *   3.125 / 8 (3-bit) and 1.75 / 8 (5 trits per byte, when K/128 is a
+ *   multiple of 8; the row padding adds at most 15 bytes otherwise).
  *
  * QUANTIZATION RULES (readings where the pages are silent)
  *   scale  s = bf16_rne(absmax / d), d = |qmin| = 1, 2, 4 for ternary,
@@ -95,7 +103,8 @@ typedef void *tb_stream_t; /* a cudaStream_t */
 typedef enum {
     TB_GRID_TERNARY = 0, /* {-1, 0, 1}, 2-bit container, offset 2 */
     TB_GRID_INT2 = 1,    /* {-2, -1, 0, 1}, offset 2 */
-    TB_GRID_INT3 = 2     /* {-4, ..., 3}, three bit-planes, offset 4 */
+    TB_GRID_INT3 = 2,    /* {-4, ..., 3}, three bit-planes, offset 4 */
+    TB_GRID_TERNARY_B3 = 3 /* {-1, 0, 1}, 5 trits per byte (optional denser ternary layout) */
 } tb_grid_t;
 
 typedef enum { TB_F32 = 0, TB_BF16 = 1 } tb_dtype_t;
@@ -116,7 +125,8 @@ TB_API int tb_version(void);
 TB_API const char *tb_status_string(tb_status_t status);
 
 /* Bytes of the packed codes of an N x K matrix (scales not included):
- * N*K/4 for ternary and 2-bit, 3*N*K/8 for 3-bit; 0 for bad arguments. */
+ * N*K/4 for ternary and 2-bit, 3*N*K/8 for 3-bit, N * 16 * ceil(26 K/128 /
+ * 16) for 5 trits per byte; 0 for bad arguments. */
 TB_API size_t tb_packed_bytes(tb_grid_t grid, int64_t N, int64_t K);
 
 /* Bytes of the bf16 scales of an N x K matrix: N * (K/128) * 2; 0 for bad
@@ -124,7 +134,7 @@ TB_API size_t tb_packed_bytes(tb_grid_t grid, int64_t N, int64_t K);
 TB_API size_t tb_scale_bytes(int64_t N, int64_t K);
 
 /* Group scales by absmax (rule above; ThinkBit page, 어떻게 동작하나, one
- * bf16 scale per 128 weights).
+ * bf16 scale per 128 weights).  TB_GRID_TERNARY_B3 uses the ternary rule.
  *   W       [N][K] fp32 or bf16 (w_dtype), device.
  *   scales  [N][K/128] bf16 bit patterns, device, written. */
 TB_API tb_status_t tb_scales_absmax(const void *W, tb_dtype_t w_dtype, int64_t N, int64_t K, tb_grid_t grid,
@@ -169,12 +179,15 @@ TB_API size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K); /* tb_gemv: M
  *   packed, scales  as produced by tb_pack.
  *   x               [K] bf16, device, 16-byte aligned; finite, |x| < 2^120.
  *   y               [N] fp32 or bf16 (y_dtype), device, written.
- *   workspace       tb_workspace_bytes(1, N, K) bytes (see above). */
+ *   workspace       tb_workspace_bytes(1, N, K) bytes (see above).
+ * TB_GRID_TERNARY_B3 runs its own kernel, which stages x in shared memory
+ * and uses no workspace: K <= 57600, else TB_ERR_UNSUPPORTED. */
 TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *x, void *y,
                            tb_dtype_t y_dtype, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
                            tb_stream_t stream);
 
-/* Small-batch GEMM Y = X W^T, 1 <= M <= 64.
+/* Small-batch GEMM Y = X W^T, 1 <= M <= 64 (TB_GRID_TERNARY_B3: one GEMV
+ * launch per batch row, K <= 57600).
  *   X          [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device; finite, |x| < 2^120.
  *              From M = 32 the activations of one 128-group share one
  *              power-of-two exponent over all M rows: an element more than
@@ -226,6 +239,9 @@ TB_API size_t tb_layer_workspace_bytes(const tb_linear_t *items, int n_items);
  *   n_items    1 .. TB_MAX_LAYER_ITEMS.
  *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS.
  *   workspace  tb_layer_workspace_bytes(items, n_items) bytes.
+ * Items in TB_GRID_TERNARY_B3 are not part of the grouped launch: each runs
+ * its own GEMV launch after it, in the same stream (K <= 57600), and needs
+ * no workspace.
  * Outputs of different items must not overlap. */
 TB_API tb_status_t tb_layer_gemv(const tb_linear_t *items, int n_items, unsigned flags, void *workspace,
                                  size_t workspace_bytes, tb_stream_t stream);

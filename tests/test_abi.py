@@ -143,6 +143,31 @@ def test_argument_errors_before_launch(lib):
     assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0, A, W, 0) == 2
 
 
+def test_b3_sizes_and_limits(lib, oracle):
+    """The 5-trits-per-byte layout: closed-form row bytes (the oracle's too),
+    the shared-memory bound on K, and no workspace for its layer items."""
+    import math
+    B3 = tb.TERNARY_B3
+    for N, K in ((1, 128), (3, 256), (5, 640), (256, 1024), (2048, 6144), (17408, 5120)):
+        want = N * 16 * math.ceil(26 * (K // 128) / 16)
+        assert tb.packed_bytes(B3, N, K) == want == oracle.packed_bytes(B3, N, K)
+    assert tb.packed_bytes(B3, 4, 100) == 0
+    A, W = FAKE, 1 << 20
+    big = 128 * 451  # 451 groups of activations do not fit in shared memory
+    assert lib.tb_gemv(A, B3, A, A, A, 0, 16, big, A, W, 0) == 4
+    assert lib.tb_gemm(A, B3, A, A, big, A, 0, 16, 3, 16, big, A, W, 0) == 4
+    assert lib.tb_gemv_noalloc(A, B3, A, A, A, 0, 16, big, 0) == 4
+    items = (tb.Linear * 2)()
+    items[0] = tb.Linear(A, A, A, A, 16, big, B3, 0)
+    items[1] = tb.Linear(A, A, A, A, 64, 1024, 1, 0)
+    assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0, A, W, 0) == 4
+    # a layer's 5-trit items add nothing to its workspace
+    one = (tb.Linear * 1)()
+    one[0] = items[1]
+    items[0].K = 1024
+    assert tb.layer_workspace_bytes(items) == tb.layer_workspace_bytes(one) > 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     saved = tb._lib
     tb._lib = None
