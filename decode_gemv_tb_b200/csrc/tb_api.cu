@@ -76,6 +76,15 @@ constexpr int64_t kMaxSKWarps = 8192;
 // batch sizes from which tb_gemm runs on the tcgen05 path
 constexpr int64_t kTCMinM = 32;
 
+// Batch-1 products of at most this many weights run the single-launch row
+// kernel (no preparation kernel, no split-tile combine), as do all products
+// in the 5-trits-per-byte layout; larger ones the stream-K TMA kernel.
+constexpr int64_t kRowWarpMaxWeights = (int64_t)1 << 24;
+
+bool use_rowwarp(int grid, int64_t N, int64_t K) {
+    return is_b3(grid) || (N <= kRowWarpMaxWeights / K && gemv_rowwarp_supported(grid, K));
+}
+
 int device_sms() {
     static int sms[64] = {0};
     int dev = 0;
@@ -334,9 +343,11 @@ tb_status_t tb_gemv(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if ((s = check_out(y, y_dtype)) != TB_OK) return s;
     if (!workspace) return TB_ERR_ARG;
     if (!aligned(x, 16) || !aligned(workspace, 256)) return TB_ERR_ALIGN;
-    if (is_b3(grid)) {
-        if (!gemv_b3_supported(K)) return TB_ERR_UNSUPPORTED;
-        return cuda_status(launch_gemv_b3(packed, scales, x, y, y_dtype, N, K, static_cast<cudaStream_t>(stream)));
+    if (workspace_bytes < tb_workspace_bytes(1, N, K)) return TB_ERR_ARG;  // the contract, whichever kernel runs
+    if (use_rowwarp(grid, N, K)) {
+        if (!gemv_rowwarp_supported(grid, K)) return TB_ERR_UNSUPPORTED;  // 5-trit layout only
+        return cuda_status(
+            launch_gemv_rowwarp(packed, grid, scales, x, y, y_dtype, N, K, static_cast<cudaStream_t>(stream)));
     }
     Item it = make_item(packed, grid, scales, x, K, y, y_dtype, N, 1, N, K);
     return launch_tma_items(&it, 1, workspace, workspace_bytes, false, static_cast<cudaStream_t>(stream));
@@ -352,13 +363,15 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if (M < 1 || M > 64 || ldx < K || ldy < N) return TB_ERR_SHAPE;
     if (!workspace) return TB_ERR_ARG;
     if (!aligned(X, 16) || ldx % 8 != 0 || !aligned(workspace, 256)) return TB_ERR_ALIGN;
+    if (workspace_bytes < tb_workspace_bytes(M, N, K)) return TB_ERR_ARG;  // the contract, whichever kernel runs
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (is_b3(grid)) {  // one GEMV launch per batch row
-        if (!gemv_b3_supported(K)) return TB_ERR_UNSUPPORTED;
+    // the row kernel: the 5-trit layout (one launch per batch row) and small batch-1 products
+    if (is_b3(grid) || (M == 1 && use_rowwarp(grid, N, K))) {
+        if (!gemv_rowwarp_supported(grid, K)) return TB_ERR_UNSUPPORTED;
         const size_t ysz = y_dtype == TB_F32 ? 4 : 2;
         for (int64_t m = 0; m < M; ++m) {
-            const cudaError_t e = launch_gemv_b3(packed, scales, X + m * ldx, static_cast<char*>(Y) + m * ldy * ysz,
-                                                 y_dtype, N, K, st);
+            const cudaError_t e = launch_gemv_rowwarp(packed, grid, scales, X + m * ldx,
+                                                      static_cast<char*>(Y) + m * ldy * ysz, y_dtype, N, K, st);
             if (e != cudaSuccess) return TB_ERR_CUDA;
         }
         return TB_OK;
@@ -400,7 +413,7 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
         if ((s = check_out(l.y, l.y_dtype)) != TB_OK) return s;
         if (!aligned(l.x, 16)) return TB_ERR_ALIGN;
         if (is_b3(l.grid)) {
-            if (!gemv_b3_supported(l.K)) return TB_ERR_UNSUPPORTED;
+            if (!gemv_rowwarp_supported(l.grid, l.K)) return TB_ERR_UNSUPPORTED;
             continue;
         }
         its[n_main++] = make_item(l.packed, l.grid, l.scales, l.x, l.K, l.y, l.y_dtype, l.N, 1, l.N, l.K);
@@ -415,7 +428,8 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
     for (int i = 0; i < n_items; ++i) {
         const tb_linear_t& l = items[i];
         if (!is_b3(l.grid)) continue;
-        if (launch_gemv_b3(l.packed, l.scales, l.x, l.y, l.y_dtype, l.N, l.K, st) != cudaSuccess) return TB_ERR_CUDA;
+        if (launch_gemv_rowwarp(l.packed, l.grid, l.scales, l.x, l.y, l.y_dtype, l.N, l.K, st) != cudaSuccess)
+            return TB_ERR_CUDA;
     }
     return TB_OK;
 }
@@ -468,9 +482,10 @@ tb_status_t tb_gemv_noalloc(const void* packed, tb_grid_t grid, const uint16_t* 
     if (!x) return TB_ERR_ARG;
     if ((s = check_out(y, y_dtype)) != TB_OK) return s;
     if (!aligned(x, 16)) return TB_ERR_ALIGN;
-    if (is_b3(grid)) {  // needs no scratch
-        if (!gemv_b3_supported(K)) return TB_ERR_UNSUPPORTED;
-        return cuda_status(launch_gemv_b3(packed, scales, x, y, y_dtype, N, K, static_cast<cudaStream_t>(stream)));
+    if (use_rowwarp(grid, N, K)) {  // needs no scratch
+        if (!gemv_rowwarp_supported(grid, K)) return TB_ERR_UNSUPPORTED;
+        return cuda_status(
+            launch_gemv_rowwarp(packed, grid, scales, x, y, y_dtype, N, K, static_cast<cudaStream_t>(stream)));
     }
     // the size rule is checked before any CUDA call
     if (tb_workspace_bytes(1, N, K) > (size_t)TB_NOALLOC_SCRATCH_BYTES) return TB_ERR_UNSUPPORTED;

@@ -42,12 +42,13 @@ int gemv_tma_resident_warps();
 // bounded waits of k_gemv_tma that gave up since the last call (clears)
 unsigned int take_gemv_timeouts();
 
-// Batch-1 GEMV over the 5-trits-per-byte layout: one launch, no workspace.
-// The activations are staged in shared memory, which bounds K
-// (gemv_b3_supported).
-bool gemv_b3_supported(int64_t K);
-cudaError_t launch_gemv_b3(const void* packed, const uint16_t* scales, const uint16_t* x, void* y, int ydt,
-                           int64_t N, int64_t K, cudaStream_t st);
+// Batch-1 GEMV in one launch, one warp per output row, no workspace: the
+// 5-trits-per-byte layout, and small problems in the other layouts.  The
+// activations are staged in shared memory, which bounds K
+// (gemv_rowwarp_supported).
+bool gemv_rowwarp_supported(int grid, int64_t K);
+cudaError_t launch_gemv_rowwarp(const void* packed, int grid, const uint16_t* scales, const uint16_t* x, void* y,
+                                int ydt, int64_t N, int64_t K, cudaStream_t st);
 
 // Small-batch GEMM on the tcgen05 tensor cores (2 <= M <= 64): preparation
 // kernel + main kernel.  Workspace: gemm_tc_workspace_bytes(M, N, K) bytes,

@@ -179,15 +179,21 @@ TB_API size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K); /* tb_gemv: M
  *   packed, scales  as produced by tb_pack.
  *   x               [K] bf16, device, 16-byte aligned; finite, |x| < 2^120.
  *   y               [N] fp32 or bf16 (y_dtype), device, written.
- *   workspace       tb_workspace_bytes(1, N, K) bytes (see above).
- * TB_GRID_TERNARY_B3 runs its own kernel, which stages x in shared memory
- * and uses no workspace: K <= 57600, else TB_ERR_UNSUPPORTED. */
+ *   workspace       tb_workspace_bytes(1, N, K) bytes (see above), whichever
+ *                   kernel runs.
+ * Two kernels serve it.  Products of at most 2^24 weights (N * K), and every
+ * TB_GRID_TERNARY_B3 product, run a single-launch kernel with one warp per
+ * output row that stages x in shared memory and uses no workspace (for
+ * TB_GRID_TERNARY_B3, K <= 57600, else TB_ERR_UNSUPPORTED).  Larger ones
+ * run the stream-K kernel of tb_layer_gemv.  Both meet the error bound
+ * above; the same product through tb_gemv and tb_layer_gemv may differ in
+ * rounding. */
 TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *x, void *y,
                            tb_dtype_t y_dtype, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
                            tb_stream_t stream);
 
-/* Small-batch GEMM Y = X W^T, 1 <= M <= 64 (TB_GRID_TERNARY_B3: one GEMV
- * launch per batch row, K <= 57600).
+/* Small-batch GEMM Y = X W^T, 1 <= M <= 64 (M = 1 as tb_gemv;
+ * TB_GRID_TERNARY_B3: one GEMV launch per batch row, K <= 57600).
  *   X          [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device; finite, |x| < 2^120.
  *              From M = 32 the activations of one 128-group share one
  *              power-of-two exponent over all M rows: an element more than

@@ -128,11 +128,28 @@ def to_dev_bits(a):
     return torch.from_numpy(a.astype(np.uint16).view(np.int16).copy()).to(DEV).view(torch.bfloat16)
 
 
+# Batch-1 products go through two kernels: tb_gemv runs the single-launch row
+# kernel up to 2^24 weights (the stream-K TMA kernel above), tb_layer_gemv
+# always the stream-K kernel.  "layer" runs the same case through a one-item
+# tb_layer_gemv.
+APIS = ("gemv", "layer")
+ROW_PATH_MAX_WEIGHTS = 1 << 24
+
+
+def gemv_via(api, p, grid, s, x, N, K, y):
+    if api == "gemv":
+        tb.tb_gemv(p, grid, s, x, N, K, y=y)
+    else:
+        tb.tb_layer_gemv([(p, grid, s, x, y, N, K)])
+    return y
+
+
 @pytest.mark.parametrize("grid", GRIDS)
 @pytest.mark.parametrize("shape", [(1, 128), (7, 256), (15, 384), (16, 1152), (17, 640), (33, 1024), (100, 2048),
                                    (256, 1024)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
-def test_gemv_parity_small(oracle, grid, shape, out):
+@pytest.mark.parametrize("api", APIS)
+def test_gemv_parity_small(oracle, grid, shape, out, api):
     N, K = shape
     W, x, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=N * 31 + K)
     y64, yabs = oracle.gemv64(p_ref, grid, s_ref, u16(x), N, K)
@@ -141,18 +158,32 @@ def test_gemv_parity_small(oracle, grid, shape, out):
     guard = 64
     ybuf = torch.full((N + guard,), 123.25, dtype=torch.float32 if out == "f32" else torch.bfloat16, device=DEV)
     y = ybuf[:N]
-    tb.tb_gemv(p, grid, s, x.to(DEV), N, K, y=y)
-    assert_within(y, y64, yabs, out, oracle, f"gemv {shape} grid {grid}")
+    gemv_via(api, p, grid, s, x.to(DEV), N, K, y)
+    assert_within(y, y64, yabs, out, oracle, f"{api} {shape} grid {grid}")
     assert torch.all(ybuf[N:] == 123.25), "wrote past the end of y"
 
 
 @pytest.mark.parametrize("case", synth.config2_cases(), ids=lambda m: m.name)
-def test_gemv_config2(oracle, case):
+@pytest.mark.parametrize("api", APIS)
+def test_gemv_config2(oracle, case, api):
     N, K, grid = case.N, case.K, case.grid
     W, x, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=case.seed)
     y64, yabs = oracle.gemv64(p_ref, grid, s_ref, u16(x), N, K)
+    y = gemv_via(api, to_dev_packed(p_ref), grid, to_dev_bits(s_ref), x.to(DEV), N, K,
+                 torch.empty(N, dtype=torch.float32, device=DEV))
+    assert_within(y, y64, yabs, "f32", oracle, f"{case.name} {api}")
+
+
+@pytest.mark.parametrize("grid", GRIDS)
+@pytest.mark.parametrize("N", [ROW_PATH_MAX_WEIGHTS // 4096, ROW_PATH_MAX_WEIGHTS // 4096 + 1])
+def test_gemv_path_boundary(oracle, grid, N):
+    """tb_gemv at exactly 2^24 weights (row kernel) and one row more
+    (stream-K kernel)."""
+    K = 4096
+    W, x, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=3000 + N + grid)
+    y64, yabs = oracle.gemv64(p_ref, grid, s_ref, u16(x), N, K)
     y = tb.tb_gemv(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), x.to(DEV), N, K)
-    assert_within(y, y64, yabs, "f32", oracle, case.name)
+    assert_within(y, y64, yabs, "f32", oracle, f"boundary {N}x{K} grid {grid}")
 
 
 def test_gemv_config1(oracle):
@@ -169,7 +200,8 @@ def test_gemv_config1(oracle):
 
 
 @pytest.mark.parametrize("grid", GRIDS)
-def test_gemv_integer_exact_bitwise(oracle, grid):
+@pytest.mark.parametrize("api", APIS)
+def test_gemv_integer_exact_bitwise(oracle, grid, api):
     """Integer x and power-of-two scales: every partial sum is exact, so the
     GPU result equals the oracle's bit for bit."""
     lo, hi = oracle.GRID_RANGE[grid]
@@ -181,7 +213,8 @@ def test_gemv_integer_exact_bitwise(oracle, grid):
     W = c.float() * 2.0 ** -5
     p_ref, _ = oracle.pack(W.numpy(), grid, u16(s))
     y64, _ = oracle.gemv64(p_ref, grid, u16(s), u16(x), N, K)
-    y = tb.tb_gemv(to_dev_packed(p_ref), grid, s.to(DEV), x.to(DEV), N, K)
+    y = gemv_via(api, to_dev_packed(p_ref), grid, s.to(DEV), x.to(DEV), N, K,
+                 torch.empty(N, dtype=torch.float32, device=DEV))
     assert np.array_equal(y.cpu().numpy(), y64.astype(np.float32))
 
 
@@ -191,9 +224,10 @@ def test_gemv_deterministic():
     x = synth.activations(K, seed=5, device=DEV)
     for grid in GRIDS:
         s, p, _ = gpu_quantize(W, grid)
-        y1 = tb.tb_gemv(p, grid, s, x, N, K)
-        y2 = tb.tb_gemv(p, grid, s, x, N, K)
-        assert torch.equal(y1, y2)
+        for api in APIS:
+            y1 = gemv_via(api, p, grid, s, x, N, K, torch.empty(N, dtype=torch.float32, device=DEV))
+            y2 = gemv_via(api, p, grid, s, x, N, K, torch.empty(N, dtype=torch.float32, device=DEV))
+            assert torch.equal(y1, y2)
 
 
 # ------------------------------------------------------------------ grouped layer
@@ -338,13 +372,15 @@ def _x_case(kind, K, seed):
 
 @pytest.mark.parametrize("grid", GRIDS)
 @pytest.mark.parametrize("kind", ["wide_range", "zero_groups", "subnormal", "large", "one_hot"])
-def test_gemv_activation_ranges(oracle, grid, kind):
+@pytest.mark.parametrize("api", APIS)
+def test_gemv_activation_ranges(oracle, grid, kind, api):
     N, K = 96, 1024
     W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=1200 + grid)
     x = _x_case(kind, K, 77)
     y64, yabs = oracle.gemv64(p_ref, grid, s_ref, u16(x), N, K)
-    y = tb.tb_gemv(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), x.to(DEV), N, K)
-    assert_within(y, y64, yabs, "f32", oracle, kind)
+    y = gemv_via(api, to_dev_packed(p_ref), grid, to_dev_bits(s_ref), x.to(DEV), N, K,
+                 torch.empty(N, dtype=torch.float32, device=DEV))
+    assert_within(y, y64, yabs, "f32", oracle, f"{kind} {api}")
 
 
 def test_layer_overlap_flag_and_shared_workspace(oracle):
