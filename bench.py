@@ -95,15 +95,16 @@ class Clocks:
 
     NAMES = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
-    def __init__(self, gpu: int):
+    def __init__(self, gpu: int, log_path: str | None = None):
+        import tempfile
         self.gpu = gpu
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu}.csv")
+        self.path = log_path or os.path.join(tempfile.gettempdir(), f"tb_bench_clocks_gpu{gpu}.csv")
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.nvml, self.thread, self.active = None, None, False
 
     def __enter__(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        os.makedirs(os.path.dirname(os.path.abspath(self.path)), exist_ok=True)
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -530,6 +531,8 @@ def main():
     ap.add_argument("--layers", type=int, default=None, help="fewer layers (debug only)")
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--clocks-log", default=None,
+                    help="nvidia-smi clock log (CSV) of the run; default: a file in the temp directory")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
@@ -560,7 +563,7 @@ def main():
     # --- device-resident timing (the headline `value`): graph of one step,
     # every layer called with the default flags
     g_step = capture(lambda: S.step(0))
-    with Clocks(local) as clk:
+    with Clocks(local, args.clocks_log) as clk:
         ms = time_region(g_step.replay, args.steps, args.warmup, cur, dist, clk)
     clocks = clk.summary()
     ms_step = ms / args.steps
