@@ -532,7 +532,8 @@ def main():
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--clocks-log", default=None,
-                    help="nvidia-smi clock log (CSV) of the run; default: a file in the temp directory")
+                    help="nvidia-smi clock log (CSV) of the run (rank r of N > 1 writes PATH.r); "
+                         "default: a file in the temp directory")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
@@ -563,7 +564,8 @@ def main():
     # --- device-resident timing (the headline `value`): graph of one step,
     # every layer called with the default flags
     g_step = capture(lambda: S.step(0))
-    with Clocks(local, args.clocks_log) as clk:
+    log = args.clocks_log if (args.clocks_log is None or world == 1) else f"{args.clocks_log}.{rank}"
+    with Clocks(local, log) as clk:
         ms = time_region(g_step.replay, args.steps, args.warmup, cur, dist, clk)
     clocks = clk.summary()
     ms_step = ms / args.steps
