@@ -157,7 +157,8 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
 
 /* Scratch ("workspace") of the products below.  Each call first writes a
  * prepared copy of its activations (bf16, K per activation row, scaled by
- * powers of two) and per-128-group sums into the workspace, then reads them;
+ * powers of two) and per-128-group sums into the workspace, then reads them
+ * (the single-launch row kernel behind small tb_gemv calls uses none of it);
  * the calls also keep per-tile arrival counters and partial sums there
  * (tiles whose K range is split are combined in a fixed order).  For M = 1
  * the size is ceil256(K/128 * 272) + ceil256(4 * ceil(N/32))
