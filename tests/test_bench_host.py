@@ -1,0 +1,63 @@
+"""bench.py's host-side arithmetic (no GPU): the algorithmic bytes of a
+product in every layout, the rule that drops the committed DRAM-traffic
+figure once the kernel's sources change, and the `config` object both arms
+print."""
+import json
+import os
+import shutil
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    import bench as b
+    return b
+
+
+def test_algo_bytes_every_layout(bench, oracle):
+    from decode_gemv_tb_b200 import tb
+    for N, K in ((256, 1024), (2048, 6144), (17408, 5120), (3, 640)):
+        for grid in (tb.TERNARY, tb.INT2, tb.INT3, tb.TERNARY_B3):
+            # packed codes as the oracle lays them out, bf16 scales, bf16 x, fp32 y
+            want = oracle.packed_bytes(grid, N, K) + 2 * N * (K // 128) + 2 * K + 4 * N
+            assert bench.algo_bytes(N, K, grid) == want, (grid, N, K)
+        # batch M: M rows of x and of y
+        assert bench.algo_bytes(N, K, tb.INT2, M=8) == oracle.packed_bytes(1, N, K) + 2 * N * (K // 128) \
+            + 8 * 2 * K + 8 * 4 * N
+
+
+def test_traffic_figure_tracks_the_kernel_sources(bench, tmp_path, monkeypatch):
+    """The committed ratio is used while the hashed sources are unchanged,
+    and dropped (None) as soon as one of them differs."""
+    rec = json.load(open(os.path.join(ROOT, "profiles", "k_gemv_tma_traffic.json")))
+    assert bench.traffic_per_launch(1000.0) == pytest.approx(1000.0 * rec["traffic_over_algorithmic"])
+    # a copy of the tree's relevant files, one source changed by a byte
+    fake = tmp_path / "root"
+    (fake / "profiles").mkdir(parents=True)
+    shutil.copy(os.path.join(ROOT, "profiles", "k_gemv_tma_traffic.json"), fake / "profiles")
+    for s in rec["kernel_sources"]:
+        dst = fake / s
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        shutil.copy(os.path.join(ROOT, s), dst)
+    monkeypatch.setattr(bench, "ROOT", str(fake))
+    assert bench.traffic_per_launch(1000.0) == pytest.approx(1000.0 * rec["traffic_over_algorithmic"])
+    with open(fake / rec["kernel_sources"][0], "a") as f:
+        f.write("\n")
+    assert bench.traffic_per_launch(1000.0) is None
+
+
+def test_workload_config_names_the_stack(bench):
+    from decode_gemv_tb_b200 import synth
+    stack = synth.config3_stack()
+    cfg = bench.workload_config(stack, 1)
+    assert cfg["batch"] == 1 and cfg["layers"] == 36 and cfg["hidden"] == 4096 and cfg["mlp"] == 12288
+    assert cfg["parallelism"] == "replicas1"
+    mix = cfg["grid_mix"]
+    assert abs(sum(mix.values()) - 1.0) < 1e-3
+    # 2.01 GB of algorithmic bytes per step (codes, scales, x and y of all 252 products)
+    step = sum(bench.algo_bytes(m.N, m.K, m.grid) for mats in stack for m in mats)
+    assert cfg["step_algorithmic_bytes"] == step
+    assert 2.0e9 < step < 2.02e9
