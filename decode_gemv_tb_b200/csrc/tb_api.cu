@@ -81,6 +81,12 @@ constexpr int64_t kTCMinM = 32;
 // in the 5-trits-per-byte layout; larger ones the stream-K TMA kernel.
 constexpr int64_t kRowWarpMaxWeights = (int64_t)1 << 24;
 
+// Batches above 64 rows (prefill) run as consecutive blocks of 64 rows, the
+// last block the remainder, each through the dispatch for its size, in
+// stream order and sharing the workspace.
+constexpr int64_t kGemmBlockM = 64;
+constexpr int64_t kMaxGemmM = (int64_t)1 << 16;
+
 bool use_rowwarp(int grid, int64_t N, int64_t K) {
     return is_b3(grid) || (N <= kRowWarpMaxWeights / K && gemv_rowwarp_supported(grid, K));
 }
@@ -263,7 +269,7 @@ const char* tb_status_string(tb_status_t s) {
     switch (s) {
         case TB_OK: return "ok";
         case TB_ERR_ARG: return "invalid argument (null pointer, unknown enum value or bad count)";
-        case TB_ERR_SHAPE: return "invalid shape (N >= 1, K a positive multiple of 128, 1 <= M <= 64, ld >= extent)";
+        case TB_ERR_SHAPE: return "invalid shape (N >= 1, K a positive multiple of 128, 1 <= M <= 65536, ld >= extent)";
         case TB_ERR_ALIGN: return "misaligned pointer or leading dimension";
         case TB_ERR_UNSUPPORTED: return "unsupported request";
         case TB_ERR_CUDA: return "CUDA error";
@@ -310,7 +316,11 @@ tb_status_t tb_unpack(const void* packed, tb_grid_t grid, int64_t N, int64_t K, 
 }
 
 size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    if (M < 1 || M > 64 || !shape_ok(N, K)) return 0;
+    if (M < 1 || M > kMaxGemmM || !shape_ok(N, K)) return 0;
+    if (M > kGemmBlockM) {  // the largest of its blocks' sizes
+        const int64_t rem = M % kGemmBlockM;
+        return std::max(tb_workspace_bytes(kGemmBlockM, N, K), rem ? tb_workspace_bytes(rem, N, K) : (size_t)0);
+    }
     if (M == 1) {  // chunk count bounded with the smaller chunk (two groups)
         const int64_t tiles = (N + 31) / 32;
         return tm_item_workspace(K) + tm_extra_workspace(tiles, tiles * ((K / kGroup + 1) / 2));
@@ -360,10 +370,21 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if (s != TB_OK) return s;
     if (!X) return TB_ERR_ARG;
     if ((s = check_out(Y, y_dtype)) != TB_OK) return s;
-    if (M < 1 || M > 64 || ldx < K || ldy < N) return TB_ERR_SHAPE;
+    if (M < 1 || M > kMaxGemmM || ldx < K || ldy < N) return TB_ERR_SHAPE;
     if (!workspace) return TB_ERR_ARG;
     if (!aligned(X, 16) || ldx % 8 != 0 || !aligned(workspace, 256)) return TB_ERR_ALIGN;
     if (workspace_bytes < tb_workspace_bytes(M, N, K)) return TB_ERR_ARG;  // the contract, whichever kernel runs
+    if (M > kGemmBlockM) {
+        const size_t ysz = y_dtype == TB_F32 ? 4 : 2;
+        for (int64_t m0 = 0; m0 < M; m0 += kGemmBlockM) {
+            const int64_t mb = std::min(kGemmBlockM, M - m0);
+            const tb_status_t s2 = tb_gemm(packed, grid, scales, X + m0 * ldx, ldx,
+                                           static_cast<char*>(Y) + m0 * ldy * ysz, y_dtype, ldy, mb, N, K, workspace,
+                                           workspace_bytes, stream);
+            if (s2 != TB_OK) return s2;
+        }
+        return TB_OK;
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // the row kernel: the 5-trit layout (one launch per batch row) and small batch-1 products
     if (is_b3(grid) || (M == 1 && use_rowwarp(grid, N, K))) {

@@ -1,7 +1,8 @@
 /*
  * tb.h -- C interface of libtb_b200: ThinkBit scalar low-bit weights on
  * NVIDIA B200 (sm_100a).  Quantize/pack, unpack, batch-1 GEMV, small-batch
- * GEMM (M <= 64) and a grouped launcher for a decoder layer's projections.
+ * GEMM (M <= 64, and prefill batches in blocks of 64) and a grouped
+ * launcher for a decoder layer's projections.
  *
  * What the method fixes -- ThinkBit page, "ThinkBit은 2비트 양자화에서 추론
  * 능력 보존을 추론 평가로 검증한다" (onedev.kr/papers/1416):
@@ -112,7 +113,7 @@ typedef enum { TB_F32 = 0, TB_BF16 = 1 } tb_dtype_t;
 typedef enum {
     TB_OK = 0,
     TB_ERR_ARG = 1,         /* null pointer, unknown enum value, bad count */
-    TB_ERR_SHAPE = 2,       /* N < 1, K < 128, K % 128 != 0, M outside 1..64, ld too small */
+    TB_ERR_SHAPE = 2,       /* N < 1, K < 128, K % 128 != 0, M outside 1..65536, ld too small */
     TB_ERR_ALIGN = 3,       /* a pointer or leading dimension breaks the alignment rules */
     TB_ERR_UNSUPPORTED = 4, /* valid request this build does not implement */
     TB_ERR_CUDA = 5         /* a CUDA call or launch failed */
@@ -167,7 +168,8 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
  *   ceil256(K/128 * (NP * 288 + 16)) + ceil256(T * K/128 * 256) + ceil256(4 * T)
  *     + [S > 1] ceil256(T * S * NP * 512)
  * with NP = M rounded up to 16, T = ceil(N / 128) and S = the K split,
- * max(1, min(floor((296 + T/2) / T), 16, K / 128)).
+ * max(1, min(floor((296 + T/2) / T), 16, K / 128)).  For M > 64 it is the
+ * larger of the sizes for 64 and for M mod 64 (when not 0).
  *   - device memory, 256-byte aligned, at least the size returned here;
  *   - owned by the caller, written by every call: two calls that share a
  *     workspace must be ordered (e.g. the same stream);
@@ -195,6 +197,9 @@ TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *s
 
 /* Small-batch GEMM Y = X W^T, 1 <= M <= 64 (M = 1 as tb_gemv;
  * TB_GRID_TERNARY_B3: one GEMV launch per batch row, K <= 57600).
+ * Prefill batches, 64 < M <= 65536, run as consecutive blocks of 64 batch
+ * rows (the last one the remainder), each like a call with that M, in
+ * stream order: the weights are decoded once per block.
  *   X          [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device; finite, |x| < 2^120.
  *              From M = 32 the activations of one 128-group share one
  *              power-of-two exponent over all M rows: an element more than

@@ -87,7 +87,7 @@ def test_workspace_sizes(lib):
         warps = min(8192, tiles * ((K // 128 + 1) // 2))
         assert tb.workspace_bytes(1, N, K) == al(272 * (K // 128)) + al(4 * tiles) + al(256 * warps)
     assert tb.workspace_bytes(0, 8, 128) == 0 and tb.workspace_bytes(1, 8, 100) == 0
-    assert tb.workspace_bytes(65, 8, 128) == 0 and tb.workspace_bytes(1, 0, 128) == 0
+    assert tb.workspace_bytes(65537, 8, 128) == 0 and tb.workspace_bytes(1, 0, 128) == 0
     items = (tb.Linear * 3)()
     shapes = ((4096, 4096, 2), (1024, 4096, 1), (4096, 12288, 0))  # (N, K, grid)
     for i, (N, K, grid) in enumerate(shapes):
@@ -117,7 +117,7 @@ def test_argument_errors_before_launch(lib):
     assert lib.tb_gemv(A, 1, A, A, A, 0, 0, 128, A, W, 0) == 2
     assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 100, A, W, 0) == 2
     assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 0, A, W, 0) == 2
-    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 16, 65, 16, 128, A, W, 0) == 2
+    assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 16, 65537, 16, 128, A, 1 << 30, 0) == 2
     assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 16, 0, 16, 128, A, W, 0) == 2
     assert lib.tb_gemm(A, 1, A, A, 120, A, 0, 16, 4, 16, 128, A, W, 0) == 2
     assert lib.tb_gemm(A, 1, A, A, 128, A, 0, 8, 4, 16, 128, A, W, 0) == 2
@@ -141,6 +141,18 @@ def test_argument_errors_before_launch(lib):
     items[1].x = A
     items[1].K = 130
     assert lib.tb_layer_gemv(ctypes.cast(items, ctypes.c_void_p), 2, 0, A, W, 0) == 2
+
+
+def test_prefill_workspace_is_the_largest_block(lib):
+    """Batches above 64 rows run in blocks of 64: the workspace covers the
+    larger of a 64-row block and the remainder block."""
+    for N, K in ((100, 5120), (17408, 5120), (7, 1024)):
+        w64 = tb.workspace_bytes(64, N, K)
+        assert tb.workspace_bytes(128, N, K) == w64
+        for M in (65, 97, 100, 130, 4096 + 17):
+            rem = M % 64
+            assert tb.workspace_bytes(M, N, K) == max(w64, tb.workspace_bytes(rem, N, K) if rem else 0)
+    assert tb.workspace_bytes(65536, 64, 128) > 0 and tb.workspace_bytes(65537, 64, 128) == 0
 
 
 def test_b3_sizes_and_limits(lib, oracle):

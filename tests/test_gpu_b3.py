@@ -139,6 +139,15 @@ def test_b3_gemm_rows_strided_bf16(oracle):
     assert torch.all(Ybuf[:, N:] == 0)
 
 
+def test_b3_gemm_prefill(oracle):
+    N, K, M = 48, 640, 70
+    W, _, s_ref, p_ref = oracle_problem(oracle, B3, N, K, seed=2150)
+    X = synth.activations(K, seed=2151, M=M)
+    Y64, Yabs = oracle.gemm64(p_ref, B3, s_ref, u16(X), N, K)
+    Y = tb.tb_gemm(to_dev_packed(p_ref), B3, to_dev_bits(s_ref), X.to(DEV), N, K)
+    assert_within(Y, Y64, Yabs, "f32", oracle, "b3 prefill")
+
+
 def test_b3_layer_items_and_noalloc(oracle):
     """5-trit items mixed into a grouped launch with the other grids; the
     no-workspace entry point on the same matrix."""

@@ -305,6 +305,36 @@ def test_gemm_strided_bf16_out(oracle):
 
 
 @pytest.mark.parametrize("grid", GRIDS)
+@pytest.mark.parametrize("M", [65, 100, 128, 161])
+def test_gemm_prefill_blocks(oracle, grid, M):
+    """Batches above 64 rows run as blocks of 64 (remainders of 1, 36 and 33
+    rows take the GEMV, tcgen05 and tcgen05 paths)."""
+    N, K = 80, 768
+    W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=3100 + M)
+    X = synth.activations(K, seed=3200 + M, M=M)
+    Y64, Yabs = oracle.gemm64(p_ref, grid, s_ref, u16(X), N, K)
+    Y = tb.tb_gemm(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), X.to(DEV), N, K)
+    assert_within(Y, Y64, Yabs, "f32", oracle, f"prefill M={M} grid {grid}")
+
+
+def test_gemm_prefill_strided_bf16_out(oracle):
+    N, K, M = 200, 1024, 130
+    W, _, s_ref, p_ref = oracle_problem(oracle, tb.INT3, N, K, seed=3300)
+    Xfull = synth.activations(K + 64, seed=3301, M=M)
+    X = Xfull[:, :K]
+    Y64, Yabs = oracle.gemm64(p_ref, tb.INT3, s_ref, u16(X.contiguous()), N, K)
+    Ybuf = torch.zeros((M, N + 24), dtype=torch.bfloat16, device=DEV)
+    pd, sd, xd = to_dev_packed(p_ref), to_dev_bits(s_ref), Xfull.to(DEV)
+    ws = tb.workspace(tb.workspace_bytes(M, N, K), DEV)
+    rc = tb.load().tb_gemm(pd.data_ptr(), tb.INT3, sd.data_ptr(), xd.data_ptr(), K + 64, Ybuf.data_ptr(), tb.BF16,
+                           N + 24, M, N, K, ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert_within(Ybuf[:, :N], Y64, Yabs, "bf16", oracle, "prefill strided")
+    assert torch.all(Ybuf[:, N:] == 0)
+
+
+@pytest.mark.parametrize("grid", GRIDS)
 @pytest.mark.parametrize("M", [16, 33, 64])
 def test_gemm_multi_tile_split(oracle, grid, M):
     """Several 128-row tiles, a ragged last tile and a 16-way K split."""
