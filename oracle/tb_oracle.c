@@ -64,6 +64,9 @@
  *  R7  W is [N out][K in] row-major, y = W x, no bias.
  *  R8  products are summed in k order in fp64; fp32 output is the RNE
  *      rounding of that sum; bf16 output is the RNE rounding of the fp32.
+ *  R9  the down projection's input is silu(gate) * up of the layer's gate
+ *      and up projections (the Qwen3 MLP; the pages name the model family,
+ *      not its layer), computed from the exact projections in fp64.
  *
  * Why the fp64 quotient gives the exact round-half-even of w/s (R2):
  * write w = W 2^a, s = S 2^b with integers |W|, S < 2^24.  If q = w/s is
@@ -324,6 +327,22 @@ int tbo_gemv_rows(const uint32_t *packed, int grid, const uint16_t *scales, cons
     int64_t G = K / TBO_GROUP, RW = tbo_row_words(grid, K);
     for (int64_t i = 0; i < nrows; ++i)
         dot_row(packed + rows[i] * RW, grid, scales + rows[i] * G, x, K, y + i, yabs + i);
+    return 0;
+}
+
+/* ---- the step between a decoder layer's gate/up and down projections ------
+ * [TB-what] (section 무엇인가): decode runs every projection of every layer
+ * for each token; in the Qwen3 layers the pages quantize, the down
+ * projection's input is the SiLU-gated product of the gate and up
+ * projections of the same input (reading R9):
+ *     h[n] = silu(g[n]) * u[n],   silu(g) = g / (1 + e^-g).
+ * Plain fp64 with libm's exp. */
+double tbo_silu(double g) { return g / (1.0 + exp(-g)); }
+
+int tbo_swiglu(const double *g, const double *u, int64_t n, double *h)
+{
+    if (n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) h[i] = tbo_silu(g[i]) * u[i];
     return 0;
 }
 

@@ -69,6 +69,10 @@ def lib():
         L.tbo_gemv.argtypes = [P, ctypes.c_int, P, P, I64, I64, P, P]
         L.tbo_gemm.argtypes = [P, ctypes.c_int, P, P, I64, I64, I64, I64, P, P]
         L.tbo_gemv_rows.argtypes = [P, ctypes.c_int, P, P, I64, P, I64, P, P]
+        L.tbo_silu.argtypes = [ctypes.c_double]
+        L.tbo_silu.restype = ctypes.c_double
+        L.tbo_swiglu.argtypes = [P, P, I64, P]
+        L.tbo_swiglu.restype = ctypes.c_int
         L.tbo_row_words.argtypes = [ctypes.c_int, I64]
         L.tbo_row_words.restype = I64
         for f in ("tbo_scales_absmax", "tbo_pack", "tbo_unpack", "tbo_gemv", "tbo_gemm", "tbo_gemv_rows"):
@@ -191,6 +195,21 @@ def gemm64(packed, grid, scales, X_bits, N, K):
     Yabs = np.empty((M, N), dtype=np.float64)
     _check(lib().tbo_gemm(_ptr(packed), grid, _ptr(scales), _ptr(X_bits), K, M, N, K, _ptr(Y), _ptr(Yabs)), "gemm")
     return Y, Yabs
+
+
+def silu(g: float) -> float:
+    """silu(g) = g / (1 + e^-g) in fp64 (reading R9)."""
+    return float(lib().tbo_silu(float(g)))
+
+
+def swiglu64(g64: np.ndarray, u64: np.ndarray) -> np.ndarray:
+    """h = silu(g) * u elementwise in fp64 (the down projection's input)."""
+    g64 = np.ascontiguousarray(g64, dtype=np.float64)
+    u64 = np.ascontiguousarray(u64, dtype=np.float64)
+    assert g64.shape == u64.shape
+    h = np.empty_like(g64)
+    _check(lib().tbo_swiglu(_ptr(g64), _ptr(u64), g64.size, _ptr(h)), "swiglu")
+    return h
 
 
 def round_out(y64: np.ndarray, out_dtype: str) -> np.ndarray:

@@ -376,6 +376,29 @@ def test_scales_absmax_against_torch(oracle, grid):
     assert np.array_equal(got_b, ref_b)
 
 
+def test_scale_rule_edges_golden(oracle):
+    """The non-finite and overflow branches of the scale rule against
+    hand-worked values (tests/golden/scale_examples.txt): NaN and +-Inf
+    entries are skipped, a zero scale becomes 1.0, one that rounds to
+    infinity becomes the largest finite bf16."""
+    names = {"ternary": 0, "int2": 1, "int3": 2}
+    n = 0
+    for line in open(os.path.join(GOLDEN, "scale_examples.txt")):
+        if not line.strip() or line.startswith("#"):
+            continue
+        grid_s, entries, want, _ = [f.strip() for f in line.split(";", 3)]
+        group = np.zeros(128, dtype=np.float32)
+        i = 0
+        for e in entries.split(","):
+            v, cnt = e.strip().split(" x")
+            group[i:i + int(cnt)] = np.float32(float(v))
+            i += int(cnt)
+        got = oracle.scales_absmax(group.reshape(1, 128), names[grid_s])
+        assert int(got[0, 0]) == int(want, 16), line
+        n += 1
+    assert n == 13
+
+
 def test_scales_reach_grid_ends(oracle):
     """With absmax/|qmin| scales, the group's most negative entry lands on
     qmin exactly (it is -|qmin| * s before rounding)."""
@@ -522,3 +545,35 @@ def test_workload_mix_matches_page():
     # Config 5 packed size: 3.82 GB scale (2.125 / 3.125 bits per weight with scales)
     tot = sum(m.N * m.K * (3.125 if m.grid == 2 else 2.125) / 8 for mats in synth.config5_stack() for m in mats)
     assert 3.75e9 < tot < 3.9e9
+
+
+# ---------------------------------------------------------------- gated MLP input (reading R9)
+
+def test_silu_against_high_precision(oracle):
+    """silu(g) = g / (1 + e^-g) in fp64 against a 60-digit decimal
+    evaluation (correctly rounded exp at that precision, independent of the
+    C library): within 4 ulps, and the special values exactly."""
+    import decimal
+    ctx = decimal.Context(prec=60)
+    pts = [-100.0, -30.0, -20.0, -5.0, -1.0, -0.25, -2.0 ** -20, 0.0, 2.0 ** -20, 0.5, 1.0, 2.0, 7.25, 30.0, 100.0]
+    for g in pts:
+        D = decimal.Decimal(g)
+        ref = float(ctx.divide(D, ctx.add(decimal.Decimal(1), ctx.exp(-D))))
+        got = oracle.silu(g)
+        assert abs(got - ref) <= 4 * np.spacing(abs(ref)) + 1e-300, (g, got, ref)
+    assert oracle.silu(0.0) == 0.0
+    assert oracle.silu(800.0) == 800.0          # e^-800 underflows: g / 1
+    assert oracle.silu(-800.0) == 0.0           # e^800 overflows: g / inf -> -0
+    # the function's shape: silu(g) - silu(-g) = g (since e^-g / (1 + e^-g) + 1 / (1 + e^-g) = 1)
+    for g in (0.3, 1.7, 4.0):
+        assert abs((oracle.silu(g) - oracle.silu(-g)) - g) <= 4 * np.spacing(g)
+
+
+def test_swiglu_is_silu_times_up(oracle):
+    rng = np.random.default_rng(31)
+    g = rng.standard_normal(257) * 3
+    u = rng.standard_normal(257)
+    h = oracle.swiglu64(g, u)
+    assert np.array_equal(h, np.array([oracle.silu(a) * b for a, b in zip(g, u)]))
+    assert np.array_equal(oracle.swiglu64(g, 2 * u), 2 * h)   # exact scaling
+    assert np.all(oracle.swiglu64(g, np.zeros_like(u)) == 0)
