@@ -24,14 +24,13 @@ bool shape_ok(int64_t N, int64_t K) { return N >= 1 && K >= kGroup && K % kGroup
 
 tb_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? TB_OK : TB_ERR_CUDA; }
 
-// packed rows are read 8 bytes (2-bit) or 4 bytes (3-bit) at a time at
-// offsets that are multiples of those sizes; the base must be 16-byte
-// aligned (also required for TMA-style bulk copies).
+// Packed rows and scales are read by tensor and bulk copies: both bases must
+// be 16-byte aligned.
 tb_status_t check_weights(const void* packed, int grid, const uint16_t* scales, int64_t N, int64_t K) {
     if (!packed || !scales) return TB_ERR_ARG;
     if (!grid_ok(grid)) return TB_ERR_ARG;
     if (!shape_ok(N, K)) return TB_ERR_SHAPE;
-    if (!aligned(packed, 16) || !aligned(scales, 2)) return TB_ERR_ALIGN;
+    if (!aligned(packed, 16) || !aligned(scales, 16)) return TB_ERR_ALIGN;
     return TB_OK;
 }
 
@@ -62,16 +61,9 @@ Item make_item(const void* packed, int grid, const uint16_t* scales, const uint1
 
 inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
-// Workspace of one item: prepared activations [M][K] bf16, then per-group
-// (offset * sum x, 2^S) pairs [K/128][M].
-size_t item_workspace(int64_t M, int64_t K) {
-    return align256((size_t)(M * K * 2)) + align256((size_t)((K / kGroup) * M * 8));
-}
-
-// Batch-1 launches additionally need one counter per 32-row tile and two
-// 32-float partial-sum slots per warp (at most kMaxSKWarps warps, and never
-// more warps than chunks).
-constexpr int64_t kMaxSKWarps = 8192;
+// The small-batch kernel (2 <= M < 32) reads the activations as they are and
+// needs no workspace; its size is reported as this nominal minimum.
+constexpr size_t kNoWorkspace = 256;
 
 // batch sizes from which tb_gemm runs on the tcgen05 path
 constexpr int64_t kTCMinM = 32;
@@ -104,9 +96,9 @@ int device_sms() {
 }
 
 // Orders items by per-tile cost (descending) so that the expensive tiles
-// are dispatched first, chooses how many warps share a 16-row tile (the
-// K split), lays out the workspace and launches.
-tb_status_t launch_items(Item* items, int n, int nt, void* ws, size_t ws_bytes, bool overlap, cudaStream_t st) {
+// are dispatched first, chooses how many warps share a 32-row tile (the
+// K split) and launches.
+tb_status_t launch_items(Item* items, int n, int nt, cudaStream_t st) {
     Launch L;
     std::memset(&L, 0, sizeof(L));
     int order[kMaxItems];
@@ -142,70 +134,73 @@ tb_status_t launch_items(Item* items, int n, int nt, void* ws, size_t ws_bytes, 
     L.scl_stride = (int32_t)((gpw + 3) / 4 * 4 + 2);  // >= gpw, = 2 mod 4
     if (linear_smem_bytes(nt, L.scl_stride) > 227 * 1024) return TB_ERR_UNSUPPORTED;
 
-    size_t need = 0;
-    int64_t ctas = 0, prep = 0;
-    char* w = static_cast<char*>(ws);
+    int64_t ctas = 0;
     for (int j = 0; j < n; ++j) {
         Item it = items[order[j]];
         it.ksplit = S[order[j]];
         it.cta_begin = (int32_t)ctas;
-        it.prep_begin = (int32_t)prep;
-        it.xs = reinterpret_cast<uint16_t*>(w + need);
-        it.cf = reinterpret_cast<float2*>(w + need + align256((size_t)(it.M * it.K * 2)));
-        need += item_workspace(it.M, it.K);
         const int64_t tiles_per_cta = 8 / it.ksplit;
         ctas += ((it.N + 31) / 32 + tiles_per_cta - 1) / tiles_per_cta;
-        prep += (it.K / kGroup) * it.M;
         L.it[j] = it;
     }
     L.n_items = n;
-    if (!ws || ws_bytes < need) return TB_ERR_ARG;
-    if (ctas > 0x7FFFFFFF || prep > 0x7FFFFFFF) return TB_ERR_SHAPE;
-    return cuda_status(launch_linear(L, nt, (int)ctas, (int)prep, overlap, st));
+    if (ctas > 0x7FFFFFFF) return TB_ERR_SHAPE;
+    return cuda_status(launch_linear(L, nt, (int)ctas, st));
 }
 
-// Batch-1 (M == 1) launch: preparation kernel + k_gemv_tma.  Each item's
-// activations become G records of kRecBytes; 3-bit items form the first
-// partition, 2-bit items the second (each warp works on one code width
-// only); warps are split between them by cost.  Chunks are C = 2 (3-bit) or
-// 4 (2-bit) groups of one 32-row tile.
-int tm_chunk_groups(int grid) { return grid == TB_GRID_INT3 ? 2 : 4; }
-size_t tm_item_workspace(int64_t K) { return align256((size_t)(K / kGroup) * kRecBytes); }
-size_t tm_extra_workspace(int64_t tiles, int64_t chunks) {
-    const int64_t w = std::min(kMaxSKWarps, std::max<int64_t>(chunks, 1));
-    return align256((size_t)(tiles * 4)) + align256((size_t)(w * 2 * 32 * 4));
+// Batch-1 (M == 1) launch on the integer tensor path: preparation kernel +
+// k_gemv8 (tb_gemv8.cu).  Every item's activations become K/128 records;
+// the items' tiles of 256 rows are cut into chunks of 4 (2-bit container)
+// or 2 (3 bits) groups, numbered item by item, and split into equal-cost
+// contiguous ranges, one per CTA.  Scales are read by tensor copies, which
+// need 16-byte rows: when K/128 is not a multiple of 8 the preparation
+// kernel first copies them with rows padded to a multiple of 8 groups.
+constexpr int64_t kMaxG8Ctas = 256;      // bound of the CTA count (partial-sum slots)
+constexpr int64_t kG8Rows = kG8TileRows;
+constexpr long long kWaitCycles = 4000000000LL;      // about 2 s
+constexpr long long kTestWaitCycles = 20000000LL;    // about 10 ms (TB_FLAG_TEST_STALL)
+
+int64_t g8_padded_groups(int64_t G) { return (G + 7) / 8 * 8; }
+bool g8_needs_spad(int64_t G) { return G % 8 != 0; }
+// workspace of one item: records, then the padded scale copy if needed
+size_t g8_item_workspace(int64_t N, int64_t K) {
+    const int64_t G = K / kGroup;
+    return align256((size_t)G * kG8RecBytes) + (g8_needs_spad(G) ? align256((size_t)(N * g8_padded_groups(G) * 2)) : 0);
+}
+size_t g8_extra_workspace(int64_t tiles, int64_t chunks) {
+    const int64_t c = std::min(kMaxG8Ctas, std::max<int64_t>(chunks, 1));
+    return align256((size_t)(tiles * 8 * 4)) + align256((size_t)(c * 2 * kG8Rows * 4));
+}
+int64_t g8_tiles(int64_t N) { return (N + kG8Rows - 1) / kG8Rows; }
+int64_t g8_chunks(int grid, int64_t N, int64_t K) {
+    const int64_t C = g8_chunk_groups(grid);
+    return g8_tiles(N) * ((K / kGroup + C - 1) / C);
 }
 
-tb_status_t launch_tma_items(const Item* items, int n, void* ws, size_t ws_bytes, bool overlap, cudaStream_t st) {
-    Launch P;
-    std::memset(&P, 0, sizeof(P));
-    TMLaunch L;
+// `pair_first` >= 0 marks items pair_first (gate) and pair_first + 1 (up)
+// of equal shape whose outputs also give h = bf16(silu(gate) * up); the
+// pair's fp32 values and counters take g8_pair_workspace bytes more.
+size_t g8_pair_workspace(int64_t N) { return align256((size_t)(N * 8)) + align256((size_t)(g8_tiles(N) * 32)); }
+
+tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes, bool overlap, bool stall,
+                            cudaStream_t st, int pair_first = -1, uint16_t* h = nullptr) {
+    G8Launch L;
     std::memset(&L, 0, sizeof(L));
-    int order[kMaxItems], n3 = 0;
-    for (int i = 0; i < n; ++i)
-        if (items[i].grid == TB_GRID_INT3) order[n3++] = i;
-    for (int i = 0, k = n3; i < n; ++i)
-        if (items[i].grid != TB_GRID_INT3) order[k++] = i;
     char* w = static_cast<char*>(ws);
     size_t need = 0;
-    int64_t prep = 0, tiles = 0, chunks_all = 0, chunk = 0, cost = 0, part_cost[2] = {0, 0};
+    int64_t prep = 0, tiles = 0, chunk = 0, cost = 0;
     for (int j = 0; j < n; ++j) {
-        if (j == n3) chunk = cost = 0;  // the 2-bit partition starts its positions again
-        Item it = items[order[j]];
-        it.prep_begin = (int32_t)prep;
-        it.rec = reinterpret_cast<uint8_t*>(w + need);
-        need += tm_item_workspace(it.K);
-        prep += it.K / kGroup;
-        P.it[j] = it;
-
-        TMItem& s = L.it[j];
+        const Item& it = items[j];
+        G8Item& s = L.it[j];
+        const int64_t G = it.K / kGroup;
+        s.x = it.X;
         s.scales = it.scales;
-        s.rec = it.rec;
         s.Y = it.Y;
         s.N = it.N;
-        s.G = (int32_t)(it.K / kGroup);
-        s.T = (int32_t)((it.N + 31) / 32);
-        s.C = tm_chunk_groups(it.grid);
+        s.G = (int32_t)G;
+        s.Gp = (int32_t)g8_padded_groups(G);
+        s.T = (int32_t)g8_tiles(it.N);
+        s.C = g8_chunk_groups(it.grid);
         s.cpt = (s.G + s.C - 1) / s.C;
         s.unit_cost = it.grid == TB_GRID_INT3 ? 3 : 2;
         s.grid = it.grid;
@@ -213,45 +208,66 @@ tb_status_t launch_tma_items(const Item* items, int n, void* ws, size_t ws_bytes
         s.chunk_base = chunk;
         s.cost_base = cost;
         s.tile_base = (int32_t)tiles;
+        s.rec = reinterpret_cast<uint8_t*>(w + need);
+        s.spad = g8_needs_spad(G) ? reinterpret_cast<uint16_t*>(w + need + align256((size_t)G * kG8RecBytes))
+                                  : nullptr;
+        need += g8_item_workspace(it.N, it.K);
+        // items reading the same x with the same code width share one record set
+        int owner = -1;
+        for (int i = 0; i < j && owner < 0; ++i)
+            if (items[i].X == it.X && items[i].K == it.K && (items[i].grid == TB_GRID_INT3) == (it.grid == TB_GRID_INT3))
+                owner = i;
+        if (owner >= 0) {
+            s.rec = L.it[owner].rec;
+        } else {
+            G8Prep& P = L.prep[L.n_prep++];
+            P.x = it.X;
+            P.rec = s.rec;
+            P.begin = (int32_t)prep;
+            P.three = it.grid == TB_GRID_INT3 ? 1 : 0;
+            prep += G;
+        }
         chunk += (int64_t)s.T * s.cpt;
-        chunks_all += (int64_t)s.T * s.cpt;
         cost += (int64_t)s.T * s.G * s.unit_cost;
-        part_cost[j < n3 ? 0 : 1] = cost;
         tiles += s.T;
     }
-    P.n_items = n;
-    L.n_items = n;
-    if (part_cost[0] >= ((int64_t)1 << 31) || part_cost[1] >= ((int64_t)1 << 31) || chunks_all >= ((int64_t)1 << 31))
+    if (cost >= ((int64_t)1 << 31) || chunk >= ((int64_t)1 << 31) || prep >= ((int64_t)1 << 31))
         return TB_ERR_UNSUPPORTED;  // partition arithmetic is 32-bit
-    // layout with the device-independent bound on the warp count (the one
-    // tb_workspace_bytes uses), checked before any CUDA call
     L.counters = reinterpret_cast<int32_t*>(w + need);
-    L.partials = reinterpret_cast<float*>(w + need + align256((size_t)(tiles * 4)));
-    need += tm_extra_workspace(tiles, chunks_all);
-    P.zero = L.counters;
-    P.n_zero = (int32_t)tiles;
+    L.n_counters = (int32_t)(tiles * 8);
+    L.partials = reinterpret_cast<float*>(w + need + align256((size_t)(tiles * 8 * 4)));
+    need += g8_extra_workspace(tiles, chunk);
+    L.pair_first = -1;
+    if (pair_first >= 0) {  // after the partials: the pair's values, then its counters
+        const int64_t N = items[pair_first].N;
+        L.pair_first = pair_first;
+        L.pair_vals = reinterpret_cast<float*>(w + need);
+        L.pair_counters = reinterpret_cast<int32_t*>(w + need + align256((size_t)(N * 8)));
+        L.h = h;
+        need += g8_pair_workspace(N);
+    }
     if (!ws || ws_bytes < need) return TB_ERR_ARG;
-    if (tiles > 0x7FFFFFFF || prep > 0x7FFFFFFF) return TB_ERR_SHAPE;
-    for (int j = 0; j < n; ++j)
-        if (!encode_gemv_tma_map(&L.maps[j], P.it[j].packed, P.it[j].grid, P.it[j].N, P.it[j].K)) return TB_ERR_CUDA;
-    const int resident = gemv_tma_resident_warps();
+    for (int j = 0; j < n; ++j) {
+        const G8Item& s = L.it[j];
+        if (!encode_g8_wmap(&L.wmap[j], items[j].packed, items[j].grid, s.N, items[j].K)) return TB_ERR_CUDA;
+        if (!encode_g8_smap(&L.smap[j], s.spad ? s.spad : s.scales, s.N, s.Gp)) return TB_ERR_CUDA;
+    }
+    const int resident = gemv8_ctas();
     if (resident <= 0) return TB_ERR_CUDA;
-    const int64_t W = std::max<int64_t>(1, std::min<int64_t>({(int64_t)resident, chunks_all, kMaxSKWarps}));
-    const int64_t C = part_cost[0] + part_cost[1];
-    int64_t W3 = part_cost[0] == 0 ? 0 : (part_cost[1] == 0 ? W : (W * part_cost[0] + C / 2) / C);
-    if (part_cost[0] > 0) W3 = std::max<int64_t>(W3, 1);
-    if (part_cost[1] > 0) W3 = std::min<int64_t>(W3, W - 1);
-    int64_t W2 = W - W3;
-    // each quota at least one chunk's cost (3-bit: 2 x 3, 2-bit: 4 x 2): then every warp between a
-    // tile's first and last owner owns a chunk of it, which the partial-sum combine relies on
-    if (W3 > 0) W3 = std::max<int64_t>(1, std::min<int64_t>(W3, part_cost[0] / 6));
-    if (W2 > 0) W2 = std::max<int64_t>(1, std::min<int64_t>(W2, part_cost[1] / 8));
-    L.W = (int32_t)(W3 + W2);
-    L.part[0] = {0, n3, 0, (int32_t)W3, (uint32_t)part_cost[0],
-                 (uint32_t)(W3 ? (part_cost[0] + W3 - 1) / W3 : 1)};
-    L.part[1] = {n3, n - n3, (int32_t)W3, (int32_t)W2, (uint32_t)part_cost[1],
-                 (uint32_t)(W2 ? (part_cost[1] + W2 - 1) / W2 : 1)};
-    return cuda_status(launch_gemv_tma(P, (int)prep, L, (int)((L.W + 7) / 8), overlap, st));
+    // every quota at least one chunk's cost (4 x 2 or 2 x 3): then every CTA
+    // between a tile's first and last owner owns a chunk of it, which the
+    // partial-sum combine relies on
+    int64_t nctas = std::max<int64_t>(1, std::min<int64_t>({(int64_t)resident, chunk, kMaxG8Ctas, cost / 8}));
+    const int64_t Q = (cost + nctas - 1) / nctas;
+    nctas = (cost + Q - 1) / Q;
+    L.n_items = n;
+    L.nctas = (int32_t)nctas;
+    L.Ctot = (uint32_t)cost;
+    L.Q = (uint32_t)Q;
+    L.prep_warps = (int32_t)prep;
+    L.stall = stall ? 1 : 0;
+    L.wait_cycles = stall ? kTestWaitCycles : kWaitCycles;
+    return cuda_status(launch_gemv8(L, overlap, st));
 }
 
 }  // namespace
@@ -261,8 +277,15 @@ extern "C" {
 int tb_version(void) { return 100; }
 
 unsigned int tb_wait_timeouts(void) {
-    const unsigned int a = take_wait_timeouts(), b = take_gemv_timeouts();
+    const unsigned int a = take_wait_timeouts(), b = take_g8_timeouts();
     return (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) ? 0xFFFFFFFFu : a + b;
+}
+
+tb_status_t tb_sync_status(tb_stream_t stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TB_ERR_CUDA;
+    const unsigned int n = tb_wait_timeouts();
+    if (n == 0xFFFFFFFFu) return TB_ERR_CUDA;
+    return n ? TB_ERR_TIMEOUT : TB_OK;
 }
 
 const char* tb_status_string(tb_status_t s) {
@@ -273,6 +296,7 @@ const char* tb_status_string(tb_status_t s) {
         case TB_ERR_ALIGN: return "misaligned pointer or leading dimension";
         case TB_ERR_UNSUPPORTED: return "unsupported request";
         case TB_ERR_CUDA: return "CUDA error";
+        case TB_ERR_TIMEOUT: return "a bounded device-side wait gave up: the calls since the last check have no result";
     }
     return "unknown status";
 }
@@ -321,12 +345,9 @@ size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K) {
         const int64_t rem = M % kGemmBlockM;
         return std::max(tb_workspace_bytes(kGemmBlockM, N, K), rem ? tb_workspace_bytes(rem, N, K) : (size_t)0);
     }
-    if (M == 1) {  // chunk count bounded with the smaller chunk (two groups)
-        const int64_t tiles = (N + 31) / 32;
-        return tm_item_workspace(K) + tm_extra_workspace(tiles, tiles * ((K / kGroup + 1) / 2));
-    }
+    if (M == 1) return g8_item_workspace(N, K) + g8_extra_workspace(g8_tiles(N), g8_chunks(TB_GRID_INT3, N, K));
     if (M >= kTCMinM) return gemm_tc_workspace_bytes(M, N, K);
-    return item_workspace(std::min<int64_t>(M, 16), K);
+    return kNoWorkspace;
 }
 
 size_t tb_layer_workspace_bytes(const tb_linear_t* items, int n_items) {
@@ -336,12 +357,11 @@ size_t tb_layer_workspace_bytes(const tb_linear_t* items, int n_items) {
     for (int i = 0; i < n_items; ++i) {
         if (!shape_ok(items[i].N, items[i].K) || !grid_ok(items[i].grid)) return 0;
         if (is_b3(items[i].grid)) continue;  // launched on their own, without workspace
-        const int64_t t = (items[i].N + 31) / 32, C = tm_chunk_groups(items[i].grid);
-        b += tm_item_workspace(items[i].K);
-        tiles += t;
-        chunks += t * ((items[i].K / kGroup + C - 1) / C);
+        b += g8_item_workspace(items[i].N, items[i].K);
+        tiles += g8_tiles(items[i].N);
+        chunks += g8_chunks(items[i].grid, items[i].N, items[i].K);
     }
-    return b + tm_extra_workspace(tiles, chunks);
+    return b + g8_extra_workspace(tiles, chunks);
 }
 
 tb_status_t tb_gemv(const void* packed, tb_grid_t grid, const uint16_t* scales, const uint16_t* x, void* y,
@@ -360,7 +380,7 @@ tb_status_t tb_gemv(const void* packed, tb_grid_t grid, const uint16_t* scales, 
             launch_gemv_rowwarp(packed, grid, scales, x, y, y_dtype, N, K, static_cast<cudaStream_t>(stream)));
     }
     Item it = make_item(packed, grid, scales, x, K, y, y_dtype, N, 1, N, K);
-    return launch_tma_items(&it, 1, workspace, workspace_bytes, false, static_cast<cudaStream_t>(stream));
+    return launch_g8_items(&it, 1, workspace, workspace_bytes, false, false, static_cast<cudaStream_t>(stream));
 }
 
 tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, const uint16_t* X, int64_t ldx,
@@ -399,7 +419,7 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     }
     if (M == 1) {
         Item it = make_item(packed, grid, scales, X, ldx, Y, y_dtype, N, 1, N, K);
-        return launch_tma_items(&it, 1, workspace, workspace_bytes, false, st);
+        return launch_g8_items(&it, 1, workspace, workspace_bytes, false, false, st);
     }
     if (M >= kTCMinM) {
         if (workspace_bytes < gemm_tc_workspace_bytes(M, N, K)) return TB_ERR_ARG;
@@ -414,7 +434,7 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
         const int mb = (int)std::min<int64_t>(16, M - m0);
         Item it = make_item(packed, grid, scales, X + m0 * ldx, ldx, static_cast<char*>(Y) + m0 * ldy * ysz, y_dtype,
                             ldy, mb, N, K);
-        if ((s = launch_items(&it, 1, mb > 8 ? 2 : 1, workspace, workspace_bytes, false, st)) != TB_OK) return s;
+        if ((s = launch_items(&it, 1, mb > 8 ? 2 : 1, st)) != TB_OK) return s;
     }
     return TB_OK;
 }
@@ -422,7 +442,7 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
 tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags, void* workspace,
                           size_t workspace_bytes, tb_stream_t stream) {
     if (!items || n_items < 1 || n_items > TB_MAX_LAYER_ITEMS) return TB_ERR_ARG;
-    if ((flags & ~(unsigned)TB_FLAG_OVERLAP_PREVIOUS) != 0 || !workspace) return TB_ERR_ARG;
+    if ((flags & ~(unsigned)(TB_FLAG_OVERLAP_PREVIOUS | TB_FLAG_TEST_STALL)) != 0 || !workspace) return TB_ERR_ARG;
     if (!aligned(workspace, 256)) return TB_ERR_ALIGN;
     Item its[kMaxItems];
     int n_main = 0;
@@ -441,8 +461,9 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (n_main > 0) {
-        const tb_status_t s = launch_tma_items(its, n_main, workspace, workspace_bytes,
-                                               (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0, st);
+        const tb_status_t s = launch_g8_items(its, n_main, workspace, workspace_bytes,
+                                              (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0,
+                                              (flags & TB_FLAG_TEST_STALL) != 0, st);
         if (s != TB_OK) return s;
     }
     // items in the 5-trits-per-byte layout: one launch each, after the grouped launch
@@ -453,6 +474,37 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
             return TB_ERR_CUDA;
     }
     return TB_OK;
+}
+
+size_t tb_gate_up_workspace_bytes(const tb_linear_t* gate, const tb_linear_t* up) {
+    if (!gate || !up || gate->N != up->N || gate->K != up->K) return 0;
+    const tb_linear_t two[2] = {*gate, *up};
+    if (is_b3(gate->grid) || is_b3(up->grid)) return 0;
+    const size_t b = tb_layer_workspace_bytes(two, 2);
+    return b ? b + g8_pair_workspace(gate->N) : 0;
+}
+
+tb_status_t tb_gate_up_silu(const tb_linear_t* gate, const tb_linear_t* up, uint16_t* h, unsigned flags,
+                            void* workspace, size_t workspace_bytes, tb_stream_t stream) {
+    if (!gate || !up || !h || !workspace) return TB_ERR_ARG;
+    if ((flags & ~(unsigned)TB_FLAG_OVERLAP_PREVIOUS) != 0) return TB_ERR_ARG;
+    if (gate->N != up->N || gate->K != up->K) return TB_ERR_SHAPE;
+    if (!aligned(workspace, 256) || !aligned(h, 2)) return TB_ERR_ALIGN;
+    Item its[2];
+    const tb_linear_t* l2[2] = {gate, up};
+    for (int i = 0; i < 2; ++i) {
+        const tb_linear_t& l = *l2[i];
+        tb_status_t s = check_weights(l.packed, l.grid, l.scales, l.N, l.K);
+        if (s != TB_OK) return s;
+        if (!l.x) return TB_ERR_ARG;
+        if ((s = check_out(l.y, l.y_dtype)) != TB_OK) return s;
+        if (!aligned(l.x, 16)) return TB_ERR_ALIGN;
+        if (is_b3(l.grid)) return TB_ERR_UNSUPPORTED;  // the 5-trit layout runs its own kernel
+        its[i] = make_item(l.packed, l.grid, l.scales, l.x, l.K, l.y, l.y_dtype, l.N, 1, l.N, l.K);
+    }
+    if (workspace_bytes < tb_gate_up_workspace_bytes(gate, up)) return TB_ERR_ARG;
+    return launch_g8_items(its, 2, workspace, workspace_bytes, (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0, false,
+                           static_cast<cudaStream_t>(stream), 0, h);
 }
 
 }  // extern "C"
@@ -513,7 +565,7 @@ tb_status_t tb_gemv_noalloc(const void* packed, tb_grid_t grid, const uint16_t* 
     void* scratch = noalloc_scratch();
     if (!scratch) return TB_ERR_CUDA;
     Item it = make_item(packed, grid, scales, x, K, y, y_dtype, N, 1, N, K);
-    return launch_tma_items(&it, 1, scratch, TB_NOALLOC_SCRATCH_BYTES, false, static_cast<cudaStream_t>(stream));
+    return launch_g8_items(&it, 1, scratch, TB_NOALLOC_SCRATCH_BYTES, false, false, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -26,66 +26,74 @@ __host__ __device__ inline int grid_offset(int g) { return g == kInt3 ? 4 : 2; }
 // bytes of one packed row of K weights
 __host__ __device__ inline int64_t row_bytes(int g, int64_t K) { return g == kInt3 ? 3 * K / 8 : K / 4; }
 
-// ---- one linear layer inside a launch ------------------------------------
+// ---- one small-batch product inside a launch (tb_linear.cu) -----------------
 struct Item {
     const uint8_t* packed;
     const uint16_t* scales;
     const uint16_t* X;   // [M][ldx] bf16 activations
     void* Y;             // [M][ldy] outputs
-    uint16_t* xs;        // workspace: [M][K] prepared activations (see tb_linear.cu)
-    float2* cf;          // workspace: [K/128][M] per-group (offset * sum x, 2^S)
     int64_t N, K, ldx, ldy;
     int32_t grid, ydt, M;
-    int32_t cta_begin;   // first CTA of this item in the main launch
-    int32_t prep_begin;  // first warp of this item in the preparation launch
+    int32_t cta_begin;   // first CTA of this item in the launch
     int32_t ksplit;      // warps sharing one 32-row tile (1, 2, 4 or 8)
-    uint8_t* rec;        // batch-1 TMA path: per-group records (see kRecBytes) instead of xs / cf
 };
-
-// Prepared activations of one 128-group for the batch-1 TMA kernel, one
-// contiguous record: the 128 scaled activations in MMA order, first half at
-// bytes 0..127, (offset * sum x, 2^S) at 128..135, zero at 136..143, second
-// half at 144..271 (the 16-byte gap keeps the fragment loads free of bank
-// conflicts).  A chunk of consecutive groups is one bulk copy.
-constexpr int kRecBytes = 272;
 
 struct Launch {
     Item it[kMaxItems];
     int32_t n_items;
     int32_t scl_stride;  // scales staged per row per warp (>= groups per warp)
-    int32_t* zero;       // int32 words the preparation kernel clears (stream-K tile counters)
-    int32_t n_zero;
 };
 
-// ---- stream-K batch-1 launch (see tb_linear.cu) ----------------------------
-// Two partitions side by side: the 3-bit items (it[0 .. n3)) on warps
-// [0, W3), the 2-bit items (it[n3 .. n_items)) on warps [W3, W); tile-group
-// and cost positions of the 2-bit items start again at 0.
-struct SKPart {
-    int32_t first, count;  // items
-    int32_t W0, W;         // first warp, warps
-    uint32_t C, Q;         // total cost, cost quota per warp (tb_partition.h)
-};
+// ---- batch-1 launch on the integer tensor path (see tb_gemv8.cu) ----------
+// One activation record per 128-group: the group's activations as eight
+// signed 7-bit digit columns in the order the MMA B fragments are read
+// (1024 bytes), then per digit pair t = 0..3 the accumulator start values
+// of digit columns 2t, 2t+1 and the float 2^(14 t - F) (64 bytes).
+constexpr int kG8RecBytes = 1088;
+constexpr int kG8TileRows = 256;  // rows of a tile: 8 consumer warps x 32 rows
 
-// Batch-1 TMA kernel (tb_linear.cu): items read in chunks of C groups x 32
-// rows through one 2-D tensor map each (see tb_partition.h, ChunkItem).
-struct TMItem {
-    const uint16_t* scales;
-    const uint8_t* rec;  // G records of kRecBytes
+struct G8Item {
+    const uint16_t* x;       // [K] bf16 activations
+    const uint16_t* scales;  // [N][G] bf16, the caller's
+    uint16_t* spad;          // [N][Gp] copy of the scales with rows padded to 8 groups, or null
+    uint8_t* rec;            // [G] records of kG8RecBytes
     void* Y;
     int64_t N;
-    int64_t chunk_base, cost_base;  // ChunkItem fields
+    int64_t chunk_base, cost_base;  // ChunkItem fields (tb_partition.h)
     int32_t T, G, C, cpt, unit_cost;
-    int32_t grid, ydt, tile_base;
+    int32_t grid, ydt, tile_base, Gp;
 };
 
-struct TMLaunch {
-    CUtensorMap maps[kMaxItems];  // packed weights of item i: bytes x rows, box (C group bytes) x 32
-    TMItem it[kMaxItems];
-    int32_t n_items, W;
-    SKPart part[2];  // 3-bit items first, then the 2-bit container
-    int32_t* counters;
-    float* partials;
+// One set of activation records the preparation kernel writes: items that
+// read the same x with the same code width share one.
+struct G8Prep {
+    const uint16_t* x;
+    uint8_t* rec;
+    int32_t begin;  // first preparation warp (one per group)
+    int32_t three;  // the 3-bit slot map
+};
+
+struct G8Launch {
+    CUtensorMap wmap[kMaxItems];  // packed weights: bytes x rows, box (C groups) x 256 rows
+    CUtensorMap smap[kMaxItems];  // scales [N][Gp] bf16: box 8 groups x 256 rows
+    G8Item it[kMaxItems];
+    int32_t n_items, nctas;
+    uint32_t Ctot, Q;      // total cost and cost quota per CTA (tb_partition.h)
+    int32_t* counters;     // [tiles][8] arrival counters, zeroed by the preparation kernel
+    int32_t n_counters;
+    float* partials;       // [nctas][2][256] partial sums of split tiles
+    G8Prep prep[kMaxItems];
+    int32_t n_prep;
+    int32_t prep_warps;    // one per group of every record set
+    int32_t stall;         // test hook: the copies are never issued, every wait gives up
+    long long wait_cycles; // bound of every wait
+    // gated MLP input: items pair_first (gate) and pair_first + 1 (up) of equal
+    // shape; the last of the two to finish a warp's 32 rows writes
+    // h = bf16(silu(gate) * up) for them (-1: no pair)
+    int32_t pair_first;
+    int32_t* pair_counters;  // [tiles of the pair][8], cleared by the preparation kernel
+    float* pair_vals;        // [2][N] the pair's fp32 results
+    uint16_t* h;             // [N] bf16
 };
 
 // ---- cache-controlled loads ----------------------------------------------
@@ -145,6 +153,82 @@ __device__ __forceinline__ uint32_t bit_mux(uint32_t a, uint32_t b, uint32_t m) 
     uint32_t d;
     asm("lop3.b32 %0, %1, %2, %3, 0xCA;" : "=r"(d) : "r"(m), "r"(b), "r"(a));
     return d;
+}
+
+// ---- exact signed decode to bf16 (the products with M >= 2) -----------------
+// A stored code u (2 or 3 bits) at mantissa bit p <= 4 of each 16-bit half,
+// OR'ed with the exponent field of 2^(7-p), is the bf16 value 2^(7-p) + u;
+// one bf16x2 subtraction of 2^(7-p) + offset then leaves c = u - offset
+// exactly (both operands lie in [2^(7-p), 2^(8-p)), the difference is a
+// small integer).  So the tensor cores see the signed codeword itself: a
+// zero codeword contributes exactly nothing.
+__host__ __device__ constexpr uint32_t dec_exp(int p) { return ((uint32_t)(134 - p) << 7) * 0x00010001u; }
+__host__ __device__ constexpr uint32_t dec_bias(int p, int off) { return dec_exp(p) | ((uint32_t)(off << p) * 0x00010001u); }
+
+__device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+// the pair of fields of w selected by mask (at bit p), as exact signed bf16
+template <int P, int OFF>
+__device__ __forceinline__ uint32_t dec_pair(uint32_t w, uint32_t mask) {
+    return sub_bf16x2(and_or(w, mask, dec_exp(P)), dec_bias(P, OFF));
+}
+
+// 2-bit word (codes 2m at bits 2m, 2m+1 at bits 16+2m): r[m] = the codes
+// 2m, 2m+1 as a bf16 pair (natural order).  Fields 0-2 in place, 3-5 after
+// >> 6, 6-7 after >> 12 (each lands at bit 0, 2 or 4).
+template <int OFF>
+__device__ __forceinline__ void decode2_signed(uint32_t w, uint32_t (&r)[8]) {
+    const uint32_t w6 = w >> 6, w12 = w >> 12;
+    r[0] = dec_pair<0, OFF>(w, 0x00030003u);
+    r[1] = dec_pair<2, OFF>(w, 0x000C000Cu);
+    r[2] = dec_pair<4, OFF>(w, 0x00300030u);
+    r[3] = dec_pair<0, OFF>(w6, 0x00030003u);
+    r[4] = dec_pair<2, OFF>(w6, 0x000C000Cu);
+    r[5] = dec_pair<4, OFF>(w6, 0x00300030u);
+    r[6] = dec_pair<0, OFF>(w12, 0x00030003u);
+    r[7] = dec_pair<2, OFF>(w12, 0x000C000Cu);
+}
+
+// masks with a bit at first + 3i + shift (i < count) in both halves
+__host__ __device__ constexpr uint32_t bits3_at(int first, int count, int shift) {
+    uint32_t m = 0;
+    for (int i = 0; i < count; ++i) m |= (1u << (first + 3 * i + shift)) | (1u << (16 + first + 3 * i + shift));
+    return m;
+}
+
+// 3-bit block (bit f of plane p is bit p of code 2f, bit 16+f of code
+// 2f+1): r[f] = the codes 2f, 2f+1 as a bf16 pair (natural order).  The
+// planes are merged into 3-bit fields at bit f (planes 1 and 2 shifted up
+// by 1 and 2), in three sets of every third field; shifts bring each field
+// to bit p <= 4; fields 14 and 15 are assembled from the planes realigned
+// to the right.
+__device__ __forceinline__ void decode3_signed(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t (&r)[16]) {
+    const uint32_t q1 = p1 << 1, q2 = p2 << 2;
+    const uint32_t zA = bit_mux(bit_mux(p0, q1, bits3_at(0, 5, 1)), q2, bits3_at(0, 5, 2));  // fields 0,3,6,9,12
+    const uint32_t zB = bit_mux(bit_mux(p0, q1, bits3_at(1, 5, 1)), q2, bits3_at(1, 5, 2));  // fields 1,4,7,10,13
+    const uint32_t zC = bit_mux(bit_mux(p0, q1, bits3_at(2, 4, 1)), q2, bits3_at(2, 4, 2));  // fields 2,5,8,11
+    const uint32_t a6 = zA >> 6, a12 = zA >> 12, b6 = zB >> 6, b12 = zB >> 12;
+    const uint32_t c3 = zC >> 3, c6 = zC >> 6, c9 = zC >> 9;
+    r[0] = dec_pair<0, 4>(zA, 0x00070007u);
+    r[3] = dec_pair<3, 4>(zA, 0x00380038u);
+    r[6] = dec_pair<0, 4>(a6, 0x00070007u);
+    r[9] = dec_pair<3, 4>(a6, 0x00380038u);
+    r[12] = dec_pair<0, 4>(a12, 0x00070007u);
+    r[1] = dec_pair<1, 4>(zB, 0x000E000Eu);
+    r[4] = dec_pair<4, 4>(zB, 0x00700070u);
+    r[7] = dec_pair<1, 4>(b6, 0x000E000Eu);
+    r[10] = dec_pair<4, 4>(b6, 0x00700070u);
+    r[13] = dec_pair<1, 4>(b12, 0x000E000Eu);
+    r[2] = dec_pair<2, 4>(zC, 0x001C001Cu);
+    r[5] = dec_pair<2, 4>(c3, 0x001C001Cu);
+    r[8] = dec_pair<2, 4>(c6, 0x001C001Cu);
+    r[11] = dec_pair<2, 4>(c9, 0x001C001Cu);
+    const uint32_t s0 = p0 >> 14, s1 = p1 >> 13, s2 = p2 >> 12;  // plane p of fields 14, 15 at bits p, p + 1
+    r[14] = dec_pair<0, 4>(bit_mux(bit_mux(s0, s1, 0x00020002u), s2, 0x00040004u), 0x00070007u);
+    r[15] = dec_pair<1, 4>(bit_mux(bit_mux(s0, s1, 0x00040004u), s2, 0x00080008u), 0x000E000Eu);
 }
 
 }  // namespace tb

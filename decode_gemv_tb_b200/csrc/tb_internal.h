@@ -21,26 +21,28 @@ cudaError_t launch_pack(const void* W, int w_dtype, int64_t N, int64_t K, int gr
                         void* packed, int32_t* bad_count, cudaStream_t st);
 cudaError_t launch_unpack(const void* packed, int grid, int64_t N, int64_t K, int8_t* codes, cudaStream_t st);
 
-// Grouped linear launch (GEMV when every item has M == 1): the activation
-// preparation kernel, then the main kernel as its programmatic dependent.
-// `nt` is the number of 8-wide column tiles (1 or 2), `ctas` the main grid,
-// `prep_warps` the preparation warp count; `overlap` also launches the
-// preparation kernel as a programmatic dependent of the previous work.
-cudaError_t launch_linear(const Launch& L, int nt, int ctas, int prep_warps, bool overlap, cudaStream_t st);
+// Small-batch launch (2 <= M <= 16 batch rows per item): one kernel, no
+// workspace.  `nt` is the number of 8-wide column tiles (1 or 2), `ctas`
+// the grid.
+cudaError_t launch_linear(const Launch& L, int nt, int ctas, cudaStream_t st);
 // dynamic shared memory of the main kernel
 size_t linear_smem_bytes(int nt, int scl_stride);
 
-struct TMLaunch;
-// Batch-1 path with TMA staging: preparation kernel (writes records, clears
-// P.zero) + k_gemv_tma.  The tensor map of each item comes from
-// encode_gemv_tma_map (false if the driver cannot encode it).
-cudaError_t launch_gemv_tma(const Launch& P, int prep_warps, const TMLaunch& L, int ctas, bool overlap,
-                            cudaStream_t st);
-bool encode_gemv_tma_map(CUtensorMap* map, const void* packed, int grid, int64_t N, int64_t K);
-// warps of k_gemv_tma resident at once on the current device (0 on error)
-int gemv_tma_resident_warps();
-// bounded waits of k_gemv_tma that gave up since the last call (clears)
-unsigned int take_gemv_timeouts();
+struct G8Launch;
+// Batch-1 GEMV on the integer tensor path (tb_gemv8.cu): preparation kernel
+// (activation records, cleared counters, padded scale copies) + k_gemv8 as
+// its programmatic dependent.  `overlap` also launches the preparation
+// kernel as a programmatic dependent of the previous work.
+cudaError_t launch_gemv8(const G8Launch& L, bool overlap, cudaStream_t st);
+// weights of one matrix (box: one chunk x 256 rows) / its scales [N][Gp]
+bool encode_g8_wmap(CUtensorMap* map, const void* packed, int grid, int64_t N, int64_t K);
+bool encode_g8_smap(CUtensorMap* map, const uint16_t* scales, int64_t N, int64_t Gp);
+// groups per chunk (4 for the 2-bit container, 2 for 3 bits)
+int g8_chunk_groups(int grid);
+// CTAs of k_gemv8 resident at once on the current device (0 on error)
+int gemv8_ctas();
+// bounded waits of k_gemv8 that gave up since the last call (clears)
+unsigned int take_g8_timeouts();
 
 // Batch-1 GEMV in one launch, one warp per output row, no workspace: the
 // 5-trits-per-byte layout, and small problems in the other layouts.  The

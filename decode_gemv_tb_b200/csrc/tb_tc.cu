@@ -3,38 +3,32 @@
 //
 // ThinkBit page "ThinkBit은 2비트 양자화에서 추론 능력 보존을 추론 평가로
 // 검증한다" (onedev.kr/papers/1416), section 어떻게 동작하나: w = c * s with
-// one bf16 scale per 128 input weights; the product per output row n,
-// batch row m and 128-group g is
-//     Y[m][n] += s[n][g] * (sum_k u[n][k] X[m][k]  -  offset * sum_k X[m][k])
-// with u = c + offset the stored code.
+// one bf16 scale per 128 input weights; the product per output row n, batch
+// row m and 128-group g is
+//     Y[m][n] += s[n][g] * sum_k c[n][k] X[m][k].
 //
 // Data flow of one CTA (a 128-row tile of W and a contiguous range of its
 // 128-groups; 256 decoder threads, two per weight row, and one producer
 // warp):
 //   * each decoder streams its half of the row's packed group through a
-//     private cp.async ring six groups deep and decodes it without
-//     arithmetic: masking one field at bit position p of each 16-bit half
-//     gives a bf16 pair u * 2^(p-133) (a bf16 pattern below 256 is exactly
-//     that multiple of 2^-133); the pairs go to tensor memory (tcgen05.st),
-//     one TMEM lane per row, k in natural order along the columns -- the A
-//     operand;
-//   * the preparation kernel has stored X per group, with one exponent S_g
-//     for all batch rows, as
-//         X[m][k] * 2^(133 - S_g - p(k))       (exact: powers of two)
-//     in the K-major core-matrix layout the MMA reads from shared memory,
-//     each row followed by a 16-wide correction slice (sum_k X[m][k] *
-//     2^(120 - S_g) as three bf16 terms), then 2^S_g; and the group scales
-//     transposed per tile; the producer brings a group's X and the tile's
-//     128 scales in with two bulk copies, two groups ahead -- the B operand;
+//     private cp.async ring six groups deep and decodes it to the signed
+//     codeword itself, exactly, as bf16 (tb_device.cuh: the stored field
+//     OR'ed into the mantissa of 2^(7-p), minus 2^(7-p) + offset); the pairs
+//     go to tensor memory (tcgen05.st), one TMEM lane per row, k in natural
+//     order along the columns -- the A operand;
+//   * the preparation kernel has copied X per group into the K-major
+//     core-matrix layout the MMA reads from shared memory (rows M .. NP - 1
+//     zero) and transposed the group scales per tile; the producer brings a
+//     group's X and the tile's 128 scales in with two bulk copies, two groups
+//     ahead -- the B operand;
 //   * the producer warp issues the group's eight 128 x NP x 16 MMAs (bf16
 //     in, fp32 accumulate in tensor memory; one elected lane of the
-//     converged warp, so the operands stay warp-uniform), a ninth with A a
-//     constant shared-memory tile (-offset * 2^-120 in three k slots) and B
-//     the correction slices, which subtracts offset * sum X, and commits
-//     them to an mbarrier;
+//     converged warp, so the operands stay warp-uniform) and commits them to
+//     an mbarrier; every product c * x is exact and a zero codeword
+//     contributes nothing;
 //   * while they run, each decoder reads its half of the previous group's
 //     accumulator row back (tcgen05.ld) and applies the group scale:
-//         acc[m] += (s * 2^S_g) * D[m]
+//         acc[m] += s * D[m]
 //     A and D are double-buffered in tensor memory (2 x 64 + 2 x NP
 //     columns of the 256 a CTA allocates; two CTAs per SM).
 // K-splits of one tile are combined by the last CTA to finish, in split
@@ -62,22 +56,10 @@ constexpr int kTCTargetCtas = 296;               // 2 CTAs on each of 148 SMs
 constexpr int kTCMaxSplits = 16;
 constexpr size_t kTCMinSmem = 80 * 1024;         // at most two CTAs (2 x 256 TMEM columns) per SM
 
-// one prepared group: NP rows x 144 bf16 (128 activations + a 16-wide
-// correction slice) in the K-major core-matrix layout (18 chunks of 8 k per
-// 8 rows: 2304 bytes per 8 rows), then 2^S_g as a float and 12 zero bytes
-__host__ __device__ constexpr int tc_group_bytes(int np) { return np * 288 + 16; }
-constexpr int kTCBRowGroupB = 18 * 128;  // stride between 8-row core-matrix groups of B
-
-// field position (bit of its 16-bit half) of 3-bit field f after the decode below
-__host__ __device__ constexpr int pos3(int f) { return f < 12 ? f % 6 : (f & 1); }
-
-__device__ __forceinline__ uint32_t shr_fma(uint32_t x, int k) { return __umulhi(x, 1u << (32 - k)); }
-
-constexpr uint32_t bits_at(int first, int count, int shift) {
-    uint32_t m = 0;
-    for (int i = 0; i < count; ++i) m |= (1u << (first + 3 * i + shift)) | (1u << (16 + first + 3 * i + shift));
-    return m;
-}
+// one prepared group: NP rows x 128 bf16 activations in the K-major
+// core-matrix layout (16 chunks of 8 k per 8 rows: 2048 bytes per 8 rows)
+__host__ __device__ constexpr int tc_group_bytes(int np) { return np * 256; }
+constexpr int kTCBRowGroupB = 16 * 128;  // stride between 8-row core-matrix groups of B
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -161,14 +143,6 @@ __device__ __forceinline__ void mma_ts_warp(uint32_t d, uint32_t a, uint64_t bde
         "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u)
         : "memory");
 }
-// D[tmem d] += A[smem desc a] x B[smem desc b], same warp-level issue
-__device__ __forceinline__ void mma_ss_warp(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc) {
-    asm volatile(
-        "{\n .reg .pred e, p;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
-        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}" ::"r"(d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(1u), "r"(0u)
-        : "memory");
-}
 // commit by the same elected lane (the lowest active one) that issued the MMAs
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
     asm volatile(
@@ -190,50 +164,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int np) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(np >> 3) << 17) | ((uint32_t)(kTCRows >> 4) << 24);
 }
 
-// ---- decode: one row's group into 64 bf16 pairs (TMEM columns) -----------------
-// 2-bit container: word i holds codes 16i .. 16i+15; field m (codes
-// 16i+2m, 16i+2m+1) masked in place for m < 4 (p = 2m) and after >> 8 for
-// m >= 4 (p = 2m - 8): column 8i + m.
+// ---- decode: a row's half group into 32 bf16 pairs (TMEM columns) ---------
+// 2-bit container: word i holds codes 16i .. 16i+15 -> columns 8i .. 8i+7.
 __device__ __forceinline__ void decode2_pair(uint32_t w0, uint32_t w1, uint32_t (&r)[16]) {
-    const uint32_t h0 = shr_fma(w0, 8), h1 = shr_fma(w1, 8);
+    uint32_t a[8], b[8];
+    decode2_signed<2>(w0, a);
+    decode2_signed<2>(w1, b);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const uint32_t mk = 0x00030003u << (2 * m);
-        r[m] = w0 & mk;
-        r[4 + m] = h0 & mk;
-        r[8 + m] = w1 & mk;
-        r[12 + m] = h1 & mk;
+    for (int m = 0; m < 8; ++m) {
+        r[m] = a[m];
+        r[8 + m] = b[m];
     }
-}
-// 3-bit block: planes p0..p2 of codes 32j .. 32j+31; field f (codes 32j+2f,
-// 32j+2f+1) assembled from the planes at position pos3(f): column 16j + f.
-__device__ __forceinline__ void decode3_block(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t (&r)[16]) {
-    const uint32_t q1 = p1 << 1, q2 = p2 << 2;
-    const uint32_t zA = bit_mux(bit_mux(p0, q1, bits_at(0, 5, 1)), q2, bits_at(0, 5, 2));  // fields 0,3,6,9,12
-    const uint32_t zB = bit_mux(bit_mux(p0, q1, bits_at(1, 5, 1)), q2, bits_at(1, 5, 2));  // fields 1,4,7,10,13
-    const uint32_t zC = bit_mux(bit_mux(p0, q1, bits_at(2, 4, 1)), q2, bits_at(2, 4, 2));  // fields 2,5,8,11
-    const uint32_t a6 = shr_fma(zA, 6), b6 = shr_fma(zB, 6), c6 = shr_fma(zC, 6);
-    const uint32_t a12 = shr_fma(zA, 12), b12 = shr_fma(zB, 12);
-    // fields 14, 15 (plane bits 14/15 and 30/31): plane p realigned right by 14 - p
-    const uint32_t r0 = shr_fma(p0, 14), r1 = shr_fma(p1, 13), r2 = shr_fma(p2, 12);
-    const uint32_t z14 = bit_mux(bit_mux(r0, r1, 0x00020002u), r2, 0x00040004u);
-    const uint32_t z15 = bit_mux(bit_mux(r0, r1, 0x00040004u), r2, 0x00080008u);
-    r[0] = zA & 0x00070007u;
-    r[1] = zB & 0x000E000Eu;
-    r[2] = zC & 0x001C001Cu;
-    r[3] = zA & 0x00380038u;
-    r[4] = zB & 0x00700070u;
-    r[5] = zC & 0x00E000E0u;
-    r[6] = a6 & 0x00070007u;
-    r[7] = b6 & 0x000E000Eu;
-    r[8] = c6 & 0x001C001Cu;
-    r[9] = a6 & 0x00380038u;
-    r[10] = b6 & 0x00700070u;
-    r[11] = c6 & 0x00E000E0u;
-    r[12] = a12 & 0x00070007u;
-    r[13] = b12 & 0x000E000Eu;
-    r[14] = z14 & 0x00070007u;
-    r[15] = z15 & 0x000E000Eu;
 }
 
 }  // namespace
@@ -254,23 +195,10 @@ struct TCArgs {
 namespace {
 
 // ---- preparation: one CTA per group g -----------------------------------------
-// Rows m < M of X for group g become X[m][k] * 2^(133 - S_g - p(k)), with one
-// exponent S_g = (largest exponent of the group over all batch rows) + 7, in
-// the K-major core-matrix layout; rows M .. NP - 1 are zero.  The 16-wide
-// correction slice of row m holds Sum_k X[m][k] * 2^(120 - S_g) split exactly
-// into three bf16 terms: against the constant A slice (-offset * 2^-120 in
-// three k slots) the MMA then adds -offset * Sum_k X[m][k] * 2^-S_g to
-// D[.][m], so that D = 2^-S_g * (Sum_k u X - offset Sum_k X) and the epilogue
-// is acc += (s * 2^S_g) * D.  The CTAs also clear the tile counters and
-// transpose the group scales per 128-row tile.
-__device__ __forceinline__ float pow2_scale(float v, int sh) {  // v * 2^sh, sh within +-252, exact
-    const int s1 = sh >> 1, s2 = sh - s1;
-    return v * __int_as_float((s1 + 127) << 23) * __int_as_float((s2 + 127) << 23);
-}
-
+// Rows m < M of X for group g are copied into the K-major core-matrix
+// layout the MMA reads (rows M .. NP - 1 zero).  The CTAs also clear the
+// tile counters and transpose the group scales per 128-row tile.
 __global__ void __launch_bounds__(256) k_prep_tc(const __grid_constant__ TCArgs A) {
-    __shared__ int wmax[8];
-    __shared__ float sums[64];
     for (int i = blockIdx.x * 256 + threadIdx.x; i < A.tiles; i += gridDim.x * 256) A.counters[i] = 0;
     // scales transposed per 128-row tile, so that one bulk copy brings a tile's 128 scales of a group
     // (element i: tile-group pair i / 128 = t * G + g, row t * 128 + i % 128)
@@ -283,67 +211,13 @@ __global__ void __launch_bounds__(256) k_prep_tc(const __grid_constant__ TCArgs 
     const int g = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (g >= A.G) return;  // uniform over the CTA
     uint8_t* gb = A.bprep + (int64_t)g * tc_group_bytes(A.NP);
-    // pass 1: largest exponent over every row, and each row's sum
-    int e = 0;
-    for (int m = warp; m < A.M; m += 8) {
-        const uint2 raw = *reinterpret_cast<const uint2*>(A.X + (int64_t)m * A.ldx + (int64_t)g * kGroup + 4 * lane);
-        const uint32_t hv[4] = {raw.x & 0xFFFFu, raw.x >> 16, raw.y & 0xFFFFu, raw.y >> 16};
-        float sum = 0.f;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            e = max(e, (int)((hv[j] >> 7) & 0xFFu));
-            sum += bf16_bits_to_float(hv[j]);
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) sums[m] = sum;
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
-    if (lane == 0) wmax[warp] = e;
-    __syncthreads();
-    e = wmax[0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) e = max(e, wmax[w]);
-    // S = exponent of max |x| + 7 (a zero or subnormal group counts as 2^-126)
-    const int S = min(max(e, 1) - 127 + 7, 127);
-    // pass 2: the scaled rows and their correction slices
     for (int m = warp; m < A.NP; m += 8) {
         uint8_t* rowb = gb + (m >> 3) * kTCBRowGroupB + (m & 7) * 16;  // chunk c of row m at rowb + 128 c
-        uint2 outv = make_uint2(0u, 0u);
-        uint4 corr = make_uint4(0u, 0u, 0u, 0u);
-        if (m < A.M) {
-            const uint2 raw =
-                *reinterpret_cast<const uint2*>(A.X + (int64_t)m * A.ldx + (int64_t)g * kGroup + 4 * lane);
-            const uint32_t hv[4] = {raw.x & 0xFFFFu, raw.x >> 16, raw.y & 0xFFFFu, raw.y >> 16};
-            uint32_t out[2] = {0u, 0u};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int k = 4 * lane + j;
-                const int p = A.grid == kInt3 ? pos3((k & 31) >> 1) : 2 * ((k >> 1) & 3);
-                const float v = pow2_scale(bf16_bits_to_float(hv[j]), 133 - S - p);  // exact: 8 significant bits
-                out[j >> 1] |= (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v)) << (16 * (j & 1));
-            }
-            outv = make_uint2(out[0], out[1]);
-            if (lane == 0) {
-                const float v = pow2_scale(sums[m], 120 - S);
-                const __nv_bfloat16 h1 = __float2bfloat16_rn(v);
-                const float r1 = v - __bfloat162float(h1);
-                const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
-                const __nv_bfloat16 h3 = __float2bfloat16_rn(r1 - __bfloat162float(h2));
-                corr.x = (uint32_t)__bfloat16_as_ushort(h1) | ((uint32_t)__bfloat16_as_ushort(h2) << 16);
-                corr.y = (uint32_t)__bfloat16_as_ushort(h3);
-            }
-        }
+        uint2 v = make_uint2(0u, 0u);
+        if (m < A.M) v = *reinterpret_cast<const uint2*>(A.X + (int64_t)m * A.ldx + (int64_t)g * kGroup + 4 * lane);
         // elements k = 4 lane .. 4 lane + 3: chunk lane / 2, bytes 8 (lane % 2)
-        *reinterpret_cast<uint2*>(rowb + (lane >> 1) * 128 + 8 * (lane & 1)) = outv;
-        if (lane == 0) {
-            *reinterpret_cast<uint4*>(rowb + 16 * 128) = corr;                       // k 128 .. 135
-            *reinterpret_cast<uint4*>(rowb + 17 * 128) = make_uint4(0u, 0u, 0u, 0u);  // k 136 .. 143
-        }
+        *reinterpret_cast<uint2*>(rowb + (lane >> 1) * 128 + 8 * (lane & 1)) = v;
     }
-    if (threadIdx.x == 0)
-        *reinterpret_cast<float4*>(gb + A.NP * 288) = make_float4(__int_as_float((S + 127) << 23), 0.f, 0.f, 0.f);
 }
 
 // ---- main kernel -------------------------------------------------------------
@@ -435,9 +309,9 @@ __device__ __forceinline__ void decode_half(const uint4* src, uint32_t acol) {
         const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         constexpr int o = 2 * H;
         uint32_t r[16];
-        decode3_block(w[o], w[o + 1], w[o + 2], r);
+        decode3_signed(w[o], w[o + 1], w[o + 2], r);
         tmem_st16(acol, r);
-        decode3_block(w[o + 3], w[o + 4], w[o + 5], r);
+        decode3_signed(w[o + 3], w[o + 4], w[o + 5], r);
         tmem_st16(acol + 16, r);
     }
 }
@@ -452,8 +326,6 @@ __global__ void __launch_bounds__(kTCBlock, 2) k_gemm_tc(const __grid_constant__
     constexpr uint32_t kIdesc = idesc_bf16(NP);
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* const wring = smem + kTCStages * SB;  // [kTCWStages][256][kTCWStride]
-    // constant A of the correction slice: 128 rows x 16 k, -offset * 2^-120 in k = 0, 1, 2
-    uint8_t* const aconst = wring + kTCWStages * kTCDecoders * kTCWStride;
     __shared__ __align__(8) uint64_t bar_full[kTCStages];
     __shared__ __align__(8) uint64_t bar_afull[2], bar_dfree[2], bar_mma[2];
     __shared__ uint32_t tmem_sh;
@@ -467,13 +339,6 @@ __global__ void __launch_bounds__(kTCBlock, 2) k_gemm_tc(const __grid_constant__
     const int64_t row = (int64_t)tile * kTCRows + r;
     const bool row_ok = tid < kTCDecoders && row < A.N;
 
-    if (tid < kTCRows) {  // row tid of the constant slice: chunk 0 (k 0 .. 7) and chunk 1 (k 8 .. 15)
-        const uint32_t c = KIND ? 0x8480u : 0x8400u;  // bf16 -4 * 2^-120 / -2 * 2^-120
-        uint8_t* rowa = aconst + (tid >> 3) * 256 + (tid & 7) * 16;
-        *reinterpret_cast<uint4*>(rowa) = make_uint4(c | (c << 16), c, 0u, 0u);
-        *reinterpret_cast<uint4*>(rowa + 128) = make_uint4(0u, 0u, 0u, 0u);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // read by the tensor cores
-    }
     if (tid == 0) {
         for (int s = 0; s < kTCStages; ++s) mbar_init(&bar_full[s], 1);
         for (int b = 0; b < 2; ++b) {
@@ -527,8 +392,6 @@ __global__ void __launch_bounds__(kTCBlock, 2) k_gemm_tc(const __grid_constant__
 #pragma unroll
             for (int j = 0; j < 8; ++j)  // K slice j: 8 TMEM columns of A, 256 bytes (16 descriptor units) of B
                 mma_ts_warp(dcol, acol + 8u * j, bdesc + 16u * j, kIdesc, j > 0 ? 1u : 0u);
-            // correction slice: constant A (shared memory) x chunks 16, 17 of B
-            mma_ss_warp(dcol, kmajor_desc(smem_addr(aconst), 256), bdesc + 16u * 8, kIdesc);
             mma_commit_warp(&bar_mma[b]);
             committed = i + 1;
             // the next stage to fill, (i + kTCStages - 1) % kTCStages, last held group i - 1
@@ -581,9 +444,8 @@ __global__ void __launch_bounds__(kTCBlock, 2) k_gemm_tc(const __grid_constant__
                 }
                 tc_fence_after();
                 const uint8_t* st = smem + sp * SB;
-                // D = 2^-S (sum u x - offset sum x): one factor s * 2^S per row and group
-                const float f = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + GB + 2 * r)) *
-                                *reinterpret_cast<const float*>(st + NP * 288);
+                // D = sum c x: one factor, the group scale s, per row and group
+                const float f = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(st + GB + 2 * r));
                 float d[NH];
                 tmem_ld_cols<NH>(tmem + lane_base + 128u + (uint32_t)(bp * NP + h * NH), d);
 #pragma unroll
@@ -669,7 +531,7 @@ size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 size_t tc_smem_bytes(int np) {
     return std::max(kTCMinSmem, (size_t)kTCStages * (tc_group_bytes(np) + 256) +
-                                    (size_t)kTCWStages * kTCDecoders * kTCWStride + 4096 + 1024);
+                                    (size_t)kTCWStages * kTCDecoders * kTCWStride + 1024);
 }
 
 template <int NP, int KIND>

@@ -140,6 +140,28 @@ def activations(K: int, seed: int, device="cpu", M: int | None = None) -> torch.
     return torch.randn(shape, generator=_gen(seed + 7, device), device=device).to(torch.bfloat16)
 
 
+def outlier_activations(K: int, seed: int, magnitudes=(2.0 ** 10, 2.0 ** 12, 2.0 ** 14), device="cpu",
+                        M: int | None = None) -> torch.Tensor:
+    """bf16 x ~ N(0, 1) with one outlier channel per 128-group: a position
+    drawn uniformly inside the group, set to +-m with m drawn from
+    `magnitudes` and a random sign (the few very large activation channels
+    of decoder layers).  Shape [K], or [M][K] when M is given (the outlier
+    channels are shared by the rows, as a channel is)."""
+    g = _gen(seed + 11, device)
+    shape = (K,) if M is None else (M, K)
+    x = torch.randn(shape, generator=g, device=device)
+    G = K // 128
+    pos = torch.randint(0, 128, (G,), generator=g, device=device) + 128 * torch.arange(G, device=device)
+    mag = torch.tensor(magnitudes, dtype=torch.float32, device=device)[
+        torch.randint(0, len(magnitudes), (G,), generator=g, device=device)]
+    sign = torch.randint(0, 2, (G,), generator=g, device=device).float() * 2 - 1
+    if M is None:
+        x[pos] = mag * sign
+    else:
+        x[:, pos] = (mag * sign).unsqueeze(0) * (1 + torch.rand((M, G), generator=g, device=device))
+    return x.to(torch.bfloat16)
+
+
 def gaussian_weights(N: int, K: int, seed: int, std: float = 0.02, device="cpu", dtype=torch.float32):
     """W ~ N(0, std^2), [N][K], returned in `dtype` (fp32 or bf16)."""
     w = torch.randn((N, K), generator=_gen(seed, device), device=device, dtype=torch.float32)

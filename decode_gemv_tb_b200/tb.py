@@ -20,9 +20,11 @@ TERNARY_B3 = 3  # the ternary grid, 5 codes per byte
 F32, BF16 = 0, 1
 MAX_LAYER_ITEMS = 16
 FLAG_OVERLAP_PREVIOUS = 1
+FLAG_TEST_STALL = 0x80000000  # test hook: the batch-1 kernel's waits give up (see include/tb.h)
 NOALLOC_SCRATCH_BYTES = 4 << 20  # TB_NOALLOC_SCRATCH_BYTES
 
-STATUS = {0: "TB_OK", 1: "TB_ERR_ARG", 2: "TB_ERR_SHAPE", 3: "TB_ERR_ALIGN", 4: "TB_ERR_UNSUPPORTED", 5: "TB_ERR_CUDA"}
+STATUS = {0: "TB_OK", 1: "TB_ERR_ARG", 2: "TB_ERR_SHAPE", 3: "TB_ERR_ALIGN", 4: "TB_ERR_UNSUPPORTED", 5: "TB_ERR_CUDA",
+          6: "TB_ERR_TIMEOUT"}
 
 # every entry point the header declares: (name, restype, argtypes)
 _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -41,6 +43,9 @@ SIGNATURES = {
     "tb_layer_gemv": (_I32, [_P, _I32, ctypes.c_uint, _P, _SZ, _P]),
     "tb_gemv_noalloc": (_I32, [_P, _I32, _P, _P, _P, _I32, _I64, _I64, _P]),
     "tb_wait_timeouts": (ctypes.c_uint, []),
+    "tb_sync_status": (_I32, [_P]),
+    "tb_gate_up_workspace_bytes": (_SZ, [_P, _P]),
+    "tb_gate_up_silu": (_I32, [_P, _P, _P, ctypes.c_uint, _P, _SZ, _P]),
 }
 
 
@@ -117,6 +122,13 @@ def _bits(t: torch.Tensor, name: str) -> int:
 def wait_timeouts() -> int:
     """Bounded device waits that gave up since the last call (synchronizes)."""
     return int(load().tb_wait_timeouts())
+
+
+def sync_status(stream: int | None = None) -> int:
+    """tb_sync_status on the current stream: 0 (TB_OK), 6 (TB_ERR_TIMEOUT) or 5."""
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return int(load().tb_sync_status(stream))
 
 
 def version() -> int:
@@ -225,3 +237,21 @@ def tb_layer_gemv(items, ws: torch.Tensor | None = None, flags: int = 0, stream:
         ws = workspace(layer_workspace_bytes(arr), torch.device("cuda", torch.cuda.current_device()))
     _check(load().tb_layer_gemv(ctypes.cast(arr, ctypes.c_void_p), len(arr), flags, ws.data_ptr(), ws.numel(),
                                 stream), "tb_layer_gemv")
+
+
+def tb_gate_up_silu(gate, up, h: torch.Tensor, ws: torch.Tensor | None = None, flags: int = 0,
+                    stream: int | None = None) -> torch.Tensor:
+    """gate, up: (packed, grid, scales, x, y, N, K) of equal N and K; writes
+    their y and h = bf16(silu(gate) * up) ([N] bf16)."""
+    arr = linear_items([gate, up])
+    if h.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TBError("h must hold bf16")
+    g_ptr = ctypes.cast(ctypes.byref(arr, 0), ctypes.c_void_p)
+    u_ptr = ctypes.cast(ctypes.byref(arr, ctypes.sizeof(Linear)), ctypes.c_void_p)
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    if ws is None:
+        ws = workspace(load().tb_gate_up_workspace_bytes(g_ptr, u_ptr), torch.device("cuda", torch.cuda.current_device()))
+    _check(load().tb_gate_up_silu(g_ptr, u_ptr, _dev(h, "h"), flags, ws.data_ptr(), ws.numel(), stream),
+           "tb_gate_up_silu")
+    return h

@@ -62,12 +62,19 @@
  *   positive finite number gives code 0; every such weight is counted.
  *
  * PRODUCTS
- *   y[n] = sum_k x[k] * c[n][k] * s[n][k/128], accumulated in fp32 per
- *   128-group and scaled once per group; fp32 output, or bf16 rounded half
- *   to even from the fp32 result.  Error bound: |y - y_exact| <= 1e-5 *
- *   sum_k |x[k] c[n][k] s[n][k/128]| (plus 4e-3 |y| for bf16 outputs).
- *   Results are bitwise deterministic from run to run (no atomics in any
- *   reduction).
+ *   y[n] = sum_k x[k] * c[n][k] * s[n][k/128], every product x * c formed
+ *   exactly from the signed codeword (a zero codeword contributes nothing),
+ *   summed per 128-group, scaled once per group, accumulated in fp32; fp32
+ *   output, or bf16 rounded half to even from the fp32 result.  Error
+ *   bound: |y - y_exact| <= 1e-5 * sum_k |x[k] c[n][k] s[n][k/128]| (plus
+ *   4e-3 |y| for bf16 outputs).  Results are bitwise deterministic from run
+ *   to run (no atomics in any reduction).
+ *   ACTIVATION RANGE: x must be finite with |x| < 2^120.  The batch-1
+ *   products (M = 1) form each group's sum in integers on a fixed-point
+ *   grid 2^55 below the group's largest |x|: an activation more than 2^42
+ *   below its group's largest one loses its low bits, by less than 2^-48
+ *   of that largest |x| each (the bound above holds whenever such tiny
+ *   activations are not the group's only ones meeting nonzero codes).
  *
  * ------------------------------------------------------------------------
  * CONVENTIONS
@@ -77,8 +84,9 @@
  *     nothing and keeps no allocation between calls.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All calls
  *     are asynchronous on `stream`; none synchronizes.
- *   - Alignment: packed, W, x / X rows: 16 bytes; scales: 2 bytes; y / Y:
- *     4 bytes (fp32) or 2 bytes (bf16).
+ *   - Alignment: packed, W, x / X rows: 16 bytes; scales: 16 bytes for the
+ *     products (they are read by tensor copies), 2 bytes for
+ *     tb_scales_absmax and tb_pack; y / Y: 4 bytes (fp32) or 2 bytes (bf16).
  *   - Argument errors are reported before anything is launched; a launch
  *     failure is reported as TB_ERR_CUDA (cudaGetLastError is consumed).
  *   - Outputs must not overlap inputs.
@@ -116,7 +124,8 @@ typedef enum {
     TB_ERR_SHAPE = 2,       /* N < 1, K < 128, K % 128 != 0, M outside 1..65536, ld too small */
     TB_ERR_ALIGN = 3,       /* a pointer or leading dimension breaks the alignment rules */
     TB_ERR_UNSUPPORTED = 4, /* valid request this build does not implement */
-    TB_ERR_CUDA = 5         /* a CUDA call or launch failed */
+    TB_ERR_CUDA = 5,        /* a CUDA call or launch failed */
+    TB_ERR_TIMEOUT = 6      /* a bounded device-side wait gave up (tb_sync_status only) */
 } tb_status_t;
 
 /* Library version as 10000*major + 100*minor + patch. */
@@ -152,27 +161,41 @@ TB_API tb_status_t tb_scales_absmax(const void *W, tb_dtype_t w_dtype, int64_t N
 TB_API tb_status_t tb_pack(const void *W, tb_dtype_t w_dtype, int64_t N, int64_t K, tb_grid_t grid,
                     const uint16_t *scales, void *packed, int32_t *bad_count, tb_stream_t stream);
 
-/* Inverse of the bit layout: codes[n][k] = c (int8), device, [N][K]. */
+/* Inverse of the bit layout: codes[n][k] = c (int8), device, [N][K] -- the
+ * integer codewords of the format (ThinkBit page, 어떻게 동작하나: w = c * s,
+ * c on the layer's grid), for inspection and tests.
+ *   packed  as produced by tb_pack, 16-byte aligned.
+ *   codes   [N][K] int8, device, 16-byte aligned, fully written. */
 TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int64_t K, int8_t *codes,
                       tb_stream_t stream);
 
-/* Scratch ("workspace") of the products below.  Each call first writes a
- * prepared copy of its activations (bf16, K per activation row, scaled by
- * powers of two) and per-128-group sums into the workspace, then reads them
- * (the single-launch row kernel behind small tb_gemv calls uses none of it);
- * the calls also keep per-tile arrival counters and partial sums there
- * (tiles whose K range is split are combined in a fixed order).  For M = 1
- * the size is ceil256(K/128 * 272) + ceil256(4 * ceil(N/32))
- * + ceil256(256 * min(8192, ceil(N/32) * ceil(K/256))).  For
- * M >= 32 (the tensor-core path) the size is exact and device independent:
- *   ceil256(K/128 * (NP * 288 + 16)) + ceil256(T * K/128 * 256) + ceil256(4 * T)
- *     + [S > 1] ceil256(T * S * NP * 512)
- * with NP = M rounded up to 16, T = ceil(N / 128) and S = the K split,
- * max(1, min(floor((296 + T/2) / T), 16, K / 128)).  For M > 64 it is the
- * larger of the sizes for 64 and for M mod 64 (when not 0).
+/* Scratch ("workspace") of the products below, by path:
+ *   M = 1 (tb_gemv above 2^24 weights, tb_layer_gemv): per call, one
+ *     1088-byte activation record per 128-group of x (written by the call's
+ *     preparation kernel, then read), a copy of the scales with rows padded
+ *     to a multiple of 8 groups when K/128 is not one, eight arrival
+ *     counters per 256-row tile and two 256-float partial-sum slots per CTA
+ *     (tiles whose K range is split between CTAs are combined in a fixed
+ *     order).  Size, device independent:
+ *       ceil256(G * 1088) + [G % 8 != 0] ceil256(N * ceil8(G) * 2)
+ *         + ceil256(32 * T1) + ceil256(2048 * min(256, T1 * ceil(G / 2)))
+ *     with G = K/128 and T1 = ceil(N / 256).  (The row kernel behind small
+ *     tb_gemv calls uses none of it.)
+ *   2 <= M < 32: none (the kernel reads X as it is); the size is reported
+ *     as 256.
+ *   M >= 32 (the tensor-core path): X copied per group into the MMA's
+ *     layout, the scales transposed per 128-row tile, a counter per tile and
+ *     the K-split partial sums:
+ *       ceil256(G * NP * 256) + ceil256(T * G * 256) + ceil256(4 * T)
+ *         + [S > 1] ceil256(T * S * NP * 512)
+ *     with NP = M rounded up to 16, T = ceil(N / 128) and S = the K split,
+ *     max(1, min(floor((296 + T/2) / T), 16, G)).
+ *   M > 64: the larger of the sizes for 64 and for M mod 64 (when not 0).
+ * The workspace is
  *   - device memory, 256-byte aligned, at least the size returned here;
  *   - owned by the caller, written by every call: two calls that share a
- *     workspace must be ordered (e.g. the same stream);
+ *     workspace must be ordered (e.g. the same stream); every call clears
+ *     what must start at zero;
  *   - no other state is kept between calls.
  * Returns 0 for bad arguments. */
 TB_API size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K); /* tb_gemv: M = 1; tb_gemm: its M */
@@ -188,23 +211,23 @@ TB_API size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K); /* tb_gemv: M
  * TB_GRID_TERNARY_B3 product, run a single-launch kernel with one warp per
  * output row that stages x in shared memory and uses no workspace (for
  * TB_GRID_TERNARY_B3, K <= 57600, else TB_ERR_UNSUPPORTED).  Larger ones
- * run the stream-K kernel of tb_layer_gemv.  Both meet the error bound
- * above; the same product through tb_gemv and tb_layer_gemv may differ in
- * rounding. */
+ * run the integer tensor-path kernel of tb_layer_gemv.  Both meet the
+ * error bound above; the same product through tb_gemv and tb_layer_gemv
+ * may differ in rounding. */
 TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *x, void *y,
                            tb_dtype_t y_dtype, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
                            tb_stream_t stream);
 
-/* Small-batch GEMM Y = X W^T, 1 <= M <= 64 (M = 1 as tb_gemv;
- * TB_GRID_TERNARY_B3: one GEMV launch per batch row, K <= 57600).
- * Prefill batches, 64 < M <= 65536, run as consecutive blocks of 64 batch
- * rows (the last one the remainder), each like a call with that M, in
- * stream order: the weights are decoded once per block.
+/* Small-batch GEMM Y = X W^T, 1 <= M <= 64 (ThinkBit page, 무엇인가: the
+ * weights are read once for all M activation rows; 어떻게 동작하나: w = c * s,
+ * so every row is the GEMV above on its own activations).  M = 1 runs as
+ * tb_gemv; 2 <= M < 32 on mma.sync, from M = 32 on the tcgen05 tensor cores,
+ * both with the codewords decoded exactly to bf16; TB_GRID_TERNARY_B3: one
+ * GEMV launch per batch row, K <= 57600.  Prefill batches, 64 < M <= 65536,
+ * run as consecutive blocks of 64 batch rows (the last one the remainder),
+ * each like a call with that M, in stream order: the weights are decoded
+ * once per block.
  *   X          [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device; finite, |x| < 2^120.
- *              From M = 32 the activations of one 128-group share one
- *              power-of-two exponent over all M rows: an element more than
- *              about 2^110 below the group's largest |X[.][k]| over the batch
- *              may count as zero.
  *   Y          [M][ldy] fp32 or bf16, ldy >= N, device; Y[m][n] for n < N written.
  *   workspace  tb_workspace_bytes(M, N, K) bytes. */
 TB_API tb_status_t tb_gemm(const void *packed, tb_grid_t grid, const uint16_t *scales, const uint16_t *X,
@@ -212,12 +235,21 @@ TB_API tb_status_t tb_gemm(const void *packed, tb_grid_t grid, const uint16_t *s
                            void *workspace, size_t workspace_bytes, tb_stream_t stream);
 
 /* Diagnostic: how many bounded device-side waits gave up since the last
- * call, on the current device (the count is then cleared).  The kernels
- * that wait on the tensor-core pipeline give up after about two seconds,
- * write NaN to their outputs and return; a nonzero count means such a
- * launch produced no result.  Synchronizes with the device; returns
- * 0xFFFFFFFF if the count cannot be read. */
+ * call, on the current device (the count is then cleared).  Every kernel
+ * that waits on a copy or on the tensor-core pipeline gives up after about
+ * two seconds, writes NaN to the outputs it has not finished and returns;
+ * a nonzero count means such a launch produced no result.  Synchronizes
+ * with the device; returns 0xFFFFFFFF if the count cannot be read. */
 TB_API unsigned int tb_wait_timeouts(void);
+
+/* Status of the work issued so far.  Every call above returns as soon as
+ * its kernels are queued, so a wait that gives up on the device (a copy
+ * that never lands, a tensor-core hand-off that never completes) can only
+ * be reported afterwards: this call synchronizes `stream`, then returns
+ * TB_ERR_TIMEOUT if any bounded wait on the current device gave up since
+ * the last check (and clears the count), TB_ERR_CUDA if the stream or the
+ * count reports a CUDA error, TB_OK otherwise. */
+TB_API tb_status_t tb_sync_status(tb_stream_t stream);
 
 /* One linear layer of a grouped launch. */
 typedef struct {
@@ -240,7 +272,15 @@ typedef struct {
  * this call (true for resident model weights during decode). */
 #define TB_FLAG_OVERLAP_PREVIOUS 1u
 
-/* Workspace bytes of tb_layer_gemv for these items (0 for bad arguments). */
+/* Test hook for the failure path of the batch-1 kernel: its copies are
+ * never issued, every bounded wait gives up after about 10 ms instead of
+ * 2 s, the outputs of the call are NaN, and the next tb_sync_status
+ * returns TB_ERR_TIMEOUT.  Nothing faults and the context stays usable. */
+#define TB_FLAG_TEST_STALL 0x80000000u
+
+/* Workspace bytes of tb_layer_gemv for these items (0 for bad arguments):
+ * the batch-1 size above summed over the items, with the counters and
+ * partial-sum slots counted once for all of them. */
 TB_API size_t tb_layer_workspace_bytes(const tb_linear_t *items, int n_items);
 
 /* Mixed-grid grouped GEMV: every item is an independent y = W x with its
@@ -258,6 +298,30 @@ TB_API size_t tb_layer_workspace_bytes(const tb_linear_t *items, int n_items);
 TB_API tb_status_t tb_layer_gemv(const tb_linear_t *items, int n_items, unsigned flags, void *workspace,
                                  size_t workspace_bytes, tb_stream_t stream);
 
+/* Workspace bytes of tb_gate_up_silu: tb_layer_workspace_bytes of the two
+ * items, plus ceil256(8 N) + ceil256(32 ceil(N / 256)) for the pair (0 for
+ * bad arguments). */
+TB_API size_t tb_gate_up_workspace_bytes(const tb_linear_t *gate, const tb_linear_t *up);
+
+/* The gate and up projections of a decoder layer's MLP in one launch, and
+ * the down projection's input from them:
+ *     gate->y = W_gate x,  up->y = W_up x,  h[n] = bf16(silu(gate[n]) * up[n]),
+ *     silu(g) = g / (1 + e^-g),
+ * (ThinkBit page, 무엇인가: decoding a token runs every projection of every
+ * layer; the SiLU-gated MLP is that of the Qwen3 layers the page quantizes).
+ * The two products are those of tb_layer_gemv (same kernel, same bound);
+ * h is formed in fp32 from the fp32 results and rounded half to even.
+ *   gate, up   HOST descriptors of equal N and K, each on its own grid (not
+ *              TB_GRID_TERNARY_B3); x is normally the same buffer, and then
+ *              its activation records are prepared once for both when the
+ *              grids have the same code width; y of each is written as for
+ *              tb_layer_gemv.
+ *   h          [N] bf16, device, written.
+ *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS.
+ *   workspace  tb_gate_up_workspace_bytes(gate, up) bytes. */
+TB_API tb_status_t tb_gate_up_silu(const tb_linear_t *gate, const tb_linear_t *up, uint16_t *h, unsigned flags,
+                                   void *workspace, size_t workspace_bytes, tb_stream_t stream);
+
 /* Size of the fixed device scratch behind tb_gemv_noalloc (4 MiB). */
 #define TB_NOALLOC_SCRATCH_BYTES (4u << 20)
 
@@ -273,12 +337,18 @@ TB_API tb_status_t tb_layer_gemv(const tb_linear_t *items, int n_items, unsigned
  *            TB_NOALLOC_SCRATCH_BYTES per device, inside this library.  A
  *            problem whose tb_workspace_bytes(1, N, K) exceeds that size is
  *            rejected with TB_ERR_UNSUPPORTED before any CUDA call (every
- *            N <= 2^20 with K <= 2^19 fits).  Nothing has to be cleared by
- *            the caller: the call itself zeroes what must start at zero.
+ *            N <= 2^20 with K <= 2^18 and K a multiple of 1024 fits; other
+ *            K also stage a padded copy of the scales, N * ceil8(K/128) * 2
+ *            bytes).  Nothing has to be cleared by the caller: the call
+ *            itself zeroes what must start at zero.
  *   setup    the first call on each device (with that device current) looks
  *            up the array's address with cudaGetSymbolAddress and caches it;
  *            make that first call before any stream capture.  A failed
  *            lookup returns TB_ERR_CUDA and is retried on the next call.
+ *            The cached address belongs to the device's current context: a
+ *            cudaDeviceReset (or any other end of that context) makes it
+ *            stale, so do not call this entry point again in the same
+ *            process after resetting the device.
  *   sharing  every call on a device uses the same array: calls on one stream
  *            are ordered and safe; calls that can overlap (other streams,
  *            other host threads) race and give wrong results -- use tb_gemv

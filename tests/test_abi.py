@@ -57,7 +57,7 @@ def test_sizes_closed_form(lib):
             assert 8 * (tb.packed_bytes(grid, N, K) + tb.scale_bytes(N, K)) == N * K * (bits + 0.125)
     assert tb.packed_bytes(1, 4, 100) == 0 and tb.packed_bytes(7, 4, 128) == 0 and tb.scale_bytes(0, 128) == 0
     assert lib.tb_version() >= 100
-    for s in range(6):
+    for s in range(7):
         assert lib.tb_status_string(s)
 
 
@@ -66,38 +66,37 @@ FAKE = 1 << 40  # a 256-byte-aligned address that is never dereferenced
 
 def test_workspace_sizes(lib):
     al = lambda b: (b + 255) // 256 * 256
-    for M, N, K in ((4, 100, 5120), (16, 17408, 17408), (17, 7, 1024)):
-        # M below the tensor-core threshold (32): prepared activations (2 bytes per element) + per-group
-        # pairs (8 bytes) of up to 16 batch rows, each 256-byte aligned
-        Mb = min(M, 16)
-        assert tb.workspace_bytes(M, N, K) == al(2 * Mb * K) + al(8 * Mb * (K // 128))
+    for M, N, K in ((2, 100, 5120), (4, 100, 5120), (16, 17408, 17408), (17, 7, 1024), (31, 64, 128)):
+        # below the tensor-core threshold (32) the kernel reads X as it is: no workspace, a nominal 256
+        assert tb.workspace_bytes(M, N, K) == 256
     for M, N, K in ((32, 100, 5120), (33, 17408, 5120), (64, 7, 1024), (64, 40000, 4096)):
-        # tensor-core path: per group NP rows of prepared X and correction slice (288 bytes) and the
-        # group exponent (16 bytes), NP = M rounded up to 16; the scales transposed per 128-row tile;
-        # a counter per tile; K-split partials of NP x 128 fp32 per tile and split
+        # tensor-core path: per group NP rows of X (256 bytes each) in the MMA's layout, NP = M rounded
+        # up to 16; the scales transposed per 128-row tile; a counter per tile; K-split partials of
+        # NP x 128 fp32 per tile and split
         NP, tiles, G = (M + 15) // 16 * 16, (N + 127) // 128, K // 128
         splits = max(1, min((296 + tiles // 2) // tiles, 16, G))
-        want = (al(G * (NP * 288 + 16)) + al(tiles * G * 128 * 2) + al(4 * tiles) +
+        want = (al(G * NP * 256) + al(tiles * G * 128 * 2) + al(4 * tiles) +
                 (al(tiles * splits * NP * 128 * 4) if splits > 1 else 0))
         assert tb.workspace_bytes(M, N, K) == want, (M, N, K)
-    for N, K in ((1, 128), (256, 1024), (17408, 5120), (100, 1408)):
-        # batch 1: one 272-byte record per 128-group of x, a counter per 32-row tile and two 32-float
-        # slots per warp (at most one warp per chunk of two groups, the smaller chunk)
-        tiles = (N + 31) // 32
-        warps = min(8192, tiles * ((K // 128 + 1) // 2))
-        assert tb.workspace_bytes(1, N, K) == al(272 * (K // 128)) + al(4 * tiles) + al(256 * warps)
+    for N, K in ((1, 128), (256, 1024), (17408, 5120), (100, 1408), (4096, 12288)):
+        # batch 1: one 1088-byte record per 128-group of x, a copy of the scales with rows padded to 8
+        # groups when K/128 is not a multiple of 8, eight counters per 256-row tile, and two 256-float
+        # partial slots per CTA (at most 256 CTAs, at most one per chunk of two groups)
+        G, tiles = K // 128, (N + 255) // 256
+        spad = al(N * -(-G // 8) * 8 * 2) if G % 8 else 0
+        ctas = min(256, tiles * -(-G // 2))
+        assert tb.workspace_bytes(1, N, K) == al(1088 * G) + spad + al(32 * tiles) + al(2048 * ctas)
     assert tb.workspace_bytes(0, 8, 128) == 0 and tb.workspace_bytes(1, 8, 100) == 0
     assert tb.workspace_bytes(65537, 8, 128) == 0 and tb.workspace_bytes(1, 0, 128) == 0
     items = (tb.Linear * 3)()
     shapes = ((4096, 4096, 2), (1024, 4096, 1), (4096, 12288, 0))  # (N, K, grid)
     for i, (N, K, grid) in enumerate(shapes):
         items[i] = tb.Linear(FAKE, FAKE, FAKE, FAKE, N, K, grid, 0)
-    tiles = sum((N + 31) // 32 for N, _, _ in shapes)
-    # chunks of two 3-bit groups or four 2-bit groups per 32-row tile
-    chunks = sum((N + 31) // 32 * -(-(K // 128) // (2 if grid == 2 else 4)) for N, K, grid in shapes)
-    per = sum(al(272 * (K // 128)) for _, K, _ in shapes)
-    assert tb.layer_workspace_bytes(items) == per + al(4 * tiles) + al(256 * min(8192, chunks))
-
+    tiles = sum((N + 255) // 256 for N, _, _ in shapes)
+    # chunks of two 3-bit groups or four 2-bit groups per 256-row tile
+    chunks = sum((N + 255) // 256 * -(-(K // 128) // (2 if grid == 2 else 4)) for N, K, grid in shapes)
+    per = sum(al(1088 * (K // 128)) for _, K, _ in shapes)
+    assert tb.layer_workspace_bytes(items) == per + al(32 * tiles) + al(2048 * min(256, chunks))
 
 def test_argument_errors_before_launch(lib):
     A = FAKE
@@ -126,6 +125,7 @@ def test_argument_errors_before_launch(lib):
     # alignment -> TB_ERR_ALIGN (3)
     assert lib.tb_gemv(A + 8, 1, A, A, A, 0, 16, 128, A, W, 0) == 3
     assert lib.tb_gemv(A, 1, A + 1, A, A, 0, 16, 128, A, W, 0) == 3
+    assert lib.tb_gemv(A, 1, A + 8, A, A, 0, 16, 128, A, W, 0) == 3  # scales: 16 bytes
     assert lib.tb_gemv(A, 1, A, A + 2, A, 0, 16, 128, A, W, 0) == 3
     assert lib.tb_gemv(A, 1, A, A, A + 2, 0, 16, 128, A, W, 0) == 3
     assert lib.tb_gemv(A, 1, A, A, A, 0, 16, 128, A + 16, W, 0) == 3
@@ -188,3 +188,32 @@ def test_binding_fails_loudly_without_library(tmp_path):
             tb.load(str(tmp_path / "missing.so"))
     finally:
         tb._lib = saved
+
+
+def test_gate_up_workspace_and_errors(lib):
+    """tb_gate_up_silu: the layer workspace of its two items plus the pair's
+    fp32 values (8 N bytes) and counters (32 per 256-row tile); shape and
+    argument errors before any launch."""
+    al = lambda b: (b + 255) // 256 * 256
+    A, W = FAKE, 1 << 30
+    for (N, K, gg, gu) in ((12288, 4096, 2, 0), (17408, 5120, 1, 1), (300, 640, 0, 2)):
+        two = (tb.Linear * 2)()
+        two[0] = tb.Linear(A, A, A, A, N, K, gg, 0)
+        two[1] = tb.Linear(A, A, A, A, N, K, gu, 0)
+        g = ctypes.cast(ctypes.byref(two, 0), ctypes.c_void_p)
+        u = ctypes.cast(ctypes.byref(two, ctypes.sizeof(tb.Linear)), ctypes.c_void_p)
+        want = tb.layer_workspace_bytes(two) + al(8 * N) + al(32 * ((N + 255) // 256))
+        assert lib.tb_gate_up_workspace_bytes(g, u) == want
+    two = (tb.Linear * 2)()
+    two[0] = tb.Linear(A, A, A, A, 64, 1024, 1, 0)
+    two[1] = tb.Linear(A, A, A, A, 32, 1024, 1, 0)
+    g = ctypes.cast(ctypes.byref(two, 0), ctypes.c_void_p)
+    u = ctypes.cast(ctypes.byref(two, ctypes.sizeof(tb.Linear)), ctypes.c_void_p)
+    assert lib.tb_gate_up_workspace_bytes(g, u) == 0                 # N differs
+    assert lib.tb_gate_up_silu(g, u, A, 0, A, W, 0) == 2               # TB_ERR_SHAPE
+    two[1].N = 64
+    assert lib.tb_gate_up_silu(g, u, 0, 0, A, W, 0) == 1               # h missing
+    assert lib.tb_gate_up_silu(g, u, A, 2, A, W, 0) == 1               # unknown flag
+    assert lib.tb_gate_up_silu(g, u, A + 1, 0, A, W, 0) == 3           # h misaligned
+    two[1].grid = 3
+    assert lib.tb_gate_up_silu(g, u, A, 0, A, W, 0) == 4               # 5-trit layout: not in the pair

@@ -2,10 +2,13 @@
 
 Collected last on purpose, so that it runs both after every other test and,
 when selected alone, in a fresh process.  The GPU case calls the entry point
-twice in a row (a large problem, then a small one that reuses the same
-scratch without any clearing in between) and compares each output with
-tb_gemv's on the same inputs and with the oracle, within the GEMV
-tolerance |dy| <= 1e-5 sum_k |x_k w_k| (+ 4e-3 |y| for bf16 outputs)."""
+twice in a row, both times on the kernel that uses the scratch (products
+above 2^24 weights): a 3-bit gate projection, then a 2-bit problem with a
+different tile count and K split, whose K/128 = 36 also makes the call
+stage padded scales in the scratch; the second call reuses the scratch
+without any clearing in between.  Each output is compared with tb_gemv's
+on the same inputs and with the oracle, within the GEMV tolerance
+|dy| <= 1e-5 sum_k |x_k w_k| (+ 4e-3 |y| for bf16 outputs)."""
 import os
 import re
 
@@ -20,6 +23,7 @@ from tests.helpers import assert_within, u16, w_np
 HEADER = os.path.join(os.path.dirname(__file__), "..", "include", "tb.h")
 FAKE = 1 << 40  # a 256-byte-aligned address that is never dereferenced
 TB_ERR_ARG, TB_ERR_ALIGN, TB_ERR_UNSUPPORTED = 1, 3, 4
+ROW_KERNEL_MAX_WEIGHTS = 1 << 24  # tb_gemv runs the row kernel (no scratch) up to this many weights
 
 
 def needs_scratch(N, K):
@@ -40,7 +44,7 @@ def test_rejections_before_any_cuda_call():
     f = lib.tb_gemv_noalloc
     # the envelope the header states fits; one K step past the limit for a
     # large N does not
-    assert needs_scratch(1 << 20, 1 << 19) <= tb.NOALLOC_SCRATCH_BYTES
+    assert needs_scratch(1 << 20, 1 << 18) <= tb.NOALLOC_SCRATCH_BYTES
     K_big = 1 << 21
     assert needs_scratch(4096, K_big) > tb.NOALLOC_SCRATCH_BYTES
     assert f(FAKE, tb.INT2, FAKE, FAKE, FAKE, tb.F32, 4096, K_big, None) == TB_ERR_UNSUPPORTED
@@ -61,11 +65,12 @@ def test_two_calls_in_a_row_match_tb_gemv(oracle):
         pytest.skip("no CUDA device")
     dev = "cuda:0"
     # a gate projection of an 8B decoder layer (3-bit, fp32 out), then a
-    # small ragged 2-bit problem (bf16 out) that reuses the same scratch
-    cases = [(tb.INT3, 12288, 4096, torch.float32, 11), (tb.INT2, 1000, 1408, torch.bfloat16, 12)]
+    # 2-bit problem (bf16 out) with 16 tiles instead of 48 that reuses the same scratch
+    cases = [(tb.INT3, 12288, 4096, torch.float32, 11), (tb.INT2, 4096, 4608, torch.bfloat16, 12)]
     prepared = []
     for grid, N, K, odt, seed in cases:
         assert needs_scratch(N, K) <= tb.NOALLOC_SCRATCH_BYTES
+        assert N * K > ROW_KERNEL_MAX_WEIGHTS  # the scratch-using kernel, not the row kernel
         W = synth.gaussian_weights(N, K, seed=seed)
         x = synth.activations(K, seed=seed)
         s_ref = oracle.scales_absmax(w_np(W), grid)
