@@ -48,12 +48,16 @@ def algo_bytes(N, K, grid, M=1, ybytes=4):
     return codes + N * (K // 128) * 2 + M * K * 2 + M * N * ybytes
 
 
+TRAFFIC_RECORD = os.path.join("profiles", "k_gemv8_traffic.json")
+
+
 def traffic_per_launch(algorithmic_bytes):
-    """DRAM bytes per k_gemv_tma launch from the committed ncu capture: its
+    """DRAM bytes per k_gemv8 launch from the committed ncu capture: its
     measured traffic / algorithmic ratio times this launch's algorithmic
-    bytes; None when the kernel's sources changed after the capture."""
+    bytes; None when there is no capture or the kernel's sources changed
+    after it."""
     import hashlib
-    p = os.path.join(ROOT, "profiles", "k_gemv_tma_traffic.json")
+    p = os.path.join(ROOT, TRAFFIC_RECORD)
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -90,8 +94,9 @@ def measured_peaks():
 
 class Clocks:
     """SM clock and throttle reasons during the timed region: NVML polled
-    every 2 ms from a thread between begin() and end(), plus an nvidia-smi
-    log (100 ms) over the whole context for the record."""
+    back to back (about every 0.1 ms) from a thread between begin() and
+    end(), plus an nvidia-smi log (100 ms) over the whole context for the
+    record."""
 
     NAMES = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
@@ -140,7 +145,6 @@ class Clocks:
                         self.reasons.add(nm)
             except Exception:
                 pass
-            threading.Event().wait(0.002)
 
     def begin(self):
         if self.nvml:
@@ -165,7 +169,7 @@ class Clocks:
     def summary(self):
         if self.samples:
             return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                    "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml 2 ms"}
+                    "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml, back to back"}
         if not self.proc or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
         sm, mx, reasons = [], None, set()
@@ -465,6 +469,22 @@ def rows_section(dev, stream):
     return out
 
 
+def host_description():
+    """nproc, the CPU model and the oracle's compiler flags (the CPU
+    baseline's context)."""
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    from oracle import tb_oracle as oracle
+    return {"nproc": os.cpu_count(), "cpu_model": model, "oracle_cflags": " ".join(oracle.CFLAGS),
+            "threads_used": 1}
+
+
 def cpu_baseline(seconds_budget=20.0):
     """The oracle as it stands, single-threaded fp64, on a bounded sample of
     the same workload: GEMV of the stack's layer-0 projections (as many as
@@ -490,7 +510,8 @@ def cpu_baseline(seconds_budget=20.0):
             break
     return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"fp64 oracle GEMV over {'+'.join(names)} of the 36-layer stack "
-                      f"({done_bytes / 1e6:.1f} MB algorithmic), {t_total:.1f} s"}
+                      f"({done_bytes / 1e6:.1f} MB algorithmic), {t_total:.1f} s",
+            "host": host_description()}
 
 
 def run_reference(args):
@@ -530,7 +551,8 @@ def run_reference(args):
             "config": workload_config(synth.config3_stack(), 1),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": "each step: fp64 single-threaded oracle GEMV of layer-0 k and v (1024x4096, "
-                                       "2-bit) of this workload; value = their algorithmic bytes / time"},
+                                       "2-bit) of this workload; value = their algorithmic bytes / time",
+                             "host": host_description()},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -584,7 +606,7 @@ def main():
     ms_step = ms / args.steps
     value = job_throughput(world, S.step_bytes, ms_step)
     us_layer = ms_step * 1e3 / n_layers
-    # dominant kernel: the stream-K GEMV of each tb_layer_gemv call; its
+    # dominant kernel: the batch-1 GEMV (k_gemv8) of each tb_layer_gemv call; its
     # duration is taken as the whole call's (preparation kernel included),
     # averaged over the timed region, so `achieved` is a lower bound
     avg_layer_bytes = S.step_bytes / n_layers
@@ -595,7 +617,11 @@ def main():
     ms_ovl = time_region(g_ovl.replay, args.steps, args.warmup, cur, dist) / args.steps
     del g_ovl
 
-    # --- end to end through the public API: H2D of all x, launches, D2H of all y
+    # --- end to end through the public API: each step copies every layer's x
+    # from pinned host memory, makes the 36 tb_layer_gemv calls (ctypes, argument
+    # checks and tensor-map encoding on the host, every step), and copies every y
+    # back; eager (the headline) and captured in a CUDA graph (host work off the
+    # timeline, for comparison)
     x_host = torch.empty_like(S.x_all, device="cpu").pin_memory()
     x_host.copy_(S.x_all.cpu())
     y_host = torch.empty_like(S.y_all, device="cpu").pin_memory()
@@ -605,9 +631,11 @@ def main():
         S.step(0)
         y_host.copy_(S.y_all, non_blocking=True)
 
-    g_e2e = capture(e2e_step)
-    ms_e2e = time_region(g_e2e.replay, args.steps, args.warmup, cur, dist)
+    ms_e2e = time_region(e2e_step, args.steps, args.warmup, cur, dist)
     e2e_value = job_throughput(world, S.step_bytes, ms_e2e / args.steps)
+    g_e2e = capture(e2e_step)
+    ms_e2e_graph = time_region(g_e2e.replay, args.steps, args.warmup, cur, dist)
+    e2e_graph_value = job_throughput(world, S.step_bytes, ms_e2e_graph / args.steps)
     del g_e2e, g_step
 
     rows = None if args.no_rows else rows_section(dev, torch.cuda.current_stream(dev))
@@ -629,11 +657,14 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": profile_traffic,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
-                         else "fallback 6.65 TB/s", "kernel": "k_gemv_tma (per tb_layer_gemv call; duration includes its k_prep)"},
+                         else "fallback 6.65 TB/s", "kernel": "k_gemv8 (per tb_layer_gemv call; the duration includes its k_prep8, so achieved is a lower bound for k_gemv8 alone)"},
             "e2e": {"value": e2e_value, "unit": "GB/s",
-                    "h2d_bytes_per_step": S.x_all.numel() * 2, "d2h_bytes_per_step": S.y_all.numel() * 4},
+                    "h2d_bytes_per_step": S.x_all.numel() * 2, "d2h_bytes_per_step": S.y_all.numel() * 4,
+                    "ms_per_step": ms_e2e / args.steps, "calls": "eager: 36 tb_layer_gemv C-ABI calls per step",
+                    "graph_value": e2e_graph_value, "graph_ms_per_step": ms_e2e_graph / args.steps},
             "gpu_launches": 2 * n_layers * args.steps,
             "clocks": clocks,
+            "us_x_median_sm_ghz_per_layer": (us_layer * clocks["sm_mhz"] / 1e3) if clocks.get("sm_mhz") else None,
             "rows": rows,
         }
         if cpu:

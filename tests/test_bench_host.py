@@ -30,23 +30,33 @@ def test_algo_bytes_every_layout(bench, oracle):
 
 
 def test_traffic_figure_tracks_the_kernel_sources(bench, tmp_path, monkeypatch):
-    """The committed ratio is used while the hashed sources are unchanged,
-    and dropped (None) as soon as one of them differs."""
-    rec = json.load(open(os.path.join(ROOT, "profiles", "k_gemv_tma_traffic.json")))
-    assert bench.traffic_per_launch(1000.0) == pytest.approx(1000.0 * rec["traffic_over_algorithmic"])
-    # a copy of the tree's relevant files, one source changed by a byte
+    """A traffic record's ratio is used while the hashed sources are
+    unchanged, and dropped (None) as soon as one of them differs or the
+    record is missing."""
+    import hashlib
     fake = tmp_path / "root"
     (fake / "profiles").mkdir(parents=True)
-    shutil.copy(os.path.join(ROOT, "profiles", "k_gemv_tma_traffic.json"), fake / "profiles")
-    for s in rec["kernel_sources"]:
+    srcs = ["decode_gemv_tb_b200/csrc/tb_gemv8.cu", "decode_gemv_tb_b200/csrc/tb_partition.h"]
+    h = hashlib.sha256()
+    for s in srcs:
         dst = fake / s
         dst.parent.mkdir(parents=True, exist_ok=True)
         shutil.copy(os.path.join(ROOT, s), dst)
+        h.update(open(dst, "rb").read())
     monkeypatch.setattr(bench, "ROOT", str(fake))
-    assert bench.traffic_per_launch(1000.0) == pytest.approx(1000.0 * rec["traffic_over_algorithmic"])
-    with open(fake / rec["kernel_sources"][0], "a") as f:
+    assert bench.traffic_per_launch(1000.0) is None  # no record
+    rec = {"kernel": "k_gemv8", "traffic_over_algorithmic": 1.0125, "kernel_sources": srcs,
+           "kernel_sources_sha256": h.hexdigest()}
+    json.dump(rec, open(fake / bench.TRAFFIC_RECORD, "w"))
+    assert bench.traffic_per_launch(1000.0) == pytest.approx(1012.5)
+    with open(fake / srcs[0], "a") as f:
         f.write("\n")
     assert bench.traffic_per_launch(1000.0) is None
+    # the committed record, if any, names existing sources
+    committed = os.path.join(ROOT, bench.TRAFFIC_RECORD)
+    if os.path.exists(committed):
+        for s in json.load(open(committed))["kernel_sources"]:
+            assert os.path.exists(os.path.join(ROOT, s))
 
 
 def test_workload_config_names_the_stack(bench):
