@@ -9,6 +9,7 @@
 #include "../../include/tb.h"
 #include "tb_device.cuh"
 #include "tb_internal.h"
+#include "tb_partition.h"
 
 using namespace tb;
 
@@ -69,8 +70,8 @@ constexpr size_t kNoWorkspace = 256;
 constexpr int64_t kTCMinM = 32;
 
 // Batch-1 products of at most this many weights run the single-launch row
-// kernel (no preparation kernel, no split-tile combine), as do all products
-// in the 5-trits-per-byte layout; larger ones the stream-K TMA kernel.
+// kernel (no split-tile combine, no workspace), as do all products in the
+// 5-trits-per-byte layout; larger ones the integer tensor-path kernel.
 constexpr int64_t kRowWarpMaxWeights = (int64_t)1 << 24;
 
 // Batches above 64 rows (prefill) run as consecutive blocks of 64 rows, the
@@ -148,47 +149,68 @@ tb_status_t launch_items(Item* items, int n, int nt, cudaStream_t st) {
     return cuda_status(launch_linear(L, nt, (int)ctas, st));
 }
 
-// Batch-1 (M == 1) launch on the integer tensor path: preparation kernel +
-// k_gemv8 (tb_gemv8.cu).  Every item's activations become K/128 records;
-// the items' tiles of 256 rows are cut into chunks of 4 (2-bit container)
-// or 2 (3 bits) groups, numbered item by item, and split into equal-cost
-// contiguous ranges, one per CTA.  Scales are read by tensor copies, which
-// need 16-byte rows: when K/128 is not a multiple of 8 the preparation
-// kernel first copies them with rows padded to a multiple of 8 groups.
-constexpr int64_t kMaxG8Ctas = 256;      // bound of the CTA count (partial-sum slots)
+// Batch-1 (M == 1) launch on the integer tensor path: one kernel, k_gemv8
+// (tb_gemv8.cu).  The items' tiles of 256 rows are cut into chunks of 4
+// (2-bit container) or 2 (3 bits) groups, numbered item by item, and split
+// into equal-cost contiguous ranges, one per CTA.
+//
+// Workspace.  The call's control words -- per CTA 256 flagged partial-sum
+// words, one 256-byte block of record counters, and per row of a gate/up
+// pair one flagged word -- are zero before and after every call and sit at
+// the FRONT of the workspace; its data -- the activation records of every
+// distinct x and code width (1088 bytes per group), used when a CTA's
+// records do not fit in its shared memory -- are overwritten before they
+// are read and sit at the BACK.  A call needs 2 max(control, data) bytes,
+// so calls of different shapes can share one workspace sized for the
+// largest: no call's data ever reaches another call's control words.
+constexpr int64_t kMaxG8Ctas = 256;      // bound of the CTA count (partial-sum words)
 constexpr int64_t kG8Rows = kG8TileRows;
 constexpr long long kWaitCycles = 4000000000LL;      // about 2 s
 constexpr long long kTestWaitCycles = 20000000LL;    // about 10 ms (TB_FLAG_TEST_STALL)
 
-int64_t g8_padded_groups(int64_t G) { return (G + 7) / 8 * 8; }
-bool g8_needs_spad(int64_t G) { return G % 8 != 0; }
-// workspace of one item: records, then the padded scale copy if needed
-size_t g8_item_workspace(int64_t N, int64_t K) {
-    const int64_t G = K / kGroup;
-    return align256((size_t)G * kG8RecBytes) + (g8_needs_spad(G) ? align256((size_t)(N * g8_padded_groups(G) * 2)) : 0);
-}
-size_t g8_extra_workspace(int64_t tiles, int64_t chunks) {
-    const int64_t c = std::min(kMaxG8Ctas, std::max<int64_t>(chunks, 1));
-    return align256((size_t)(tiles * 8 * 4)) + align256((size_t)(c * 2 * kG8Rows * 4));
-}
 int64_t g8_tiles(int64_t N) { return (N + kG8Rows - 1) / kG8Rows; }
 int64_t g8_chunks(int grid, int64_t N, int64_t K) {
     const int64_t C = g8_chunk_groups(grid);
     return g8_tiles(N) * ((K / kGroup + C - 1) / C);
 }
+bool same_records(const Item& a, const Item& b) {
+    return a.X == b.X && a.K == b.K && (a.grid == TB_GRID_INT3) == (b.grid == TB_GRID_INT3);
+}
+
+struct G8Space {
+    size_t control = 0, data = 0;
+    size_t need() const { return 2 * std::max(control, data); }
+};
+
+// control and data bytes of a batch-1 launch over items[0 .. n)
+// (`pair`: items 0 and 1 are a gate/up pair)
+G8Space g8_space(const Item* items, int n, bool pair) {
+    G8Space sp;
+    int64_t chunks = 0;
+    for (int j = 0; j < n; ++j) {
+        chunks += g8_chunks(items[j].grid, items[j].N, items[j].K);
+        bool shared = false;
+        for (int i = 0; i < j && !shared; ++i) shared = same_records(items[i], items[j]);
+        if (!shared) sp.data += align256((size_t)(items[j].K / kGroup * kG8RecBytes));
+    }
+    const int64_t ctas = std::min(kMaxG8Ctas, std::max<int64_t>(chunks, 1));
+    sp.control = align256((size_t)(ctas * kG8Rows * 8)) + 256;  // + record counters and the CTA counter
+    if (pair) sp.control += align256((size_t)(items[0].N * 8));
+    return sp;
+}
 
 // `pair_first` >= 0 marks items pair_first (gate) and pair_first + 1 (up)
-// of equal shape whose outputs also give h = bf16(silu(gate) * up); the
-// pair's fp32 values and counters take g8_pair_workspace bytes more.
-size_t g8_pair_workspace(int64_t N) { return align256((size_t)(N * 8)) + align256((size_t)(g8_tiles(N) * 32)); }
-
+// of equal shape whose outputs also give h = bf16(silu(gate) * up) (only
+// pair_first == 0 with two items is used).
 tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes, bool overlap, bool stall,
-                            cudaStream_t st, int pair_first = -1, uint16_t* h = nullptr) {
+                            cudaStream_t st, int pair_first = -1, uint16_t* h = nullptr, bool ws_records = false) {
     G8Launch L;
     std::memset(&L, 0, sizeof(L));
-    char* w = static_cast<char*>(ws);
-    size_t need = 0;
-    int64_t prep = 0, tiles = 0, chunk = 0, cost = 0;
+    const G8Space sp = g8_space(items, n, pair_first >= 0);
+    if (!ws || ws_bytes < sp.need()) return TB_ERR_ARG;
+    char* ctl = static_cast<char*>(ws);                                        // control words: the front
+    char* dat = static_cast<char*>(ws) + (ws_bytes & ~size_t(255)) - sp.data;  // data: the back
+    int64_t chunk = 0, cost = 0;
     for (int j = 0; j < n; ++j) {
         const Item& it = items[j];
         G8Item& s = L.it[j];
@@ -198,7 +220,6 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
         s.Y = it.Y;
         s.N = it.N;
         s.G = (int32_t)G;
-        s.Gp = (int32_t)g8_padded_groups(G);
         s.T = (int32_t)g8_tiles(it.N);
         s.C = g8_chunk_groups(it.grid);
         s.cpt = (s.G + s.C - 1) / s.C;
@@ -207,56 +228,54 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
         s.ydt = it.ydt;
         s.chunk_base = chunk;
         s.cost_base = cost;
-        s.tile_base = (int32_t)tiles;
-        s.rec = reinterpret_cast<uint8_t*>(w + need);
-        s.spad = g8_needs_spad(G) ? reinterpret_cast<uint16_t*>(w + need + align256((size_t)G * kG8RecBytes))
-                                  : nullptr;
-        need += g8_item_workspace(it.N, it.K);
-        // items reading the same x with the same code width share one record set
-        int owner = -1;
-        for (int i = 0; i < j && owner < 0; ++i)
-            if (items[i].X == it.X && items[i].K == it.K && (items[i].grid == TB_GRID_INT3) == (it.grid == TB_GRID_INT3))
-                owner = i;
-        if (owner >= 0) {
-            s.rec = L.it[owner].rec;
-        } else {
-            G8Prep& P = L.prep[L.n_prep++];
-            P.x = it.X;
-            P.rec = s.rec;
-            P.begin = (int32_t)prep;
-            P.three = it.grid == TB_GRID_INT3 ? 1 : 0;
-            prep += G;
-        }
+        s.stage_scales = G % 8 != 0 ? 1 : 0;  // rows of 2 G bytes: a tensor copy needs multiples of 16
         chunk += (int64_t)s.T * s.cpt;
         cost += (int64_t)s.T * s.G * s.unit_cost;
-        tiles += s.T;
     }
-    if (cost >= ((int64_t)1 << 31) || chunk >= ((int64_t)1 << 31) || prep >= ((int64_t)1 << 31))
-        return TB_ERR_UNSUPPORTED;  // partition arithmetic is 32-bit
-    L.counters = reinterpret_cast<int32_t*>(w + need);
-    L.n_counters = (int32_t)(tiles * 8);
-    L.partials = reinterpret_cast<float*>(w + need + align256((size_t)(tiles * 8 * 4)));
-    need += g8_extra_workspace(tiles, chunk);
+    if (cost >= ((int64_t)1 << 31) || chunk >= ((int64_t)1 << 31)) return TB_ERR_UNSUPPORTED;  // 32-bit partition
+    const int64_t ctas_max = std::min(kMaxG8Ctas, std::max<int64_t>(chunk, 1));
+    L.pslots = reinterpret_cast<uint64_t*>(ctl);
+    ctl += align256((size_t)(ctas_max * kG8Rows * 8));
+    int32_t* small = reinterpret_cast<int32_t*>(ctl);  // record counters [16], then the CTA counter
+    ctl += 256;
+    L.done = small + kMaxItems;
+    // activation records: items reading the same x with the same code width share one set
+    int32_t n_build = 0;
+    for (int j = 0; j < n; ++j) {
+        int owner = -1;
+        for (int i = 0; i < j && owner < 0; ++i)
+            if (same_records(items[i], items[j])) owner = L.it[i].owner;
+        if (owner < 0) {
+            owner = L.n_own++;
+            G8Owner& o = L.own[owner];
+            o.x = items[j].X;
+            o.rec = reinterpret_cast<uint8_t*>(dat);
+            o.ready = small + owner;
+            o.G = L.it[j].G;
+            o.three = items[j].grid == TB_GRID_INT3 ? 1 : 0;
+            o.build_base = n_build;
+            n_build += o.G;
+            dat += align256((size_t)(o.G * kG8RecBytes));
+        }
+        L.it[j].owner = owner;
+    }
+    L.n_build = n_build;
     L.pair_first = -1;
-    if (pair_first >= 0) {  // after the partials: the pair's values, then its counters
-        const int64_t N = items[pair_first].N;
+    if (pair_first >= 0) {
         L.pair_first = pair_first;
-        L.pair_vals = reinterpret_cast<float*>(w + need);
-        L.pair_counters = reinterpret_cast<int32_t*>(w + need + align256((size_t)(N * 8)));
+        L.pair_slots = reinterpret_cast<uint64_t*>(ctl);
         L.h = h;
-        need += g8_pair_workspace(N);
     }
-    if (!ws || ws_bytes < need) return TB_ERR_ARG;
     for (int j = 0; j < n; ++j) {
         const G8Item& s = L.it[j];
         if (!encode_g8_wmap(&L.wmap[j], items[j].packed, items[j].grid, s.N, items[j].K)) return TB_ERR_CUDA;
-        if (!encode_g8_smap(&L.smap[j], s.spad ? s.spad : s.scales, s.N, s.Gp)) return TB_ERR_CUDA;
+        if (!s.stage_scales && !encode_g8_smap(&L.smap[j], s.scales, s.N, s.G)) return TB_ERR_CUDA;
     }
     const int resident = gemv8_ctas();
     if (resident <= 0) return TB_ERR_CUDA;
     // every quota at least one chunk's cost (4 x 2 or 2 x 3): then every CTA
     // between a tile's first and last owner owns a chunk of it, which the
-    // partial-sum combine relies on
+    // split-tile combine relies on
     int64_t nctas = std::max<int64_t>(1, std::min<int64_t>({(int64_t)resident, chunk, kMaxG8Ctas, cost / 8}));
     const int64_t Q = (cost + nctas - 1) / nctas;
     nctas = (cost + Q - 1) / Q;
@@ -264,10 +283,36 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
     L.nctas = (int32_t)nctas;
     L.Ctot = (uint32_t)cost;
     L.Q = (uint32_t)Q;
-    L.prep_warps = (int32_t)prep;
+    // each CTA's range and its first chunk's place; records in shared memory when every range's fit
+    int32_t most = 0;
+    for (int64_t c = 0; c < nctas; ++c) {
+        G8Range& r = L.range[c];
+        part_chunk_range(L.it, n, (uint32_t)c, L.Q, L.Ctot, &r.cb, &r.ce);
+        r.item = 0;
+        for (int i = 1; i < n; ++i)
+            if (r.cb >= (uint32_t)L.it[i].chunk_base) r.item = i;
+        const uint32_t local = r.cb - (uint32_t)L.it[r.item].chunk_base, cpt = (uint32_t)L.it[r.item].cpt;
+        r.tile = (int32_t)(local / cpt);
+        r.j = (int32_t)(local - (uint32_t)r.tile * cpt);
+        RecSlots rs;
+        part_rec_slots(L.it, n, r.cb, r.ce, &rs);
+        most = std::max(most, rs.total);
+    }
+    L.local_records = most <= kG8RecSlots && !ws_records ? 1 : 0;
     L.stall = stall ? 1 : 0;
     L.wait_cycles = stall ? kTestWaitCycles : kWaitCycles;
     return cuda_status(launch_gemv8(L, overlap, st));
+}
+
+// the items of a layer call that run on the integer tensor path
+int g8_layer_items(const tb_linear_t* items, int n_items, Item* its) {
+    int n = 0;
+    for (int i = 0; i < n_items; ++i) {
+        const tb_linear_t& l = items[i];
+        if (is_b3(l.grid)) continue;  // launched on their own, without workspace
+        its[n++] = make_item(l.packed, l.grid, l.scales, l.x, l.K, l.y, l.y_dtype, l.N, 1, l.N, l.K);
+    }
+    return n;
 }
 
 }  // namespace
@@ -345,23 +390,21 @@ size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K) {
         const int64_t rem = M % kGemmBlockM;
         return std::max(tb_workspace_bytes(kGemmBlockM, N, K), rem ? tb_workspace_bytes(rem, N, K) : (size_t)0);
     }
-    if (M == 1) return g8_item_workspace(N, K) + g8_extra_workspace(g8_tiles(N), g8_chunks(TB_GRID_INT3, N, K));
-    if (M >= kTCMinM) return gemm_tc_workspace_bytes(M, N, K);
+    if (M == 1) {  // the 3-bit chunking (more chunks) bounds both widths
+        const Item it = make_item(nullptr, TB_GRID_INT3, nullptr, nullptr, K, nullptr, TB_F32, N, 1, N, K);
+        return g8_space(&it, 1, false).need();
+    }
+    if (M >= kTCMinM) return 2 * gemm_tc_workspace_bytes(M, N, K);
     return kNoWorkspace;
 }
 
 size_t tb_layer_workspace_bytes(const tb_linear_t* items, int n_items) {
     if (!items || n_items < 1 || n_items > TB_MAX_LAYER_ITEMS) return 0;
-    size_t b = 0;
-    int64_t tiles = 0, chunks = 0;
-    for (int i = 0; i < n_items; ++i) {
+    for (int i = 0; i < n_items; ++i)
         if (!shape_ok(items[i].N, items[i].K) || !grid_ok(items[i].grid)) return 0;
-        if (is_b3(items[i].grid)) continue;  // launched on their own, without workspace
-        b += g8_item_workspace(items[i].N, items[i].K);
-        tiles += g8_tiles(items[i].N);
-        chunks += g8_chunks(items[i].grid, items[i].N, items[i].K);
-    }
-    return b + g8_extra_workspace(tiles, chunks);
+    Item its[kMaxItems];
+    const int n = g8_layer_items(items, n_items, its);
+    return n ? g8_space(its, n, false).need() : kNoWorkspace;
 }
 
 tb_status_t tb_gemv(const void* packed, tb_grid_t grid, const uint16_t* scales, const uint16_t* x, void* y,
@@ -422,11 +465,12 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
         return launch_g8_items(&it, 1, workspace, workspace_bytes, false, false, st);
     }
     if (M >= kTCMinM) {
-        if (workspace_bytes < gemm_tc_workspace_bytes(M, N, K)) return TB_ERR_ARG;
         if (K / kGroup * 64 > INT_MAX || (N + 127) / 128 > INT_MAX / 16 ||
             (N + 127) / 128 * (K / kGroup) >= ((int64_t)1 << 32))
             return TB_ERR_SHAPE;
-        return cuda_status(launch_gemm_tc(packed, grid, scales, X, ldx, Y, y_dtype, ldy, (int)M, N, K, workspace, st));
+        // all of its workspace is data (it clears its own counters): the back
+        char* back = static_cast<char*>(workspace) + (workspace_bytes & ~size_t(255)) - gemm_tc_workspace_bytes(M, N, K);
+        return cuda_status(launch_gemm_tc(packed, grid, scales, X, ldx, Y, y_dtype, ldy, (int)M, N, K, back, st));
     }
     // column blocks of up to 16 batch rows per launch
     const size_t ysz = y_dtype == TB_F32 ? 4 : 2;
@@ -442,7 +486,9 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
 tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags, void* workspace,
                           size_t workspace_bytes, tb_stream_t stream) {
     if (!items || n_items < 1 || n_items > TB_MAX_LAYER_ITEMS) return TB_ERR_ARG;
-    if ((flags & ~(unsigned)(TB_FLAG_OVERLAP_PREVIOUS | TB_FLAG_TEST_STALL)) != 0 || !workspace) return TB_ERR_ARG;
+    if ((flags & ~(unsigned)(TB_FLAG_OVERLAP_PREVIOUS | TB_FLAG_TEST_STALL | TB_FLAG_TEST_WORKSPACE_RECORDS)) != 0 ||
+        !workspace)
+        return TB_ERR_ARG;
     if (!aligned(workspace, 256)) return TB_ERR_ALIGN;
     Item its[kMaxItems];
     int n_main = 0;
@@ -463,7 +509,8 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
     if (n_main > 0) {
         const tb_status_t s = launch_g8_items(its, n_main, workspace, workspace_bytes,
                                               (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0,
-                                              (flags & TB_FLAG_TEST_STALL) != 0, st);
+                                              (flags & TB_FLAG_TEST_STALL) != 0, st, -1, nullptr,
+                                              (flags & TB_FLAG_TEST_WORKSPACE_RECORDS) != 0);
         if (s != TB_OK) return s;
     }
     // items in the 5-trits-per-byte layout: one launch each, after the grouped launch
@@ -478,16 +525,18 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
 
 size_t tb_gate_up_workspace_bytes(const tb_linear_t* gate, const tb_linear_t* up) {
     if (!gate || !up || gate->N != up->N || gate->K != up->K) return 0;
-    const tb_linear_t two[2] = {*gate, *up};
+    if (!shape_ok(gate->N, gate->K) || !grid_ok(gate->grid) || !grid_ok(up->grid)) return 0;
     if (is_b3(gate->grid) || is_b3(up->grid)) return 0;
-    const size_t b = tb_layer_workspace_bytes(two, 2);
-    return b ? b + g8_pair_workspace(gate->N) : 0;
+    const tb_linear_t two[2] = {*gate, *up};
+    Item its[2];
+    g8_layer_items(two, 2, its);
+    return g8_space(its, 2, true).need();
 }
 
 tb_status_t tb_gate_up_silu(const tb_linear_t* gate, const tb_linear_t* up, uint16_t* h, unsigned flags,
                             void* workspace, size_t workspace_bytes, tb_stream_t stream) {
     if (!gate || !up || !h || !workspace) return TB_ERR_ARG;
-    if ((flags & ~(unsigned)TB_FLAG_OVERLAP_PREVIOUS) != 0) return TB_ERR_ARG;
+    if ((flags & ~(unsigned)(TB_FLAG_OVERLAP_PREVIOUS | TB_FLAG_TEST_WORKSPACE_RECORDS)) != 0) return TB_ERR_ARG;
     if (gate->N != up->N || gate->K != up->K) return TB_ERR_SHAPE;
     if (!aligned(workspace, 256) || !aligned(h, 2)) return TB_ERR_ALIGN;
     Item its[2];
@@ -504,7 +553,7 @@ tb_status_t tb_gate_up_silu(const tb_linear_t* gate, const tb_linear_t* up, uint
     }
     if (workspace_bytes < tb_gate_up_workspace_bytes(gate, up)) return TB_ERR_ARG;
     return launch_g8_items(its, 2, workspace, workspace_bytes, (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0, false,
-                           static_cast<cudaStream_t>(stream), 0, h);
+                           static_cast<cudaStream_t>(stream), 0, h, (flags & TB_FLAG_TEST_WORKSPACE_RECORDS) != 0);
 }
 
 }  // extern "C"
@@ -514,8 +563,9 @@ tb_status_t tb_gate_up_silu(const tb_linear_t* gate, const tb_linear_t* up, uint
 // Same kernels and results as tb_gemv; the workspace is this file-scope
 // device array instead of caller memory, so the call allocates nothing.
 // The only state that must start at zero (the per-tile arrival counters)
-// is zeroed by the preparation kernel of every call, so the array needs no
-// clearing; every call rewrites what it reads.  All calls on a device
+// starts zeroed (static storage) and every call leaves it zero again, so
+// the array needs no clearing; every call rewrites what else it reads.  All
+// calls on a device
 // share the one array: calls that may run at the same time (different
 // streams, or different host threads without stream ordering) race on it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[TB_NOALLOC_SCRATCH_BYTES];

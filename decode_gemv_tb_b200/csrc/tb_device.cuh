@@ -45,55 +45,70 @@ struct Launch {
 };
 
 // ---- batch-1 launch on the integer tensor path (see tb_gemv8.cu) ----------
-// One activation record per 128-group: the group's activations as eight
-// signed 7-bit digit columns in the order the MMA B fragments are read
-// (1024 bytes), then per digit pair t = 0..3 the accumulator start values
-// of digit columns 2t, 2t+1 and the float 2^(14 t - F) (64 bytes).
+// The activation record of one 128-group, built once per call by the first
+// CTA that needs it and copied into the stage of every chunk that needs it:
+// the group's activations as eight signed 7-bit digit columns in the order
+// the MMA B fragments are read (1024 bytes), then per digit pair t = 0..3
+// the accumulator start values of digit columns 2t, 2t+1 and the float
+// 2^(14 t - F) (64 bytes).
 constexpr int kG8RecBytes = 1088;
+constexpr int kG8Warps = 8;      // consumer warps of k_gemv8
+constexpr int kG8RecSlots = 56;  // records a CTA of k_gemv8 holds in shared memory
 constexpr int kG8TileRows = 256;  // rows of a tile: 8 consumer warps x 32 rows
 
 struct G8Item {
     const uint16_t* x;       // [K] bf16 activations
-    const uint16_t* scales;  // [N][G] bf16, the caller's
-    uint16_t* spad;          // [N][Gp] copy of the scales with rows padded to 8 groups, or null
-    uint8_t* rec;            // [G] records of kG8RecBytes
+    const uint16_t* scales;  // [N][G] bf16
     void* Y;
     int64_t N;
     int64_t chunk_base, cost_base;  // ChunkItem fields (tb_partition.h)
     int32_t T, G, C, cpt, unit_cost;
-    int32_t grid, ydt, tile_base, Gp;
+    int32_t grid, ydt, tile_base;
+    int32_t stage_scales;  // 1: the producer warp copies the scales (rows not 16-byte multiples); 0: a tensor copy
+    int32_t owner;         // index of the activation-record set this item reads
 };
 
-// One set of activation records the preparation kernel writes: items that
-// read the same x with the same code width share one.
-struct G8Prep {
-    const uint16_t* x;
-    uint8_t* rec;
-    int32_t begin;  // first preparation warp (one per group)
-    int32_t three;  // the 3-bit slot map
+// One set of activation records: those of one x at one code width (items
+// reading the same x with the same width share it), built once per call.
+struct G8Owner {
+    const uint16_t* x;  // [G * 128] bf16
+    uint8_t* rec;       // [G] records of kG8RecBytes, 256-byte aligned
+    int32_t* ready;     // records published so far: zero before the call, zero after it
+    int32_t G, three;
+    int32_t build_base;  // index of its first record in the call's build order
 };
+
+// A CTA's range of chunks [cb, ce) and the (item, tile, chunk in tile) of cb.
+struct G8Range {
+    uint32_t cb, ce;
+    int32_t item, tile, j;
+};
+constexpr int kMaxG8Ranges = 256;
 
 struct G8Launch {
     CUtensorMap wmap[kMaxItems];  // packed weights: bytes x rows, box (C groups) x 256 rows
-    CUtensorMap smap[kMaxItems];  // scales [N][Gp] bf16: box 8 groups x 256 rows
+    CUtensorMap smap[kMaxItems];  // scales [N][G] bf16: box 8 groups x 256 rows (stage_scales == 0)
     G8Item it[kMaxItems];
-    int32_t n_items, nctas;
+    G8Owner own[kMaxItems];
+    int32_t n_items, nctas, n_own, n_build;
     uint32_t Ctot, Q;      // total cost and cost quota per CTA (tb_partition.h)
-    int32_t* counters;     // [tiles][8] arrival counters, zeroed by the preparation kernel
-    int32_t n_counters;
-    float* partials;       // [nctas][2][256] partial sums of split tiles
-    G8Prep prep[kMaxItems];
-    int32_t n_prep;
-    int32_t prep_warps;    // one per group of every record set
-    int32_t stall;         // test hook: the copies are never issued, every wait gives up
+    G8Range range[kMaxG8Ranges];  // per CTA, from the partition
+    // 1: every CTA builds the records its range reads in shared memory; 0:
+    // the CTAs build each record once, in the workspace (own[], n_build)
+    int32_t local_records;
+    int32_t* done;         // CTAs finished with the workspace records: zero before the call, zero after it
+    // [nctas][256] partial sums of split tiles as (fp32 bits, flag 1) words,
+    // written by the CTA that reads the tile's end, cleared by the one that
+    // reads its start: zero before the call, zero after it
+    uint64_t* pslots;
+    int32_t stall;         // test hook: the weights are never copied, every wait gives up
     long long wait_cycles; // bound of every wait
     // gated MLP input: items pair_first (gate) and pair_first + 1 (up) of equal
-    // shape; the last of the two to finish a warp's 32 rows writes
-    // h = bf16(silu(gate) * up) for them (-1: no pair)
+    // shape; once both results of a row are final, h = bf16(silu(gate) * up)
+    // (-1: no pair)
     int32_t pair_first;
-    int32_t* pair_counters;  // [tiles of the pair][8], cleared by the preparation kernel
-    float* pair_vals;        // [2][N] the pair's fp32 results
-    uint16_t* h;             // [N] bf16
+    uint64_t* pair_slots;  // [N] gate results as (fp32 bits, flag 1): zero before the call, zero after it
+    uint16_t* h;           // [N] bf16
 };
 
 // ---- cache-controlled loads ----------------------------------------------

@@ -17,7 +17,7 @@
 //   * the activations of the group become fixed-point integers
 //     X_k = trunc(|x_k| 2^(F - cls_k)) (F from the group's largest |x|, so
 //     that X < 2^56) split into eight signed 7-bit digit columns, the B
-//     operand's eight columns (the preparation kernel below);
+//     operand's eight columns (built per chunk in shared memory, below);
 //   * the MMA sums u * 2^cls * digit exactly in int32, and starting its
 //     accumulator at -offset * sum_k 2^cls_k digit_k subtracts the offset
 //     exactly, so a zero codeword contributes exactly nothing however large
@@ -29,19 +29,33 @@
 // the truncation of activations more than 2^42 below their group's largest
 // (include/tb.h states the bound).
 //
-// Data flow.  One CTA per SM: a producer warp and eight consumer warps.  The
-// work of a call is the sequence of chunks (item, tile of 256 rows, C
-// consecutive groups: C = 4 for the 2-bit container, 2 for 3 bits) in item,
-// tile, group order; each CTA owns a contiguous range of equal cost
-// (tb_partition.h).  The producer streams each chunk into a ring of stages
-// with three copies completing on the stage's mbarrier: a 2-D tensor copy of
-// the packed weights (256 rows x 128 or 96 bytes; no multicast), a 2-D
-// tensor copy of the scales (256 rows x 8 groups) and a bulk copy of the
-// chunk's activation records, which every consumer warp shares.  Consumer
-// warp w decodes rows 32w .. 32w+31 with LOP3 masks, runs eight MMAs per
-// group and accumulates in fp32.  A tile whose groups are split between
-// CTAs is combined by the last CTA to finish its part (per warp rows,
-// arrival counter), in CTA order: results are bitwise deterministic.
+// Data flow.  One kernel per call, one CTA per SM: eight consumer warps and
+// a producer warp.  The work of a call is the sequence of chunks (item, tile
+// of 256 rows, C consecutive groups: C = 4 for the 2-bit container, 2 for 3
+// bits) in item, tile, group order; each CTA owns a contiguous range of
+// equal cost (tb_partition.h).
+//   * Records.  When the records a range reads fit in shared memory (the
+//     usual case: a range covers about one tile of one or two items), the
+//     consumer warps build them there once the previous kernel in the stream
+//     has finished (x prefetched into L2 before that), then meet at a named
+//     barrier.  Otherwise the consumer warps of all CTAs build each record
+//     once, in the workspace, count them per record set, and the producer
+//     copies a chunk's records into its stage once the set is complete.
+//   * Stages.  Each chunk passes through a ring of shared-memory stages.
+//     The producer copies the packed weights (a 2-D tensor copy of 256 rows
+//     x 128 or 96 bytes, no multicast) and the scales (256 rows x 8 groups)
+//     into the stage -- inputs no earlier kernel writes, so the first stages
+//     are requested at once, even before the previous call in the stream has
+//     finished.
+//   * Consumer warp w decodes rows 32w .. 32w+31 with LOP3 masks, runs eight
+//     MMAs per group and accumulates in fp32.
+// A stage is full when its copies have landed and the producer has
+// arrived; empty when all eight consumers have.  A tile whose groups are
+// split between CTAs is combined by the CTA that reads its first chunk --
+// for which it is the last segment of its range, so the others have long
+// finished theirs: each later CTA publishes its partial sum of the tile's
+// rows as (fp32 bits, flag) in one 64-bit store, and the combining CTA adds
+// them in CTA order (results are bitwise deterministic) and clears them.
 // Every wait is bounded; a wait that gives up is counted, the warp stops
 // waiting and writes NaN for the rest of its range.
 #include "tb_device.cuh"
@@ -56,16 +70,21 @@ __device__ unsigned int g_g8_timeouts = 0;  // bounded waits of this file's kern
 
 namespace {
 
-constexpr int kCWarps = 8;                         // consumer warps
-constexpr int kG8Threads = (kCWarps + 1) * 32;     // + the producer warp
+constexpr int kCWarps = kG8Warps;                  // consumer warps
+constexpr int kProducer = kCWarps;                 // the producer warp
+constexpr int kG8Threads = (kCWarps + 1) * 32;
 constexpr int kStages = 4;
+constexpr int kLookahead = 8;                      // chunks beyond the ring requested into L2 ahead of their copy
 constexpr int kSOff = 32768;                       // scales box: 256 rows x 8 bf16
-constexpr int kROff = kSOff + 4096;                // records: up to 4 x 1088 bytes
+constexpr int kROff = kSOff + 4096;                // records copied from the workspace: up to 4 x 1088 bytes
 constexpr int kStageBytes = 41984;                 // >= kROff + 4 * kG8RecBytes, a multiple of 1 KB
-constexpr int kG8Smem = kStages * kStageBytes + 1024;  // + alignment slack (swizzled boxes: 1 KB)
-constexpr int kPrepThreads = 256;
+constexpr int kCache = kStages * kStageBytes;      // record cache (or the builders' scratch)
+constexpr int kG8Smem = kCache + kG8RecSlots * kG8RecBytes + 1024;  // + alignment slack (swizzled boxes: 1 KB)
 
 static_assert(kROff + 4 * kG8RecBytes <= kStageBytes, "stage layout");
+static_assert(kCWarps * kG8RecBytes <= kG8RecSlots * kG8RecBytes, "scratch");
+static_assert(kG8Smem <= 227 * 1024, "shared memory");
+constexpr int kSlotsPerWarp = (kG8RecSlots + kCWarps - 1) / kCWarps;
 
 // ---- small PTX helpers ------------------------------------------------------
 __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -73,21 +92,24 @@ __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cv
 __device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
+// raises the transaction count of the current phase (no arrival)
 __device__ __forceinline__ void bar_expect(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ void bar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// true once the phase with this parity has completed; false after `limit` cycles
+// true once the phase with this parity has completed; false after `limit`
+// cycles.  Each try suspends the thread until the phase completes or about
+// 20 us pass, so a waiting warp takes no issue slots from the working ones.
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, long long limit) {
     const long long t0 = clock64();
     for (;;) {
         uint32_t done;
         asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
             : "=r"(done)
-            : "r"(bar), "r"(parity)
+            : "r"(bar), "r"(parity), "r"(20000u)
             : "memory");
         if (done) return true;
         if (clock64() - t0 > limit) return false;
@@ -101,11 +123,58 @@ __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, in
         "l"(map), "r"(x), "r"(y), "r"(bar)
         : "memory");
 }
-// 1-D bulk copy global -> shared (no multicast)
+// hint: bring the 2-D box at (x, y) of map into L2 (no copy into shared memory)
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y) : "memory");
+}
+// 1-D bulk copy global -> shared (no multicast): bytes a multiple of 16, both addresses 16-byte aligned
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+// 64-bit words read and written whole (single-copy atomic)
+__device__ __forceinline__ void st_word(uint64_t* p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_word(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint64_t flagged(float v) { return (1ull << 32) | __float_as_uint(v); }
+// the value of a flagged word once its flag is set; false after `limit` cycles
+__device__ __forceinline__ bool wait_word(const uint64_t* p, long long limit, float* v) {
+    const long long t0 = clock64();
+    for (;;) {
+        const uint64_t w = ld_word(p);
+        if (w >> 32) {
+            *v = __uint_as_float((uint32_t)w);
+            return true;
+        }
+        if (clock64() - t0 > limit) return false;
+        __nanosleep(64);
+    }
+}
+// hints: bring bytes of global memory into L2; fetch a tensor map's descriptor
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const void* p) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(p) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // d += A B, A 16 x 32 unsigned bytes (row), B 32 x 8 signed bytes (col), int32 accumulate
@@ -164,152 +233,161 @@ __device__ __forceinline__ void decode3(uint32_t p0, uint32_t p1, uint32_t p2, u
     R[7] = bit_mux(bit_mux(r0, r1, 0x40404040u), p2, 0x80808080u) & 0xE0E0E0E0u;  // bit 7 fields at 5..7
 }
 
-// ---- preparation: one warp per (item, group) -----------------------------------
-// Record of group g (kG8RecBytes):
+// ---- activation records ---------------------------------------------------
+// Record of a group (kG8RecBytes), built by one warp:
 //   bytes [512 h + 16 L + 8 (kk & 1) + 4 hf + b], h = kk >> 1, lane L = 4 j + t:
 //     digit j of the activation in MMA kk, slot 16 hf + 4 t + b;
 //   bytes 1024 + 16 t: int32 -offset * O_{2t}, -offset * O_{2t+1}, float 2^(14 t - F), 0,
 //     O_j = sum over the group's slots of 2^cls * digit j.
 // F = min(55 - E, 149), E the exponent of the group's largest |x| (a zero or
 // subnormal group counts as 2^-126), so every X = trunc(|x| 2^(F - cls)) is
-// below 2^56 and every scale factor 2^(14 t - F) is a float.
-__global__ void __launch_bounds__(kPrepThreads) k_prep8(const __grid_constant__ G8Launch L) {
-    pdl_trigger();  // the main kernel may start streaming weights now
-    pdl_wait();     // x may come from the previous kernel, which may also still read the workspace
-    const int tid = blockIdx.x * kPrepThreads + threadIdx.x, nthr = gridDim.x * kPrepThreads;
-    for (int i = tid; i < L.n_counters; i += nthr) L.counters[i] = 0;  // arrival counters
-    if (L.pair_first >= 0)
-        for (int i = tid; i < L.it[L.pair_first].T * kCWarps; i += nthr) L.pair_counters[i] = 0;
-    for (int ii = 0; ii < L.n_items; ++ii) {  // scale rows padded to a multiple of 8 groups (tensor-copy stride)
-        const G8Item& I = L.it[ii];
-        if (!I.spad) continue;
-        const int64_t n = I.N * I.Gp;
-        for (int64_t e = tid; e < n; e += nthr) {
-            const int64_t row = e / I.Gp, col = e - row * I.Gp;
-            I.spad[e] = col < I.G ? I.scales[row * I.G + col] : (uint16_t)0;
-        }
-    }
-    const int wi = tid >> 5, lane = threadIdx.x & 31;
-    if (wi >= L.prep_warps) return;
-    int pi = 0;
-    for (int i = 1; i < L.n_prep; ++i)
-        if (wi >= L.prep[i].begin) pi = i;
-    const G8Prep& P = L.prep[pi];
-    const int64_t grp = wi - P.begin;
-    const uint16_t* xg = P.x + grp * kGroup;
-    uint8_t* rec = P.rec + grp * kG8RecBytes;
-
-    const uint2 raw = *reinterpret_cast<const uint2*>(xg + 4 * lane);
+// below 2^56 and every scale factor 2^(14 t - F) is a float.  The eight
+// bits of an activation's mantissa fill at most two consecutive 7-bit
+// digits.  The offset sums come from four MMAs of the record's own B
+// fragments against A = 2^cls in every byte (a group of codes u = 1).
+// `raw` holds x[4 lane .. 4 lane + 3] of the group.
+__device__ __noinline__ void make_record(const uint2 raw, bool three, uint8_t* rec) {
+    const int lane = threadIdx.x & 31;
     int e = max(max((int)((raw.x >> 7) & 0xFFu), (int)((raw.x >> 23) & 0xFFu)),
                 max((int)((raw.y >> 7) & 0xFFu), (int)((raw.y >> 23) & 0xFFu)));
 #pragma unroll
     for (int o = 16; o; o >>= 1) e = max(e, __shfl_xor_sync(0xffffffffu, e, o));
     const int E = max(e, 1) - 127;
     const int F = min(55 - E, 149);
-
-    const bool three = P.three != 0;
     const int gq = lane >> 2, tq = lane & 3;
     const int kk = gq >> 1, hf = gq & 1, r = 2 * kk + hf;
     const int cls = slot_class(three, r);
-    uint32_t dig[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    int osum[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    uint32_t lo[4], hi[4];  // digit bytes 0-3 / 4-7 of the lane's four slots
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-        const uint32_t h = xg[32 * tq + slot_code(three, r, b)];
+        const int code = 32 * tq + slot_code(three, r, b);
+        const uint32_t vx = __shfl_sync(0xffffffffu, raw.x, code >> 2), vy = __shfl_sync(0xffffffffu, raw.y, code >> 2);
+        const uint32_t v2 = (code & 2) ? vy : vx;
+        const uint32_t h = (code & 1) ? (v2 >> 16) : (v2 & 0xFFFFu);
         const int eb = (int)((h >> 7) & 0xFFu);
-        const uint64_t m = (h & 0x7Fu) | (eb ? 0x80u : 0u);  // |x| = m 2^(max(eb,1) - 134)
-        const int sh = max(eb, 1) - 134 + F - cls;           // <= 48 - cls
-        const uint64_t X = sh >= 0 ? (m << sh) : (-sh >= 64 ? 0ull : (m >> -sh));
-        const bool neg = (h >> 15) != 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int d0 = (int)((X >> (7 * j)) & 127u), d = neg ? -d0 : d0;
-            dig[j] |= (uint32_t)(d & 0xFF) << (8 * b);
-            osum[j] += d;
+        uint32_t m = (h & 0x7Fu) | (eb ? 0x80u : 0u);  // |x| = m 2^(max(eb,1) - 134)
+        int sh = max(eb, 1) - 134 + F - cls;           // <= 48 - cls
+        if (sh < 0) {
+            m = -sh >= 8 ? 0u : m >> -sh;  // truncated below 2^0
+            sh = 0;
         }
+        const int j0 = (sh * 37) >> 8;  // sh / 7 for 0 <= sh <= 48
+        const uint32_t v = m << (sh - 7 * j0);           // < 2^14: digits j0 and j0 + 1
+        uint64_t mag = (uint64_t)((v & 127u) | ((v >> 7) << 8)) << (8 * j0);
+        if (h >> 15) mag = (0x8080808080808080ull - mag) ^ 0x8080808080808080ull;  // bytewise negation
+        lo[b] = (uint32_t)mag;
+        hi[b] = (uint32_t)(mag >> 32);
     }
+    // digit column j of the four slots as one word, stored where lane (j, tq) reads its B fragment
+    uint8_t* dst = rec + (kk >> 1) * 512 + tq * 16 + (kk & 1) * 8 + hf * 4;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        *reinterpret_cast<uint32_t*>(rec + (kk >> 1) * 512 + (4 * j + tq) * 16 + (kk & 1) * 8 + hf * 4) = dig[j];
-        int o = osum[j] * (1 << cls);  // |o| <= 4 * 127 * 2^6 per lane, the group total below 2^21
-#pragma unroll
-        for (int s = 16; s; s >>= 1) o += __shfl_xor_sync(0xffffffffu, o, s);
-        osum[j] = o;
+        const uint32_t* src = j < 4 ? lo : hi;
+        const uint32_t sel = (uint32_t)(j & 3) | ((uint32_t)(4 + (j & 3)) << 4);
+        const uint32_t p01 = __byte_perm(src[0], src[1], sel), p23 = __byte_perm(src[2], src[3], sel);
+        *reinterpret_cast<uint32_t*>(dst + 64 * j) = __byte_perm(p01, p23, 0x5410);
     }
-    if (lane < 4) {
-        const int off = three ? 4 : 2, t = lane, v = 14 * t - F;  // v in [-149, 114]
+    __syncwarp();
+    // offset sums: D[.][j] = sum over slots of 2^cls * digit j
+    const uint4 B0 = *reinterpret_cast<const uint4*>(rec + 16 * lane);
+    const uint4 B1 = *reinterpret_cast<const uint4*>(rec + 512 + 16 * lane);
+    uint32_t A[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) A[q] = 0x01010101u << slot_class(three, q);
+    int d[4] = {0, 0, 0, 0};
+    mma_u8s8(d, A[0], A[0], A[1], A[1], B0.x, B0.y);
+    mma_u8s8(d, A[2], A[2], A[3], A[3], B0.z, B0.w);
+    mma_u8s8(d, A[4], A[4], A[5], A[5], B1.x, B1.y);
+    mma_u8s8(d, A[6], A[6], A[7], A[7], B1.z, B1.w);
+    if (lane < 4) {  // g = 0, t = lane: columns 2t, 2t+1
+        const int off = three ? 4 : 2, v = 14 * lane - F;  // v in [-149, 114]
         const uint32_t ebits = v >= -126 ? (uint32_t)(v + 127) << 23 : 1u << (v + 149);
-        *reinterpret_cast<uint4*>(rec + 1024 + 16 * t) =
-            make_uint4((uint32_t)(-off * osum[2 * t]), (uint32_t)(-off * osum[2 * t + 1]), ebits, 0u);
+        *reinterpret_cast<uint4*>(rec + 1024 + 16 * lane) =
+            make_uint4((uint32_t)(-off * d[0]), (uint32_t)(-off * d[1]), ebits, 0u);
     }
 }
 
-// ---- main kernel ------------------------------------------------------------------
-// Row of the 256-row tile that MMA row (tile rt, half h: rows g / g+8) of
-// lane group g in warp w reads: eight consecutive rows of a quarter differ in
-// (row & 7) >> 1 within each half warp, which keeps the 128-byte-swizzled
-// weight loads free of bank conflicts.
-__device__ __forceinline__ int tile_row(int w, int rt, int h, int g) { return 32 * w + 8 * (2 * rt + h) + 2 * (g & 3) + (g >> 2); }
+// Builds record g of set O in this warp's scratch, writes it to the
+// workspace and counts it as published.
+__device__ __noinline__ void publish_record(const G8Owner& O, int g, uint8_t* scratch) {
+    const int lane = threadIdx.x & 31;
+    make_record(__ldcg(reinterpret_cast<const uint2*>(O.x + (int64_t)g * kGroup) + lane), O.three != 0, scratch);
+    __syncwarp();
+    uint4* dst = reinterpret_cast<uint4*>(O.rec + (int64_t)g * kG8RecBytes);
+    for (int i = lane; i < kG8RecBytes / 16; i += 32) __stcg(dst + i, reinterpret_cast<const uint4*>(scratch)[i]);
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) atomicAdd(O.ready, 1);
+    __syncwarp();  // the scratch is free again
+}
 
-// Byte offsets of a consumer lane's data inside a stage, fixed for the
-// whole kernel: its four rows i = 2 rt + h of the warp's 32.
+// ---- consumer layout --------------------------------------------------------------
+// Consumer warp w works on the 64 rows 64 rb .. 64 rb + 63 of every tile
+// (rb = w & 3) and on half of every chunk's groups (gh = w >> 2: local
+// groups gh C/2 .. gh C/2 + C/2 - 1), so that each record is read by four
+// warps, not eight.  Lane (g, t) takes part in MMA rows g and g + 8 of the
+// warp's four 16-row MMA tiles rt: 8-row blocks i = 2 rt (rows g) and
+// i = 2 rt + 1 (rows g + 8), tile row 64 rb + 8 i + k7 with
+// k7 = 2 (g & 3) + (g >> 2).  The eight lane groups of a block differ in
+// row & 7 = k7, which keeps the 128-byte-swizzled weight loads free of bank
+// conflicts, and block i of a lane is block 0 plus i x 8 rows: a constant
+// offset.
+__device__ __forceinline__ int lane_k7(int g) { return 2 * (g & 3) + (g >> 2); }
+
+// Byte offsets of block 0 of a consumer lane's rows inside a stage.
 struct LaneOff {
-    uint32_t w2[4][4];  // 2-bit weights of row i, group gi (128-byte swizzle applied)
-    uint32_t w3[4];     // 3-bit weights of row i, group 0 (group gi: + 48 gi)
-    uint32_t sc[4];     // scales of row i, column 0
+    uint32_t w2[2];  // 2-bit: local group 2 gh + q (128-byte swizzle applied), + 8 (t & 1)
+    uint32_t w3;     // 3-bit: local group gh, + 12 t
+    uint32_t sc;     // scales, column 0
 };
 
-__device__ __forceinline__ LaneOff lane_offsets(int w, int g, int t) {
+__device__ __forceinline__ LaneOff lane_offsets(int rb, int gh, int g, int t) {
     LaneOff o;
+    const int k7 = lane_k7(g), r = 64 * rb + k7;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = tile_row(w, i >> 1, i & 1, g);
-#pragma unroll
-        for (int gi = 0; gi < 4; ++gi)
-            o.w2[i][gi] = (uint32_t)(r * 128 + (((2 * gi + (t >> 1)) ^ (r & 7)) << 4) + 8 * (t & 1));
-        o.w3[i] = (uint32_t)(r * 96 + 12 * t);
-        o.sc[i] = (uint32_t)(kSOff + r * 16);
-    }
+    for (int q = 0; q < 2; ++q)
+        o.w2[q] = (uint32_t)(r * 128 + (((2 * (2 * gh + q) + (t >> 1)) ^ k7) << 4) + 8 * (t & 1));
+    o.w3 = (uint32_t)(r * 96 + 48 * gh + 12 * t);
+    o.sc = (uint32_t)(kSOff + r * 16);
     return o;
 }
 
-// One chunk of C groups (geff of them present) for the lane's four rows.
+// The warp's groups of one chunk (geff groups present; `recs` holds the
+// chunk's records in order) for the lane's eight row blocks.
 template <int KIND>
-__device__ __forceinline__ void g8_chunk(const uint8_t* stage, const LaneOff& o, int geff, int scol, int lane, int t,
-                                         float (&acc)[4]) {
-    constexpr int C = KIND ? 2 : 4;
-    // the chunk's scales of the lane's rows: C consecutive bf16 of the staged 8 (aligned to C)
-    uint32_t sv[4][C / 2];
+__device__ __forceinline__ void g8_chunk(const uint8_t* stage, const uint8_t* recs, const LaneOff& o, int geff,
+                                         int gh, int scol, int lane, int t, float (&acc)[8]) {
+    constexpr int C = KIND ? 2 : 4, CW = C / 2, WROW = KIND ? 96 * 8 : 128 * 8;
+    const int gl0 = gh * CW;
+    if (gl0 >= geff) return;  // the ragged end of a row: this half has no group
+    // the scales of the warp's groups, per row block (2-bit: two bf16 in one word; 3-bit: one, as fp32 bits)
+    uint32_t sv[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if (C == 4) {
-            const uint2 v = *reinterpret_cast<const uint2*>(stage + o.sc[i] + 2 * scol);
-            sv[i][0] = v.x;
-            sv[i][C / 2 - 1] = v.y;
-        } else {
-            sv[i][0] = *reinterpret_cast<const uint32_t*>(stage + o.sc[i] + 2 * scol);
-        }
+    for (int i = 0; i < 8; ++i) {
+        const uint8_t* p = stage + o.sc + 128 * i + 2 * (scol + gl0);
+        sv[i] = KIND ? (uint32_t)*reinterpret_cast<const uint16_t*>(p) << 16 : *reinterpret_cast<const uint32_t*>(p);
     }
 #pragma unroll
-    for (int gi = 0; gi < C; ++gi) {
-        if (gi >= geff) break;  // only the ragged end of a row has fewer groups
-        const uint8_t* rec = stage + kROff + gi * kG8RecBytes;
+    for (int q = 0; q < CW; ++q) {
+        if (gl0 + q >= geff) break;
+        const uint8_t* rec = recs + (gl0 + q) * kG8RecBytes;
         const uint4 B0 = *reinterpret_cast<const uint4*>(rec + 16 * lane);
         const uint4 B1 = *reinterpret_cast<const uint4*>(rec + 512 + 16 * lane);
         const uint4 H = *reinterpret_cast<const uint4*>(rec + 1024 + 16 * t);
         const float et = __uint_as_float(H.z);
+        const uint8_t* wb = stage + (KIND ? o.w3 : o.w2[q]);
 #pragma unroll
-        for (int rt = 0; rt < 2; ++rt) {
+        for (int rt = 0; rt < 4; ++rt) {
             uint32_t R[2][8];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int i = 2 * rt + h;
+                const uint8_t* p = wb + (2 * rt + h) * WROW;
                 if (KIND == 0) {
-                    const uint2 v = *reinterpret_cast<const uint2*>(stage + o.w2[i][gi]);
+                    const uint2 v = *reinterpret_cast<const uint2*>(p);
                     decode2(v.x, v.y, R[h]);
                 } else {
-                    const uint32_t* p = reinterpret_cast<const uint32_t*>(stage + o.w3[i] + 48 * gi);
-                    decode3(p[0], p[1], p[2], R[h]);
+                    const uint32_t* w = reinterpret_cast<const uint32_t*>(p);
+                    decode3(w[0], w[1], w[2], R[h]);
                 }
             }
             int d[4] = {(int)H.x, (int)H.y, (int)H.x, (int)H.y};
@@ -319,9 +397,9 @@ __device__ __forceinline__ void g8_chunk(const uint8_t* stage, const LaneOff& o,
             mma_u8s8(d, R[0][6], R[1][6], R[0][7], R[1][7], B1.z, B1.w);
             // digit columns 2t, 2t+1 joined (|value| < 2^30), converted once
             const float p0 = (float)(d[0] + 128 * d[1]), p1 = (float)(d[2] + 128 * d[3]);
-            const uint32_t w0 = sv[2 * rt][gi >> 1], w1 = sv[2 * rt + 1][gi >> 1];
-            const float s0 = __uint_as_float((gi & 1) ? (w0 & 0xFFFF0000u) : (w0 << 16));
-            const float s1 = __uint_as_float((gi & 1) ? (w1 & 0xFFFF0000u) : (w1 << 16));
+            const uint32_t w0 = sv[2 * rt], w1 = sv[2 * rt + 1];
+            const float s0 = __uint_as_float(KIND || q == 0 ? w0 << (KIND ? 0 : 16) : w0 & 0xFFFF0000u);
+            const float s1 = __uint_as_float(KIND || q == 0 ? w1 << (KIND ? 0 : 16) : w1 & 0xFFFF0000u);
             acc[2 * rt] = fmaf(s0 * et, p0, acc[2 * rt]);
             acc[2 * rt + 1] = fmaf(s1 * et, p1, acc[2 * rt + 1]);
         }
@@ -334,96 +412,159 @@ __device__ __forceinline__ void store_y(const G8Item& I, int64_t row, float v) {
     else static_cast<__nv_bfloat16*>(I.Y)[row] = __float2bfloat16_rn(v);
 }
 
-// The gated MLP input for a warp's 32 rows of a tile of the gate/up pair:
-// each of the two items, once its final values are written, publishes them
-// in fp32; the second to arrive computes h = bf16(silu(gate) * up).
-__device__ __forceinline__ void pair_epilogue(const G8Launch& L, int item, uint32_t tile, int w, int64_t row, float v) {
+// The gated MLP input for one row of the gate/up pair: the gate's final
+// value is published as a flagged word; the up item's, once final, waits for
+// it and writes h = bf16(silu(gate) * up), then clears the word.
+__device__ __forceinline__ void pair_epilogue(const G8Launch& L, int item, int64_t row, float v) {
     const int which = item - L.pair_first;  // 0: gate, 1: up
-    if (L.pair_first < 0 || which < 0 || which > 1) return;
-    const int64_t N = L.it[item].N;
-    const int lane = threadIdx.x & 31;
-    if (row < N) __stcg(L.pair_vals + which * N + row, v);
-    __threadfence();
-    __syncwarp();
-    int second = 0;
-    if (lane == 0) second = atomicAdd(L.pair_counters + (int64_t)tile * kCWarps + w, 1) == 1;
-    second = __shfl_sync(0xffffffffu, second, 0);
-    if (!second) return;
-    __threadfence();
-    if (row < N) {
-        const float other = __ldcg(L.pair_vals + (1 - which) * N + row);
-        const float g = which == 0 ? v : other, u = which == 0 ? other : v;
-        L.h[row] = __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.f + expf(-g)) * u));
-    }
-}
-
-// End of a warp's segment of a tile (its 32 rows): write y, or hand the
-// partial sums over and combine them if this CTA arrives last.  The
-// contributors are the owners of the tile's first and last chunk starts;
-// every CTA between them owns at least one (the quota is at least one
-// chunk's cost).
-__device__ __noinline__ void g8_flush(const G8Launch& L, int cta, int w, int item, uint32_t tile, bool whole,
-                                      bool first_seg, float a0, float a1, float a2, float a3) {
-    const G8Item& I = L.it[item];
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    float v[4] = {a0, a1, a2, a3};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {  // the quad's digit pairs; the same sum in all four lanes
-        v[i] += __shfl_xor_sync(0xffffffffu, v[i], 1);
-        v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);
-    }
-    const float mine = t == 0 ? v[0] : (t == 1 ? v[1] : (t == 2 ? v[2] : v[3]));
-    const int rin = tile_row(w, t >> 1, t & 1, g);  // 32 lanes, 32 distinct rows
-    const int64_t row0 = (int64_t)tile * kG8TileRows;
-    if (whole) {
-        store_y(I, row0 + rin, mine);
-        pair_epilogue(L, item, tile, w, row0 + rin, mine);
+    if (L.pair_first < 0 || which < 0 || which > 1 || row >= L.it[item].N) return;
+    uint64_t* slot = L.pair_slots + row;
+    if (which == 0) {
+        st_word(slot, flagged(v));
         return;
     }
-    __stcg(L.partials + ((int64_t)cta * 2 + (first_seg ? 0 : 1)) * kG8TileRows + rin, mine);
-    __threadfence();
-    __syncwarp();
-    const uint32_t uc = (uint32_t)I.unit_cost;
-    const uint32_t pA = (uint32_t)I.cost_base + tile * (uint32_t)I.G * uc;
-    const uint32_t pZ = pA + (uint32_t)(I.cpt - 1) * (uint32_t)I.C * uc;
-    const uint32_t c0 = part_owner(pA, L.Q), c1 = part_owner(pZ, L.Q);
-    int last = 0;
-    if (lane == 0) last = atomicAdd(L.counters + ((int64_t)I.tile_base + tile) * kCWarps + w, 1) == (int)(c1 - c0);
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (!last) return;
-    __threadfence();
-    const uint32_t cA = (uint32_t)I.chunk_base + tile * (uint32_t)I.cpt;
-    float sum = 0.f;
-    for (uint32_t c = c0; c <= c1; ++c) {
-        // a CTA that starts inside this tile has it as its first segment (slot 0), an earlier one as its last
-        const uint32_t cb = part_first_chunk(L.it, L.n_items, c * L.Q);
-        sum += __ldcg(L.partials + ((int64_t)c * 2 + (cb >= cA ? 0 : 1)) * kG8TileRows + 32 * w + lane);
+    float g;
+    if (!wait_word(slot, L.wait_cycles, &g)) {
+        atomicAdd(&g_g8_timeouts, 1u);
+        g = __int_as_float(0x7FC00000);
     }
-    store_y(I, row0 + 32 * w + lane, sum);
-    pair_epilogue(L, item, tile, w, row0 + 32 * w + lane, sum);
+    st_word(slot, 0);
+    L.h[row] = __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.f + expf(-g)) * v));
+}
+
+// How a range's segment of a tile ends: the whole tile (write y); a later
+// part of a tile begun by an earlier range (publish); or the beginning of a
+// tile that later ranges finish (combine).
+enum SegKind { kWhole = 0, kPublish = 1, kCombine = 2 };
+
+// One row's end of segment (its sum over this range's chunks of the tile).
+__device__ __forceinline__ void finish_row(const G8Launch& L, int cta, int item, uint32_t tile, int kind, int rin,
+                                           uint32_t c1, float sum) {
+    if (kind == kPublish) {
+        st_word(L.pslots + (int64_t)cta * kG8TileRows + rin, flagged(sum));
+        return;
+    }
+    if (kind == kCombine) {  // the later ranges that read this tile, in order
+        for (uint32_t c = (uint32_t)cta + 1; c <= c1; ++c) {
+            uint64_t* slot = L.pslots + (int64_t)c * kG8TileRows + rin;
+            float p;
+            if (!wait_word(slot, L.wait_cycles, &p)) {
+                atomicAdd(&g_g8_timeouts, 1u);
+                p = __int_as_float(0x7FC00000);
+            }
+            st_word(slot, 0);
+            sum += p;
+        }
+    }
+    const int64_t row = (int64_t)tile * kG8TileRows + rin;
+    store_y(L.it[item], row, sum);
+    pair_epilogue(L, item, row, sum);
+}
+
+// End of a warp's segment of a tile: the quad's digit pairs are summed, the
+// group half gh = 1 hands its sums to gh = 0 through shared memory (double
+// buffered by `flip`), which adds them (gh 0 + gh 1) and finishes the rows.
+struct Acc8 {
+    float v[8];
+};
+
+__device__ __noinline__ void g8_flush(const G8Launch& L, int cta, int rb, int gh, int item, uint32_t tile, int kind,
+                                      const Acc8 acc, float* pairbuf, int flip) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // the same sum in all four lanes of the quad
+        v[i] = acc.v[i] + __shfl_xor_sync(0xffffffffu, acc.v[i], 1);
+        v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);
+    }
+    // lane t keeps blocks 2t and 2t + 1
+    float m0 = v[0], m1 = v[1];
+#pragma unroll
+    for (int q = 1; q < 4; ++q)
+        if (t == q) {
+            m0 = v[2 * q];
+            m1 = v[2 * q + 1];
+        }
+    float* pb = pairbuf + flip * kG8TileRows + rb * 64 + 2 * lane;
+    if (gh == 1) {
+        pb[0] = m0;
+        pb[1] = m1;
+    }
+    named_sync(2 + rb, 64);
+    if (gh == 1) return;
+    m0 += pb[0];
+    m1 += pb[1];
+    const G8Item& I = L.it[item];
+    uint32_t c1 = 0;
+    if (kind == kCombine) {
+        const uint32_t uc = (uint32_t)I.unit_cost;
+        c1 = part_owner((uint32_t)I.cost_base + tile * (uint32_t)I.G * uc + (uint32_t)(I.cpt - 1) * (uint32_t)I.C * uc,
+                        L.Q);
+    }
+    const int rin = 64 * rb + 16 * t + lane_k7(g);  // block 2t; block 2t + 1 is 8 rows on
+    finish_row(L, cta, item, tile, kind, rin, c1, m0);
+    finish_row(L, cta, item, tile, kind, rin + 8, c1, m1);
+}
+
+// The range's record slots (part_rec_slots), one item per lane of a warp.
+__device__ __forceinline__ void record_slots(const G8Launch& L, uint32_t cb, uint32_t ce, RecSlots* rs) {
+    const int lane = threadIdx.x & 31;
+    int32_t lo = 0, cnt = 0, owner = -1 - lane;
+    if (lane < L.n_items) {
+        part_group_window(L.it[lane], cb, ce, &lo, &cnt);
+        if (cnt > 0) owner = L.it[lane].owner;
+    }
+    // the first earlier item with the same set and window, if any
+    int share = -1;
+    for (int j = 0; j < kMaxItems; ++j) {
+        const int oj = __shfl_sync(0xffffffffu, owner, j), lj = __shfl_sync(0xffffffffu, lo, j),
+                  cj = __shfl_sync(0xffffffffu, cnt, j);
+        if (share < 0 && j < lane && oj == owner && lj == lo && cj == cnt) share = j;
+    }
+    // slots: an inclusive scan of the counts of the items that take their own
+    int own = share < 0 ? cnt : 0, scan = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, scan, o);
+        if (lane >= o) scan += v;
+    }
+    int base = scan - own;
+    const int shared_base = __shfl_sync(0xffffffffu, base, share < 0 ? lane : share);
+    if (share >= 0) base = shared_base;
+    if (lane < kMaxItems) {
+        rs->base[lane] = base;
+        rs->g_lo[lane] = lo;
+        rs->count[lane] = cnt;
+    }
+    if (lane == 31) rs->total = scan;
 }
 
 __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__ G8Launch L) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], built;
+    __shared__ int producer_failed;  // set before the producer completes stages it could not fill
+    __shared__ RecSlots rs;          // the range's record slots (local records)
+    __shared__ float pairbuf[2 * kG8TileRows];  // row sums handed between the two halves of a row block
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
     const uint32_t raw = saddr(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // stages on 1 KB boundaries
+    uint8_t* cache = base + kCache;
     const uint32_t base_s = saddr(base);
+    const uint32_t cb = L.range[cta].cb, ce = L.range[cta].ce;
+    const int32_t n = cb < ce ? (int32_t)(ce - cb) : 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            bar_init(saddr(&full[s]), 1);
+            bar_init(saddr(&full[s]), 1);  // the producer's arrival (after its byte counts)
             bar_init(saddr(&empty[s]), kCWarps);
         }
+        bar_init(saddr(&built), kCWarps);  // every consumer warp has published its workspace records
+        producer_failed = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (warp == 0 && L.local_records) record_slots(L, cb, ce, &rs);
     __syncthreads();  // the only CTA-wide barrier
-
-    uint32_t cb, ce;
-    part_chunk_range(L.it, L.n_items, (uint32_t)cta, L.Q, L.Ctot, &cb, &ce);
-    const int32_t n = cb < ce ? (int32_t)(ce - cb) : 0;
 
     // cursor over the chunks of [cb, ce)
     struct Cur {
@@ -431,15 +572,7 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
         uint32_t tile;
         int32_t j;
     };
-    auto first_cur = [&]() {
-        Cur c{0, 0, 0};
-        for (int i = 1; i < L.n_items; ++i)
-            if (cb >= (uint32_t)L.it[i].chunk_base) c.item = i;
-        const uint32_t local = cb - (uint32_t)L.it[c.item].chunk_base, cpt = (uint32_t)L.it[c.item].cpt;
-        c.tile = local / cpt;
-        c.j = (int32_t)(local - c.tile * cpt);
-        return c;
-    };
+    auto first_cur = [&]() { return Cur{L.range[cta].item, (uint32_t)L.range[cta].tile, L.range[cta].j}; };
     auto advance = [&](Cur& c) {
         if (++c.j == L.it[c.item].cpt) {
             c.j = 0;
@@ -450,64 +583,173 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
         }
     };
 
-    if (warp == kCWarps) {
-        // ---------------- producer: one thread ----------------
-        if (lane != 0 || n == 0 || L.stall) return;
-        auto geff_of = [&](const Cur& c) { return min(L.it[c.item].C, L.it[c.item].G - c.j * L.it[c.item].C); };
-        // The weights, and the caller's scales, are not written by earlier
-        // work in flight, so they may be requested before the preparation
-        // kernel is waited for; its records and padded scale copies after.
-        auto issue_w = [&](const Cur& c, int k) {  // the stage's byte count, weights (+ caller's scales)
+    if (warp == kProducer) {
+        // ---------------- producer warp ----------------
+        const bool active = n > 0 && !L.stall;
+        const bool ws_records = !L.local_records;
+        auto weights = [&](const Cur& c, int s) {  // lane 0: the chunk's weights (and scales) into stage s
             const G8Item& I = L.it[c.item];
-            const int s = k % kStages;
             const uint32_t st = base_s + s * kStageBytes, bar = saddr(&full[s]);
             const int wb = I.grid == kInt3 ? 96 : 128;
-            const int geff = geff_of(c);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            bar_expect(bar, (uint32_t)(kG8TileRows * wb + kG8TileRows * 16 + geff * kG8RecBytes));
+            bar_expect(bar, (uint32_t)(kG8TileRows * wb + (I.stage_scales ? 0 : kG8TileRows * 16)));
             tma_box(st, &L.wmap[c.item], c.j * wb, (int)(c.tile * kG8TileRows), bar);
-            if (!I.spad) tma_box(st + kSOff, &L.smap[c.item], (c.j * I.C) & ~7, (int)(c.tile * kG8TileRows), bar);
+            if (!I.stage_scales) tma_box(st + kSOff, &L.smap[c.item], (c.j * I.C) & ~7, (int)(c.tile * kG8TileRows), bar);
         };
-        auto issue_r = [&](const Cur& c, int k) {  // the chunk's activation records (+ padded scales)
+        auto to_l2 = [&](const Cur& c) {  // lane 0: the chunk's weights (and scales) into L2
             const G8Item& I = L.it[c.item];
-            const int s = k % kStages;
-            const uint32_t st = base_s + s * kStageBytes, bar = saddr(&full[s]);
-            if (I.spad) tma_box(st + kSOff, &L.smap[c.item], (c.j * I.C) & ~7, (int)(c.tile * kG8TileRows), bar);
-            bulk_copy(st + kROff, I.rec + (int64_t)c.j * I.C * kG8RecBytes, (uint32_t)(geff_of(c) * kG8RecBytes), bar);
+            const int wb = I.grid == kInt3 ? 96 : 128;
+            tma_prefetch_l2(&L.wmap[c.item], c.j * wb, (int)(c.tile * kG8TileRows));
+            if (!I.stage_scales) tma_prefetch_l2(&L.smap[c.item], (c.j * I.C) & ~7, (int)(c.tile * kG8TileRows));
         };
-        const int npre = min(n, kStages);
-        Cur c = first_cur();
-        for (int k = 0; k < npre; ++k, advance(c)) issue_w(c, k);
-        pdl_wait();  // records written and counters cleared by the preparation kernel past this point
-        Cur r = first_cur();
-        for (int k = 0; k < npre; ++k, advance(r)) issue_r(r, k);
-        for (int k = npre; k < n; ++k, advance(c)) {
-            const int s = k % kStages;
-            if (!bar_wait(saddr(&empty[s]), (uint32_t)((k / kStages) - 1) & 1u, L.wait_cycles)) {
-                atomicAdd(&g_g8_timeouts, 1u);
-                // let the copies already issued land (bounded) before the CTA can exit
-                for (int q = max(0, k - kStages); q < k; ++q)
-                    bar_wait(saddr(&full[q % kStages]), (uint32_t)(q / kStages) & 1u, L.wait_cycles);
-                return;
+        // The weights and scales are inputs no earlier kernel in the stream
+        // writes: the first stages are requested at once, before the previous
+        // kernel has finished (when the call may overlap it), and the next
+        // kLookahead chunks into L2, so that memory keeps streaming while the
+        // records are built and the copies into the ring hit L2.
+        Cur pf = first_cur();  // next chunk to request into L2
+        int pf_k = 0;
+        if (active && lane == 0) {
+            for (int i = 0; i < L.n_items; ++i) {
+                prefetch_map(&L.wmap[i]);
+                if (!L.it[i].stage_scales) prefetch_map(&L.smap[i]);
             }
-            issue_w(c, k);
-            issue_r(c, k);
+            for (; pf_k < n && pf_k < kStages; ++pf_k, advance(pf)) weights(pf, pf_k);
+            for (; pf_k < n && pf_k < kStages + kLookahead; ++pf_k, advance(pf)) to_l2(pf);
+        }
+        if (ws_records) pdl_wait();  // the record counters and the records belong to the workspace
+        uint32_t ready_mask = 0;     // record sets seen complete
+        int issued = 0;
+        bool ok = active;
+        if (active) {
+            Cur c = first_cur();
+            for (int k = 0; k < n; ++k, advance(c)) {
+                const int s = k % kStages;
+                const G8Item& I = L.it[c.item];
+                int go = 1;
+                if (lane == 0) {
+                    if (k >= kStages) {
+                        go = bar_wait(saddr(&empty[s]), (uint32_t)((k / kStages) - 1) & 1u, L.wait_cycles);
+                        if (go) {
+                            weights(c, s);
+                            if (pf_k < n) {
+                                to_l2(pf);
+                                ++pf_k;
+                                advance(pf);
+                            }
+                        }
+                    }
+                    if (ws_records && go) {
+                        const G8Owner& O = L.own[I.owner];
+                        if (!(ready_mask >> I.owner & 1u)) {  // every record of the set published?
+                            const long long t0 = clock64();
+                            while (!(go = ld_acquire(O.ready) == O.G) && clock64() - t0 <= L.wait_cycles)
+                                __nanosleep(64);
+                            if (go) {
+                                ready_mask |= 1u << I.owner;
+                                asm volatile("fence.proxy.async.global;" ::: "memory");  // read by the async proxy
+                            }
+                        }
+                        if (go) {
+                            const int geff = min(I.C, I.G - c.j * I.C);
+                            const uint32_t bar = saddr(&full[s]);
+                            bar_expect(bar, (uint32_t)(geff * kG8RecBytes));
+                            bulk_copy(base_s + s * kStageBytes + kROff, O.rec + (int64_t)c.j * I.C * kG8RecBytes,
+                                      (uint32_t)(geff * kG8RecBytes), bar);
+                        }
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, go, 0)) {
+                    if (lane == 0) atomicAdd(&g_g8_timeouts, 1u);
+                    ok = false;
+                    break;
+                }
+                if (I.stage_scales) {  // rows of the scales that a tensor copy cannot address: plain loads
+                    uint16_t* sc = reinterpret_cast<uint16_t*>(base + s * kStageBytes + kSOff);
+                    const int geff = min(I.C, I.G - c.j * I.C), scol = (c.j * I.C) & 7;
+                    for (int rr = lane; rr < kG8TileRows; rr += 32) {
+                        const int64_t row = (int64_t)c.tile * kG8TileRows + rr;
+                        for (int gi = 0; gi < geff; ++gi)
+                            sc[rr * 8 + scol + gi] =
+                                row < I.N ? __ldg(I.scales + row * I.G + c.j * I.C + gi) : (uint16_t)0;
+                    }
+                    // a later tensor copy may overwrite what these generic stores wrote
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
+                __syncwarp();
+                if (lane == 0) bar_arrive(saddr(&full[s]));
+                issued = k + 1;
+            }
+        }
+        if (lane == 0) {
+            // the copies requested (stages beyond `issued` may hold weights only) land before the CTA can exit
+            const int req = active ? max(issued, min(n, kStages)) : 0;
+            if (!ok) {  // complete the phases of the stages requested but not filled, marked as failed
+                producer_failed = 1;
+                for (int q = issued; q < req; ++q) bar_arrive(saddr(&full[q % kStages]));
+            }
+            for (int q = max(0, req - kStages); q < req; ++q)
+                bar_wait(saddr(&full[q % kStages]), (uint32_t)(q / kStages) & 1u, L.wait_cycles);
+            // workspace records: every CTA counts itself done with them once its
+            // consumer warps have published theirs; the last one clears the counters
+            if (ws_records && bar_wait(saddr(&built), 0u, L.wait_cycles) &&
+                atom_add_acq_rel(L.done, 1) == L.nctas - 1) {
+                for (int o = 0; o < L.n_own; ++o) *L.own[o].ready = 0;
+                *L.done = 0;
+            }
         }
         return;
     }
 
-    // ---------------- consumers: warp w owns rows 32w .. 32w+31 of every tile ----------------
-    pdl_wait();  // arrival counters cleared past this point
+    // ---------------- consumers: records, then rows 32w .. 32w+31 of every tile ----------------
     const int w = warp, g = lane >> 2, t = lane & 3;
+    if (L.local_records) {
+        // slots w, w + 8, ... of the range's records: x into L2 now, built once x may be read
+        const uint16_t* xg[kSlotsPerWarp];
+        bool three[kSlotsPerWarp];
+#pragma unroll
+        for (int k = 0; k < kSlotsPerWarp; ++k) {
+            const int s = w + kCWarps * k;
+            xg[k] = nullptr;
+            three[k] = false;
+            if (s >= rs.total) continue;
+            int i = 0;
+            while (!(rs.count[i] > 0 && s >= rs.base[i] && s < rs.base[i] + rs.count[i])) ++i;
+            int gr = rs.g_lo[i] + (s - rs.base[i]);
+            if (gr >= L.it[i].G) gr -= L.it[i].G;
+            xg[k] = L.it[i].x + (int64_t)gr * kGroup;
+            three[k] = L.it[i].grid == kInt3;
+            if (lane == 0) prefetch_l2(xg[k], kGroup * 2);
+        }
+        pdl_wait();  // x may come from the previous kernel in the stream
+        uint2 xr[kSlotsPerWarp];
+#pragma unroll
+        for (int k = 0; k < kSlotsPerWarp; ++k)
+            if (xg[k]) xr[k] = __ldcg(reinterpret_cast<const uint2*>(xg[k]) + lane);
+#pragma unroll
+        for (int k = 0; k < kSlotsPerWarp; ++k)
+            if (xg[k]) make_record(xr[k], three[k], cache + (w + kCWarps * k) * kG8RecBytes);
+        named_sync(1, kCWarps * 32);  // all of the range's records are in place
+    } else {
+        pdl_wait();  // x and the workspace may still be in use by the previous kernel in the stream
+        uint8_t* scratch = cache + w * kG8RecBytes;
+        int o = 0;
+        for (int b = cta + L.nctas * w; b < L.n_build; b += L.nctas * kCWarps) {
+            while (o + 1 < L.n_own && b >= L.own[o + 1].build_base) ++o;
+            publish_record(L.own[o], b - L.own[o].build_base, scratch);
+        }
+        if (lane == 0) bar_arrive(saddr(&built));
+    }
     if (n == 0) return;
-    const LaneOff off = lane_offsets(w, g, t);
+    const int rb = w & 3, gh = w >> 2;
+    const LaneOff off = lane_offsets(rb, gh, g, t);
     Cur c = first_cur();
     // the fields of the item under the cursor, in registers (re-read when it changes)
     int it_C = L.it[c.item].C, it_G = L.it[c.item].G, it_cpt = L.it[c.item].cpt, it_T = L.it[c.item].T;
     bool it_three = L.it[c.item].grid == kInt3;
-    int32_t seg_j = c.j;
-    bool first_seg = true, failed = false;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int it_rbase = L.local_records ? rs.base[c.item] : 0, it_glo = L.local_records ? rs.g_lo[c.item] : 0;
+    bool failed = false;
+    int flip = 0;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
     for (int32_t k = 0; k < n; ++k) {
         const int s = k % kStages;
@@ -516,26 +758,37 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
                 if (lane == 0) atomicAdd(&g_g8_timeouts, 1u);
                 failed = true;  // no result: the rest of the range is written as NaN, the ring is left alone
             }
+            failed = failed || *reinterpret_cast<volatile int*>(&producer_failed) != 0;
         }
         if (!failed) {
             const uint8_t* stage = base + s * kStageBytes;
             const int geff = min(it_C, it_G - c.j * it_C);
             const int scol = (c.j * it_C) & 7;
-            if (it_three) g8_chunk<1>(stage, off, geff, scol, lane, t, acc);
-            else g8_chunk<0>(stage, off, geff, scol, lane, t, acc);
+            const uint8_t* recs = stage + kROff;
+            if (L.local_records) {
+                int d = c.j * it_C - it_glo;  // the chunk's first group in the item's window
+                if (d < 0) d += it_G;
+                recs = cache + (it_rbase + d) * kG8RecBytes;
+            }
+            if (it_three) g8_chunk<1>(stage, recs, off, geff, gh, scol, lane, t, acc);
+            else g8_chunk<0>(stage, recs, off, geff, gh, scol, lane, t, acc);
             __syncwarp();
             if (lane == 0) bar_arrive(saddr(&empty[s]));
         } else {
-            acc[0] = acc[1] = acc[2] = acc[3] = __int_as_float(0x7FC00000);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __int_as_float(0x7FC00000);
         }
-        const int32_t cj_next = c.j + 1;
         const bool more = k + 1 < n;
-        if (cj_next == it_cpt || !more) {
-            g8_flush(L, cta, w, c.item, c.tile, seg_j == 0 && cj_next == it_cpt, first_seg, acc[0], acc[1], acc[2],
-                     acc[3]);
-            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-            first_seg = false;
-            seg_j = 0;
+        if (c.j + 1 == it_cpt || !more) {  // end of the range's segment of this tile
+            const uint32_t first = (uint32_t)L.it[c.item].chunk_base + c.tile * (uint32_t)it_cpt;
+            const int kind = first < cb ? kPublish : (first + (uint32_t)it_cpt > ce ? kCombine : kWhole);
+            Acc8 a8;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a8.v[i] = acc[i];
+            g8_flush(L, cta, rb, gh, c.item, c.tile, kind, a8, pairbuf, flip);
+            flip ^= 1;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
         }
         // advance the cursor (the item's fields are reloaded only when it changes)
         if (++c.j == it_cpt) {
@@ -548,6 +801,10 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
                 it_cpt = L.it[c.item].cpt;
                 it_T = L.it[c.item].T;
                 it_three = L.it[c.item].grid == kInt3;
+                if (L.local_records) {
+                    it_rbase = rs.base[c.item];
+                    it_glo = rs.g_lo[c.item];
+                }
             }
         }
     }
@@ -617,7 +874,8 @@ bool encode_g8_wmap(CUtensorMap* map, const void* packed, int grid, int64_t N, i
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Scales [N][Gp] bf16 (Gp a multiple of 8): box 8 groups x 256 rows.
+// Scales [N][G] bf16 (G a multiple of 8, 16-byte aligned base): box 8
+// groups x 256 rows.
 bool encode_g8_smap(CUtensorMap* map, const uint16_t* scales, int64_t N, int64_t Gp) {
     EncodeFn enc = encoder();
     if (!enc) return false;
@@ -651,15 +909,8 @@ cudaError_t launch_gemv8(const G8Launch& L, bool overlap, cudaStream_t st) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (!prepare_device(dev)) return cudaErrorInvalidDevice;
-    {
-        void* args[] = {const_cast<G8Launch*>(&L)};
-        const int warps_per_cta = kPrepThreads / 32;
-        const unsigned grid = (unsigned)std::max((L.prep_warps + warps_per_cta - 1) / warps_per_cta, 1);
-        e = launch_with_pdl((const void*)k_prep8, args, grid, kPrepThreads, 0, st, overlap);
-        if (e != cudaSuccess) return e;
-    }
     void* args[] = {const_cast<G8Launch*>(&L)};
-    return launch_with_pdl((const void*)k_gemv8, args, (unsigned)L.nctas, kG8Threads, kG8Smem, st, true);
+    return launch_with_pdl((const void*)k_gemv8, args, (unsigned)L.nctas, kG8Threads, kG8Smem, st, overlap);
 }
 
 unsigned int take_g8_timeouts() {

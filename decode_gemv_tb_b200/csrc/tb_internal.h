@@ -29,12 +29,11 @@ cudaError_t launch_linear(const Launch& L, int nt, int ctas, cudaStream_t st);
 size_t linear_smem_bytes(int nt, int scl_stride);
 
 struct G8Launch;
-// Batch-1 GEMV on the integer tensor path (tb_gemv8.cu): preparation kernel
-// (activation records, cleared counters, padded scale copies) + k_gemv8 as
-// its programmatic dependent.  `overlap` also launches the preparation
-// kernel as a programmatic dependent of the previous work.
+// Batch-1 GEMV on the integer tensor path (tb_gemv8.cu): one kernel,
+// k_gemv8.  `overlap` launches it as a programmatic dependent of the
+// previous work (it streams weights before that work has finished).
 cudaError_t launch_gemv8(const G8Launch& L, bool overlap, cudaStream_t st);
-// weights of one matrix (box: one chunk x 256 rows) / its scales [N][Gp]
+// weights of one matrix (box: one chunk x 256 rows) / its scales [N][G] (G % 8 == 0)
 bool encode_g8_wmap(CUtensorMap* map, const void* packed, int grid, int64_t N, int64_t K);
 bool encode_g8_smap(CUtensorMap* map, const uint16_t* scales, int64_t N, int64_t Gp);
 // groups per chunk (4 for the 2-bit container, 2 for 3 bits)

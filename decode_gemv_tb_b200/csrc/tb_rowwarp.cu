@@ -1,7 +1,7 @@
 // tb_rowwarp.cu -- batch-1 GEMV in a single launch, one warp per output row:
 // the 5-trits-per-byte ternary layout (every size), and the 2-bit container
 // and 3-bit planes for problems small enough that the stream-K path's fixed
-// cost (preparation kernel, dependent launch, split-tile combine) would
+// cost (activation records, pipeline ramp, split-tile combine) would
 // dominate.  y[n] = sum_j s[n][j] * sum_{k in group j} c[n][k] x[k].
 //
 // ThinkBit page "ThinkBit은 2비트 양자화에서 추론 능력 보존을 추론 평가로

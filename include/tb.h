@@ -169,33 +169,45 @@ TB_API tb_status_t tb_pack(const void *W, tb_dtype_t w_dtype, int64_t N, int64_t
 TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int64_t K, int8_t *codes,
                       tb_stream_t stream);
 
-/* Scratch ("workspace") of the products below, by path:
- *   M = 1 (tb_gemv above 2^24 weights, tb_layer_gemv): per call, one
- *     1088-byte activation record per 128-group of x (written by the call's
- *     preparation kernel, then read), a copy of the scales with rows padded
- *     to a multiple of 8 groups when K/128 is not one, eight arrival
- *     counters per 256-row tile and two 256-float partial-sum slots per CTA
- *     (tiles whose K range is split between CTAs are combined in a fixed
- *     order).  Size, device independent:
- *       ceil256(G * 1088) + [G % 8 != 0] ceil256(N * ceil8(G) * 2)
- *         + ceil256(32 * T1) + ceil256(2048 * min(256, T1 * ceil(G / 2)))
- *     with G = K/128 and T1 = ceil(N / 256).  (The row kernel behind small
- *     tb_gemv calls uses none of it.)
+/* Scratch ("workspace") of the products below.  A call's scratch is of two
+ * kinds: CONTROL words (arrival and completion counters), which must be
+ * zero when a call starts and which every completed call leaves zero; and
+ * DATA, which a call overwrites before it reads it.  Control words sit at
+ * the front of the workspace, data at its back (ending at
+ * workspace_bytes rounded down to 256), and each call asks for
+ *       2 * max(control bytes, data bytes),
+ * so that calls of any shapes and paths can share one workspace sized for
+ * the largest of them: no call's data reaches another call's control words.
+ * By path:
+ *   M = 1 (tb_gemv above 2^24 weights, tb_layer_gemv, tb_gate_up_silu):
+ *     control: per CTA 256 flagged partial-sum words (tiles whose K range
+ *       is split between CTAs are combined in a fixed order by the CTA that
+ *       reads the tile's start) and one 256-byte block of record counters:
+ *         ceil256(2048 * min(256, T1 * ceil(G / 2))) + 256;
+ *     data: the activation records of x (1088 bytes per 128-group, built
+ *       once per call when a CTA's own records do not fit in its shared
+ *       memory):
+ *         ceil256(1088 * G);
+ *     with G = K/128 and T1 = ceil(N / 256).  tb_layer_workspace_bytes: the
+ *     chunks of all items, the records of each distinct (x, code width);
+ *     tb_gate_up_workspace_bytes adds ceil256(8 N) to the control words.
+ *     (The row kernel behind small tb_gemv calls uses none of it.)
  *   2 <= M < 32: none (the kernel reads X as it is); the size is reported
  *     as 256.
- *   M >= 32 (the tensor-core path): X copied per group into the MMA's
- *     layout, the scales transposed per 128-row tile, a counter per tile and
- *     the K-split partial sums:
- *       ceil256(G * NP * 256) + ceil256(T * G * 256) + ceil256(4 * T)
- *         + [S > 1] ceil256(T * S * NP * 512)
- *     with NP = M rounded up to 16, T = ceil(N / 128) and S = the K split,
- *     max(1, min(floor((296 + T/2) / T), 16, G)).
+ *   M >= 32 (the tensor-core path), data only: X copied per group into the
+ *     MMA's layout, the scales transposed per 128-row tile, a counter per
+ *     tile (cleared by the call itself) and the K-split partial sums,
+ *       D = ceil256(G * NP * 256) + ceil256(T * G * 256) + ceil256(4 * T)
+ *         + [S > 1] ceil256(T * S * NP * 512),
+ *     size 2 D, with NP = M rounded up to 16, T = ceil(N / 128) and S = the
+ *     K split, max(1, min(floor((296 + T/2) / T), 16, G)).
  *   M > 64: the larger of the sizes for 64 and for M mod 64 (when not 0).
  * The workspace is
- *   - device memory, 256-byte aligned, at least the size returned here;
+ *   - device memory, 256-byte aligned, at least the size returned here (for
+ *     every call that uses it), ZERO-FILLED ONCE when allocated, and again
+ *     after a call that reported TB_ERR_TIMEOUT;
  *   - owned by the caller, written by every call: two calls that share a
- *     workspace must be ordered (e.g. the same stream); every call clears
- *     what must start at zero;
+ *     workspace must be ordered (e.g. the same stream);
  *   - no other state is kept between calls.
  * Returns 0 for bad arguments. */
 TB_API size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K); /* tb_gemv: M = 1; tb_gemm: its M */
@@ -278,9 +290,16 @@ typedef struct {
  * returns TB_ERR_TIMEOUT.  Nothing faults and the context stays usable. */
 #define TB_FLAG_TEST_STALL 0x80000000u
 
+/* Test hook: the batch-1 kernel builds every activation record once, in
+ * the workspace, even when each CTA's records would fit in its shared
+ * memory (the path that large ranges take).  Results are bitwise those of
+ * the default path. */
+#define TB_FLAG_TEST_WORKSPACE_RECORDS 0x40000000u
+
 /* Workspace bytes of tb_layer_gemv for these items (0 for bad arguments):
- * the batch-1 size above summed over the items, with the counters and
- * partial-sum slots counted once for all of them. */
+ * the batch-1 rule above over all items together -- the tiles and chunks of
+ * every item, the records of each distinct (x, code width) -- or 256 when
+ * every item is in TB_GRID_TERNARY_B3. */
 TB_API size_t tb_layer_workspace_bytes(const tb_linear_t *items, int n_items);
 
 /* Mixed-grid grouped GEMV: every item is an independent y = W x with its
@@ -289,7 +308,8 @@ TB_API size_t tb_layer_workspace_bytes(const tb_linear_t *items, int n_items);
  * own grid; ThinkBit page, 무엇과 다른가: grids chosen per layer).
  *   items      HOST array of n_items descriptors (read before returning).
  *   n_items    1 .. TB_MAX_LAYER_ITEMS.
- *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS.
+ *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS (test hooks: TB_FLAG_TEST_STALL,
+ *              TB_FLAG_TEST_WORKSPACE_RECORDS).
  *   workspace  tb_layer_workspace_bytes(items, n_items) bytes.
  * Items in TB_GRID_TERNARY_B3 are not part of the grouped launch: each runs
  * its own GEMV launch after it, in the same stream (K <= 57600), and needs
@@ -298,9 +318,9 @@ TB_API size_t tb_layer_workspace_bytes(const tb_linear_t *items, int n_items);
 TB_API tb_status_t tb_layer_gemv(const tb_linear_t *items, int n_items, unsigned flags, void *workspace,
                                  size_t workspace_bytes, tb_stream_t stream);
 
-/* Workspace bytes of tb_gate_up_silu: tb_layer_workspace_bytes of the two
- * items, plus ceil256(8 N) + ceil256(32 ceil(N / 256)) for the pair (0 for
- * bad arguments). */
+/* Workspace bytes of tb_gate_up_silu: the batch-1 rule above for the two
+ * items, with ceil256(8 N) more control bytes for the pair; 0 for bad
+ * arguments. */
 TB_API size_t tb_gate_up_workspace_bytes(const tb_linear_t *gate, const tb_linear_t *up);
 
 /* The gate and up projections of a decoder layer's MLP in one launch, and
@@ -317,7 +337,8 @@ TB_API size_t tb_gate_up_workspace_bytes(const tb_linear_t *gate, const tb_linea
  *              grids have the same code width; y of each is written as for
  *              tb_layer_gemv.
  *   h          [N] bf16, device, written.
- *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS.
+ *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS (test hook:
+ *              TB_FLAG_TEST_WORKSPACE_RECORDS).
  *   workspace  tb_gate_up_workspace_bytes(gate, up) bytes. */
 TB_API tb_status_t tb_gate_up_silu(const tb_linear_t *gate, const tb_linear_t *up, uint16_t *h, unsigned flags,
                                    void *workspace, size_t workspace_bytes, tb_stream_t stream);
@@ -337,10 +358,10 @@ TB_API tb_status_t tb_gate_up_silu(const tb_linear_t *gate, const tb_linear_t *u
  *            TB_NOALLOC_SCRATCH_BYTES per device, inside this library.  A
  *            problem whose tb_workspace_bytes(1, N, K) exceeds that size is
  *            rejected with TB_ERR_UNSUPPORTED before any CUDA call (every
- *            N <= 2^20 with K <= 2^18 and K a multiple of 1024 fits; other
- *            K also stage a padded copy of the scales, N * ceil8(K/128) * 2
- *            bytes).  Nothing has to be cleared by the caller: the call
- *            itself zeroes what must start at zero.
+ *            K <= 2^17 fits, whatever N: the size does not grow with N).
+ *            Nothing has to be cleared by the caller: the array starts
+ *            zeroed (static storage) and every call leaves its control
+ *            words zero again.
  *   setup    the first call on each device (with that device current) looks
  *            up the array's address with cudaGetSymbolAddress and caches it;
  *            make that first call before any stream capture.  A failed

@@ -70,33 +70,44 @@ def test_workspace_sizes(lib):
         # below the tensor-core threshold (32) the kernel reads X as it is: no workspace, a nominal 256
         assert tb.workspace_bytes(M, N, K) == 256
     for M, N, K in ((32, 100, 5120), (33, 17408, 5120), (64, 7, 1024), (64, 40000, 4096)):
-        # tensor-core path: per group NP rows of X (256 bytes each) in the MMA's layout, NP = M rounded
-        # up to 16; the scales transposed per 128-row tile; a counter per tile; K-split partials of
-        # NP x 128 fp32 per tile and split
+        # tensor-core path, data only: per group NP rows of X (256 bytes each) in the MMA's layout,
+        # NP = M rounded up to 16; the scales transposed per 128-row tile; a counter per tile; K-split
+        # partials of NP x 128 fp32 per tile and split; twice that (control words front, data back)
         NP, tiles, G = (M + 15) // 16 * 16, (N + 127) // 128, K // 128
         splits = max(1, min((296 + tiles // 2) // tiles, 16, G))
-        want = (al(G * NP * 256) + al(tiles * G * 128 * 2) + al(4 * tiles) +
+        data = (al(G * NP * 256) + al(tiles * G * 128 * 2) + al(4 * tiles) +
                 (al(tiles * splits * NP * 128 * 4) if splits > 1 else 0))
-        assert tb.workspace_bytes(M, N, K) == want, (M, N, K)
+        assert tb.workspace_bytes(M, N, K) == 2 * data, (M, N, K)
     for N, K in ((1, 128), (256, 1024), (17408, 5120), (100, 1408), (4096, 12288)):
-        # batch 1: one 1088-byte record per 128-group of x, a copy of the scales with rows padded to 8
-        # groups when K/128 is not a multiple of 8, eight counters per 256-row tile, and two 256-float
-        # partial slots per CTA (at most 256 CTAs, at most one per chunk of two groups)
+        # batch 1: control = 256 flagged 8-byte partial words per CTA (at most 256 CTAs, at most one per
+        # chunk of two groups) + one 256-byte block of record counters; data = the activation records
+        # of x (1088 bytes per group); size 2 max(control, data)
         G, tiles = K // 128, (N + 255) // 256
-        spad = al(N * -(-G // 8) * 8 * 2) if G % 8 else 0
         ctas = min(256, tiles * -(-G // 2))
-        assert tb.workspace_bytes(1, N, K) == al(1088 * G) + spad + al(32 * tiles) + al(2048 * ctas)
+        control, data = al(2048 * ctas) + 256, al(1088 * G)
+        assert tb.workspace_bytes(1, N, K) == 2 * max(control, data)
     assert tb.workspace_bytes(0, 8, 128) == 0 and tb.workspace_bytes(1, 8, 100) == 0
     assert tb.workspace_bytes(65537, 8, 128) == 0 and tb.workspace_bytes(1, 0, 128) == 0
-    items = (tb.Linear * 3)()
-    shapes = ((4096, 4096, 2), (1024, 4096, 1), (4096, 12288, 0))  # (N, K, grid)
-    for i, (N, K, grid) in enumerate(shapes):
-        items[i] = tb.Linear(FAKE, FAKE, FAKE, FAKE, N, K, grid, 0)
-    tiles = sum((N + 255) // 256 for N, _, _ in shapes)
+    # a layer: the items together; records once per distinct (x, K, code width)
+    X1, X2 = FAKE, FAKE + 4096
+    shapes = ((4096, 4096, 2, X1), (1024, 4096, 1, X1), (1024, 4096, 0, X1), (4096, 12288, 0, X1),
+              (4096, 4096, 2, X2))  # (N, K, grid, x): k and v share their records, nothing else does
+    items = (tb.Linear * len(shapes))()
+    for i, (N, K, grid, x) in enumerate(shapes):
+        items[i] = tb.Linear(FAKE, FAKE, x, FAKE, N, K, grid, 0)
+    tiles = sum((N + 255) // 256 for N, _, _, _ in shapes)
     # chunks of two 3-bit groups or four 2-bit groups per 256-row tile
-    chunks = sum((N + 255) // 256 * -(-(K // 128) // (2 if grid == 2 else 4)) for N, K, grid in shapes)
-    per = sum(al(1088 * (K // 128)) for _, K, _ in shapes)
-    assert tb.layer_workspace_bytes(items) == per + al(32 * tiles) + al(2048 * min(256, chunks))
+    chunks = sum((N + 255) // 256 * -(-(K // 128) // (2 if grid == 2 else 4)) for N, K, grid, _ in shapes)
+    rec = sum(al(1088 * (K // 128)) for i, (_, K, _, _) in enumerate(shapes) if i != 2)
+    control, data = al(2048 * min(256, chunks)) + 256, rec
+    assert tb.layer_workspace_bytes(items) == 2 * max(control, data)
+    # a layer whose records outweigh its control words
+    wide = (tb.Linear * 2)()
+    wide[0] = tb.Linear(FAKE, FAKE, X1, FAKE, 256, 1 << 17, 1, 0)
+    wide[1] = tb.Linear(FAKE, FAKE, X2, FAKE, 256, 1 << 17, 2, 0)
+    control, data = al(2048 * 256) + 256, 2 * al(1088 * 1024)
+    assert data > control and tb.layer_workspace_bytes(wide) == 2 * data
+
 
 def test_argument_errors_before_launch(lib):
     A = FAKE
@@ -164,7 +175,7 @@ def test_b3_sizes_and_limits(lib, oracle):
         want = N * 16 * math.ceil(26 * (K // 128) / 16)
         assert tb.packed_bytes(B3, N, K) == want == oracle.packed_bytes(B3, N, K)
     assert tb.packed_bytes(B3, 4, 100) == 0
-    A, W = FAKE, 1 << 20
+    A, W = FAKE, 1 << 30  # workspace size, never touched
     big = 128 * 451  # 451 groups of activations do not fit in shared memory
     assert lib.tb_gemv(A, B3, A, A, A, 0, 16, big, A, W, 0) == 4
     assert lib.tb_gemm(A, B3, A, A, big, A, 0, 16, 3, 16, big, A, W, 0) == 4
@@ -191,9 +202,9 @@ def test_binding_fails_loudly_without_library(tmp_path):
 
 
 def test_gate_up_workspace_and_errors(lib):
-    """tb_gate_up_silu: the layer workspace of its two items plus the pair's
-    fp32 values (8 N bytes) and counters (32 per 256-row tile); shape and
-    argument errors before any launch."""
+    """tb_gate_up_silu: the batch-1 rule for its two items with the pair's
+    flagged gate values (8 N bytes of control words); shape and argument
+    errors before any launch."""
     al = lambda b: (b + 255) // 256 * 256
     A, W = FAKE, 1 << 30
     for (N, K, gg, gu) in ((12288, 4096, 2, 0), (17408, 5120, 1, 1), (300, 640, 0, 2)):
@@ -202,8 +213,12 @@ def test_gate_up_workspace_and_errors(lib):
         two[1] = tb.Linear(A, A, A, A, N, K, gu, 0)
         g = ctypes.cast(ctypes.byref(two, 0), ctypes.c_void_p)
         u = ctypes.cast(ctypes.byref(two, ctypes.sizeof(tb.Linear)), ctypes.c_void_p)
-        want = tb.layer_workspace_bytes(two) + al(8 * N) + al(32 * ((N + 255) // 256))
-        assert lib.tb_gate_up_workspace_bytes(g, u) == want
+        G, T = K // 128, (N + 255) // 256
+        chunks = sum(T * -(-G // (2 if gr == 2 else 4)) for gr in (gg, gu))
+        shared = (gg == 2) == (gu == 2)  # same x: one record set when the code widths agree
+        control = al(2048 * min(256, chunks)) + 256 + al(8 * N)
+        data = al(1088 * G) * (1 if shared else 2)
+        assert lib.tb_gate_up_workspace_bytes(g, u) == 2 * max(control, data)
     two = (tb.Linear * 2)()
     two[0] = tb.Linear(A, A, A, A, 64, 1024, 1, 0)
     two[1] = tb.Linear(A, A, A, A, 32, 1024, 1, 0)

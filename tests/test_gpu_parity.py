@@ -454,6 +454,58 @@ def test_layer_overlap_flag_and_shared_workspace(oracle):
                 assert torch.equal(y, alone[L][i]), (flags, L, i)
 
 
+def test_workspace_records_path_bitwise(oracle):
+    """The two ways the batch-1 kernel can hold its activation records --
+    in each CTA's shared memory (the default when they fit) and once in the
+    workspace (forced here by the test hook) -- give the same bits, on a
+    layer whose k and v share one x (one record set for both) and whose
+    items mix the grids."""
+    shapes = synth.qwen3_layer_shapes(512, 1536, kv_dim=128)
+    xs = {K: synth.activations(K, seed=3300 + K).to(DEV) for K in {K for _, _, K in shapes}}
+    items = []
+    for i, (name, N, K) in enumerate(shapes):
+        grid = (tb.INT2, tb.INT3, tb.TERNARY)[i % 3]
+        W = synth.gaussian_weights(N, K, seed=3200 + i).to(DEV)
+        s, p, _ = gpu_quantize(W, grid)
+        x = xs[K] if name in ("k", "v") else synth.activations(K, seed=3400 + i).to(DEV)
+        items.append((p, grid, s, x, torch.empty(N, dtype=torch.float32, device=DEV), N, K))
+    tb.tb_layer_gemv(items)
+    torch.cuda.synchronize()
+    local = [it[4].clone() for it in items]
+    for flags in (tb.FLAG_TEST_WORKSPACE_RECORDS, tb.FLAG_TEST_WORKSPACE_RECORDS | tb.FLAG_OVERLAP_PREVIOUS):
+        for it in items:
+            it[4].fill_(float("nan"))
+        tb.tb_layer_gemv(items, flags=flags)
+        torch.cuda.synchronize()
+        for i, it in enumerate(items):
+            assert torch.equal(it[4], local[i]), (flags, i)
+    assert tb.sync_status() == 0
+
+
+@pytest.mark.parametrize("grid", [tb.INT2, tb.INT3])
+def test_gemv_ranges_beyond_shared_records(oracle, grid):
+    """A tall matrix whose CTA ranges each read more than a tile's worth of
+    groups (K = 8192: 64 groups per row) takes the workspace-record path on
+    its own; sampled rows (tile edges, ends, random) against the oracle and
+    the whole output against the forced path bit for bit."""
+    N, K = 40000, 8192
+    W = synth.gaussian_weights(N, K, seed=3500 + grid)
+    s_ref = oracle.scales_absmax(w_np(W), grid)
+    p_ref, _ = oracle.pack(w_np(W), grid, s_ref)
+    x = synth.activations(K, seed=3600 + grid)
+    rng = np.random.default_rng(grid)
+    rows = np.unique(np.concatenate([[0, 1, N - 1], np.arange(255, N, 256 * 16), rng.integers(0, N, 48)]))
+    y64, yabs = oracle.gemv_rows64(p_ref, grid, s_ref, u16(x), K, rows)
+    pd, sd, xd = to_dev_packed(p_ref), to_dev_bits(s_ref), x.to(DEV)
+    y = torch.empty(N, dtype=torch.float32, device=DEV)
+    tb.tb_layer_gemv([(pd, grid, sd, xd, y, N, K)])
+    y2 = torch.empty_like(y)
+    tb.tb_layer_gemv([(pd, grid, sd, xd, y2, N, K)], flags=tb.FLAG_TEST_WORKSPACE_RECORDS)
+    assert tb.sync_status() == 0
+    assert torch.equal(y, y2)
+    assert_within(y[torch.from_numpy(rows).to(DEV)], y64, yabs, "f32", oracle, f"tall grid {grid}")
+
+
 def test_zz_no_bounded_wait_gave_up():
     """After every test above: no device-side bounded wait (TMA copies,
     tensor-core hand-offs) timed out, so every result above is a real one."""
