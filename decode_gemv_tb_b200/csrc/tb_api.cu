@@ -155,12 +155,11 @@ tb_status_t launch_items(Item* items, int n, int nt, cudaStream_t st) {
 // into equal-cost contiguous ranges, one per CTA.
 //
 // Workspace.  The call's control words -- per CTA 256 flagged partial-sum
-// words, one 256-byte block of record counters, and per row of a gate/up
-// pair one flagged word -- are zero before and after every call and sit at
-// the FRONT of the workspace; its data -- the activation records of every
-// distinct x and code width (1088 bytes per group), used when a CTA's
-// records do not fit in its shared memory -- are overwritten before they
-// are read and sit at the BACK.  A call needs 2 max(control, data) bytes,
+// words, and per row of a gate/up pair one flagged word -- are zero before
+// and after every call and sit at the FRONT of the workspace; its data --
+// the activation records of every distinct x and code width (1088 bytes per
+// group), written by the record kernel -- are overwritten before they are
+// read and sit at the BACK.  A call needs 2 max(control, data) bytes,
 // so calls of different shapes can share one workspace sized for the
 // largest: no call's data ever reaches another call's control words.
 constexpr int64_t kMaxG8Ctas = 256;      // bound of the CTA count (partial-sum words)
@@ -194,7 +193,7 @@ G8Space g8_space(const Item* items, int n, bool pair) {
         if (!shared) sp.data += align256((size_t)(items[j].K / kGroup * kG8RecBytes));
     }
     const int64_t ctas = std::min(kMaxG8Ctas, std::max<int64_t>(chunks, 1));
-    sp.control = align256((size_t)(ctas * kG8Rows * 8)) + 256;  // + record counters and the CTA counter
+    sp.control = align256((size_t)(ctas * kG8Rows * 8));
     if (pair) sp.control += align256((size_t)(items[0].N * 8));
     return sp;
 }
@@ -203,7 +202,7 @@ G8Space g8_space(const Item* items, int n, bool pair) {
 // of equal shape whose outputs also give h = bf16(silu(gate) * up) (only
 // pair_first == 0 with two items is used).
 tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes, bool overlap, bool stall,
-                            cudaStream_t st, int pair_first = -1, uint16_t* h = nullptr, bool ws_records = false) {
+                            cudaStream_t st, int pair_first = -1, uint16_t* h = nullptr) {
     G8Launch L;
     std::memset(&L, 0, sizeof(L));
     const G8Space sp = g8_space(items, n, pair_first >= 0);
@@ -236,9 +235,6 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
     const int64_t ctas_max = std::min(kMaxG8Ctas, std::max<int64_t>(chunk, 1));
     L.pslots = reinterpret_cast<uint64_t*>(ctl);
     ctl += align256((size_t)(ctas_max * kG8Rows * 8));
-    int32_t* small = reinterpret_cast<int32_t*>(ctl);  // record counters [16], then the CTA counter
-    ctl += 256;
-    L.done = small + kMaxItems;
     // activation records: items reading the same x with the same code width share one set
     int32_t n_build = 0;
     for (int j = 0; j < n; ++j) {
@@ -250,7 +246,6 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
             G8Owner& o = L.own[owner];
             o.x = items[j].X;
             o.rec = reinterpret_cast<uint8_t*>(dat);
-            o.ready = small + owner;
             o.G = L.it[j].G;
             o.three = items[j].grid == TB_GRID_INT3 ? 1 : 0;
             o.build_base = n_build;
@@ -283,8 +278,7 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
     L.nctas = (int32_t)nctas;
     L.Ctot = (uint32_t)cost;
     L.Q = (uint32_t)Q;
-    // each CTA's range and its first chunk's place; records in shared memory when every range's fit
-    int32_t most = 0;
+    // each CTA's range and its first chunk's place
     for (int64_t c = 0; c < nctas; ++c) {
         G8Range& r = L.range[c];
         part_chunk_range(L.it, n, (uint32_t)c, L.Q, L.Ctot, &r.cb, &r.ce);
@@ -294,11 +288,7 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
         const uint32_t local = r.cb - (uint32_t)L.it[r.item].chunk_base, cpt = (uint32_t)L.it[r.item].cpt;
         r.tile = (int32_t)(local / cpt);
         r.j = (int32_t)(local - (uint32_t)r.tile * cpt);
-        RecSlots rs;
-        part_rec_slots(L.it, n, r.cb, r.ce, &rs);
-        most = std::max(most, rs.total);
     }
-    L.local_records = most <= kG8RecSlots && !ws_records ? 1 : 0;
     L.stall = stall ? 1 : 0;
     L.wait_cycles = stall ? kTestWaitCycles : kWaitCycles;
     return cuda_status(launch_gemv8(L, overlap, st));
@@ -486,9 +476,7 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
 tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags, void* workspace,
                           size_t workspace_bytes, tb_stream_t stream) {
     if (!items || n_items < 1 || n_items > TB_MAX_LAYER_ITEMS) return TB_ERR_ARG;
-    if ((flags & ~(unsigned)(TB_FLAG_OVERLAP_PREVIOUS | TB_FLAG_TEST_STALL | TB_FLAG_TEST_WORKSPACE_RECORDS)) != 0 ||
-        !workspace)
-        return TB_ERR_ARG;
+    if ((flags & ~(unsigned)(TB_FLAG_OVERLAP_PREVIOUS | TB_FLAG_TEST_STALL)) != 0 || !workspace) return TB_ERR_ARG;
     if (!aligned(workspace, 256)) return TB_ERR_ALIGN;
     Item its[kMaxItems];
     int n_main = 0;
@@ -509,8 +497,7 @@ tb_status_t tb_layer_gemv(const tb_linear_t* items, int n_items, unsigned flags,
     if (n_main > 0) {
         const tb_status_t s = launch_g8_items(its, n_main, workspace, workspace_bytes,
                                               (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0,
-                                              (flags & TB_FLAG_TEST_STALL) != 0, st, -1, nullptr,
-                                              (flags & TB_FLAG_TEST_WORKSPACE_RECORDS) != 0);
+                                              (flags & TB_FLAG_TEST_STALL) != 0, st);
         if (s != TB_OK) return s;
     }
     // items in the 5-trits-per-byte layout: one launch each, after the grouped launch
@@ -536,7 +523,7 @@ size_t tb_gate_up_workspace_bytes(const tb_linear_t* gate, const tb_linear_t* up
 tb_status_t tb_gate_up_silu(const tb_linear_t* gate, const tb_linear_t* up, uint16_t* h, unsigned flags,
                             void* workspace, size_t workspace_bytes, tb_stream_t stream) {
     if (!gate || !up || !h || !workspace) return TB_ERR_ARG;
-    if ((flags & ~(unsigned)(TB_FLAG_OVERLAP_PREVIOUS | TB_FLAG_TEST_WORKSPACE_RECORDS)) != 0) return TB_ERR_ARG;
+    if ((flags & ~(unsigned)TB_FLAG_OVERLAP_PREVIOUS) != 0) return TB_ERR_ARG;
     if (gate->N != up->N || gate->K != up->K) return TB_ERR_SHAPE;
     if (!aligned(workspace, 256) || !aligned(h, 2)) return TB_ERR_ALIGN;
     Item its[2];
@@ -553,7 +540,7 @@ tb_status_t tb_gate_up_silu(const tb_linear_t* gate, const tb_linear_t* up, uint
     }
     if (workspace_bytes < tb_gate_up_workspace_bytes(gate, up)) return TB_ERR_ARG;
     return launch_g8_items(its, 2, workspace, workspace_bytes, (flags & TB_FLAG_OVERLAP_PREVIOUS) != 0, false,
-                           static_cast<cudaStream_t>(stream), 0, h, (flags & TB_FLAG_TEST_WORKSPACE_RECORDS) != 0);
+                           static_cast<cudaStream_t>(stream), 0, h);
 }
 
 }  // extern "C"

@@ -53,7 +53,6 @@ struct Launch {
 // 2^(14 t - F) (64 bytes).
 constexpr int kG8RecBytes = 1088;
 constexpr int kG8Warps = 8;      // consumer warps of k_gemv8
-constexpr int kG8RecSlots = 56;  // records a CTA of k_gemv8 holds in shared memory
 constexpr int kG8TileRows = 256;  // rows of a tile: 8 consumer warps x 32 rows
 
 struct G8Item {
@@ -69,11 +68,11 @@ struct G8Item {
 };
 
 // One set of activation records: those of one x at one code width (items
-// reading the same x with the same width share it), built once per call.
+// reading the same x with the same width share it), built once per call by
+// the record kernel into the workspace.
 struct G8Owner {
     const uint16_t* x;  // [G * 128] bf16
     uint8_t* rec;       // [G] records of kG8RecBytes, 256-byte aligned
-    int32_t* ready;     // records published so far: zero before the call, zero after it
     int32_t G, three;
     int32_t build_base;  // index of its first record in the call's build order
 };
@@ -93,10 +92,6 @@ struct G8Launch {
     int32_t n_items, nctas, n_own, n_build;
     uint32_t Ctot, Q;      // total cost and cost quota per CTA (tb_partition.h)
     G8Range range[kMaxG8Ranges];  // per CTA, from the partition
-    // 1: every CTA builds the records its range reads in shared memory; 0:
-    // the CTAs build each record once, in the workspace (own[], n_build)
-    int32_t local_records;
-    int32_t* done;         // CTAs finished with the workspace records: zero before the call, zero after it
     // [nctas][256] partial sums of split tiles as (fp32 bits, flag 1) words,
     // written by the CTA that reads the tile's end, cleared by the one that
     // reads its start: zero before the call, zero after it

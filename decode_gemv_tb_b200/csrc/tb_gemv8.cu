@@ -74,17 +74,15 @@ constexpr int kCWarps = kG8Warps;                  // consumer warps
 constexpr int kProducer = kCWarps;                 // the producer warp
 constexpr int kG8Threads = (kCWarps + 1) * 32;
 constexpr int kStages = 4;
-constexpr int kLookahead = 8;                      // chunks beyond the ring requested into L2 ahead of their copy
+constexpr int kEarly = kStages;                    // stages filled before the previous kernel has finished
 constexpr int kSOff = 32768;                       // scales box: 256 rows x 8 bf16
 constexpr int kROff = kSOff + 4096;                // records copied from the workspace: up to 4 x 1088 bytes
 constexpr int kStageBytes = 41984;                 // >= kROff + 4 * kG8RecBytes, a multiple of 1 KB
-constexpr int kCache = kStages * kStageBytes;      // record cache (or the builders' scratch)
-constexpr int kG8Smem = kCache + kG8RecSlots * kG8RecBytes + 1024;  // + alignment slack (swizzled boxes: 1 KB)
+constexpr int kG8Smem = kStages * kStageBytes + 1024;  // + alignment slack (swizzled boxes: 1 KB)
+constexpr int kRecWarps = 8;                       // warps of a CTA of the record kernel
 
 static_assert(kROff + 4 * kG8RecBytes <= kStageBytes, "stage layout");
-static_assert(kCWarps * kG8RecBytes <= kG8RecSlots * kG8RecBytes, "scratch");
 static_assert(kG8Smem <= 227 * 1024, "shared memory");
-constexpr int kSlotsPerWarp = (kG8RecSlots + kCWarps - 1) / kCWarps;
 
 // ---- small PTX helpers ------------------------------------------------------
 __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -123,25 +121,11 @@ __device__ __forceinline__ void tma_box(uint32_t dst, const CUtensorMap* map, in
         "l"(map), "r"(x), "r"(y), "r"(bar)
         : "memory");
 }
-// hint: bring the 2-D box at (x, y) of map into L2 (no copy into shared memory)
-__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y) : "memory");
-}
 // 1-D bulk copy global -> shared (no multicast): bytes a multiple of 16, both addresses 16-byte aligned
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
-}
-__device__ __forceinline__ int ld_acquire(const int32_t* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int v) {
-    int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
 }
 // 64-bit words read and written whole (single-copy atomic)
 __device__ __forceinline__ void st_word(uint64_t* p, uint64_t v) {
@@ -307,18 +291,31 @@ __device__ __noinline__ void make_record(const uint2 raw, bool three, uint8_t* r
     }
 }
 
-// Builds record g of set O in this warp's scratch, writes it to the
-// workspace and counts it as published.
-__device__ __noinline__ void publish_record(const G8Owner& O, int g, uint8_t* scratch) {
-    const int lane = threadIdx.x & 31;
-    make_record(__ldcg(reinterpret_cast<const uint2*>(O.x + (int64_t)g * kGroup) + lane), O.three != 0, scratch);
+// The records of a call: warp b of the grid builds record b of the call's
+// build order (set o, group g) in shared memory and writes it to the
+// workspace.  x is requested into L2 at once and read once the previous
+// kernel in the stream has finished; the main kernel, a programmatic
+// dependent of this one, reads the records after this kernel completes.
+__global__ void __launch_bounds__(kRecWarps * 32) k_g8_records(const __grid_constant__ G8Launch L) {
+    __shared__ __align__(16) uint8_t scratch[kRecWarps][kG8RecBytes];
+    pdl_trigger();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x * kRecWarps + warp;
+    if (b >= L.n_build) {
+        pdl_wait();
+        return;
+    }
+    int o = 0;
+    while (o + 1 < L.n_own && b >= L.own[o + 1].build_base) ++o;
+    const G8Owner& O = L.own[o];
+    const int g = b - O.build_base;
+    const uint16_t* xg = O.x + (int64_t)g * kGroup;
+    if (lane == 0) prefetch_l2(xg, kGroup * 2);
+    pdl_wait();  // x may come from the previous kernel in the stream
+    make_record(__ldcg(reinterpret_cast<const uint2*>(xg) + lane), O.three != 0, scratch[warp]);
     __syncwarp();
     uint4* dst = reinterpret_cast<uint4*>(O.rec + (int64_t)g * kG8RecBytes);
-    for (int i = lane; i < kG8RecBytes / 16; i += 32) __stcg(dst + i, reinterpret_cast<const uint4*>(scratch)[i]);
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) atomicAdd(O.ready, 1);
-    __syncwarp();  // the scratch is free again
+    for (int i = lane; i < kG8RecBytes / 16; i += 32) dst[i] = reinterpret_cast<const uint4*>(scratch[warp])[i];
 }
 
 // ---- consumer layout --------------------------------------------------------------
@@ -445,15 +442,25 @@ __device__ __forceinline__ void finish_row(const G8Launch& L, int cta, int item,
         return;
     }
     if (kind == kCombine) {  // the later ranges that read this tile, in order
-        for (uint32_t c = (uint32_t)cta + 1; c <= c1; ++c) {
-            uint64_t* slot = L.pslots + (int64_t)c * kG8TileRows + rin;
-            float p;
-            if (!wait_word(slot, L.wait_cycles, &p)) {
-                atomicAdd(&g_g8_timeouts, 1u);
-                p = __int_as_float(0x7FC00000);
+        for (uint32_t c = (uint32_t)cta + 1; c <= c1; c += 4) {  // four words in flight at a time
+            uint64_t* slot[4];
+            uint64_t wv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                slot[q] = L.pslots + (int64_t)(c + q) * kG8TileRows + rin;
+                wv[q] = c + q <= c1 ? ld_word(slot[q]) : 0;
             }
-            st_word(slot, 0);
-            sum += p;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (c + q > c1) break;
+                float p = __uint_as_float((uint32_t)wv[q]);
+                if (!(wv[q] >> 32) && !wait_word(slot[q], L.wait_cycles, &p)) {
+                    atomicAdd(&g_g8_timeouts, 1u);
+                    p = __int_as_float(0x7FC00000);
+                }
+                st_word(slot[q], 0);
+                sum += p;
+            }
         }
     }
     const int64_t row = (int64_t)tile * kG8TileRows + rin;
@@ -506,51 +513,16 @@ __device__ __noinline__ void g8_flush(const G8Launch& L, int cta, int rb, int gh
     finish_row(L, cta, item, tile, kind, rin + 8, c1, m1);
 }
 
-// The range's record slots (part_rec_slots), one item per lane of a warp.
-__device__ __forceinline__ void record_slots(const G8Launch& L, uint32_t cb, uint32_t ce, RecSlots* rs) {
-    const int lane = threadIdx.x & 31;
-    int32_t lo = 0, cnt = 0, owner = -1 - lane;
-    if (lane < L.n_items) {
-        part_group_window(L.it[lane], cb, ce, &lo, &cnt);
-        if (cnt > 0) owner = L.it[lane].owner;
-    }
-    // the first earlier item with the same set and window, if any
-    int share = -1;
-    for (int j = 0; j < kMaxItems; ++j) {
-        const int oj = __shfl_sync(0xffffffffu, owner, j), lj = __shfl_sync(0xffffffffu, lo, j),
-                  cj = __shfl_sync(0xffffffffu, cnt, j);
-        if (share < 0 && j < lane && oj == owner && lj == lo && cj == cnt) share = j;
-    }
-    // slots: an inclusive scan of the counts of the items that take their own
-    int own = share < 0 ? cnt : 0, scan = own;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, scan, o);
-        if (lane >= o) scan += v;
-    }
-    int base = scan - own;
-    const int shared_base = __shfl_sync(0xffffffffu, base, share < 0 ? lane : share);
-    if (share >= 0) base = shared_base;
-    if (lane < kMaxItems) {
-        rs->base[lane] = base;
-        rs->g_lo[lane] = lo;
-        rs->count[lane] = cnt;
-    }
-    if (lane == 31) rs->total = scan;
-}
-
 __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__ G8Launch L) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], built;
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
     __shared__ int producer_failed;  // set before the producer completes stages it could not fill
-    __shared__ RecSlots rs;          // the range's record slots (local records)
     __shared__ float pairbuf[2 * kG8TileRows];  // row sums handed between the two halves of a row block
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
     const uint32_t raw = saddr(smem_raw);
     uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // stages on 1 KB boundaries
-    uint8_t* cache = base + kCache;
     const uint32_t base_s = saddr(base);
     const uint32_t cb = L.range[cta].cb, ce = L.range[cta].ce;
     const int32_t n = cb < ce ? (int32_t)(ce - cb) : 0;
@@ -559,11 +531,9 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
             bar_init(saddr(&full[s]), 1);  // the producer's arrival (after its byte counts)
             bar_init(saddr(&empty[s]), kCWarps);
         }
-        bar_init(saddr(&built), kCWarps);  // every consumer warp has published its workspace records
         producer_failed = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0 && L.local_records) record_slots(L, cb, ce, &rs);
     __syncthreads();  // the only CTA-wide barrier
 
     // cursor over the chunks of [cb, ce)
@@ -586,7 +556,6 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
     if (warp == kProducer) {
         // ---------------- producer warp ----------------
         const bool active = n > 0 && !L.stall;
-        const bool ws_records = !L.local_records;
         auto weights = [&](const Cur& c, int s) {  // lane 0: the chunk's weights (and scales) into stage s
             const G8Item& I = L.it[c.item];
             const uint32_t st = base_s + s * kStageBytes, bar = saddr(&full[s]);
@@ -595,29 +564,23 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
             tma_box(st, &L.wmap[c.item], c.j * wb, (int)(c.tile * kG8TileRows), bar);
             if (!I.stage_scales) tma_box(st + kSOff, &L.smap[c.item], (c.j * I.C) & ~7, (int)(c.tile * kG8TileRows), bar);
         };
-        auto to_l2 = [&](const Cur& c) {  // lane 0: the chunk's weights (and scales) into L2
-            const G8Item& I = L.it[c.item];
-            const int wb = I.grid == kInt3 ? 96 : 128;
-            tma_prefetch_l2(&L.wmap[c.item], c.j * wb, (int)(c.tile * kG8TileRows));
-            if (!I.stage_scales) tma_prefetch_l2(&L.smap[c.item], (c.j * I.C) & ~7, (int)(c.tile * kG8TileRows));
-        };
         // The weights and scales are inputs no earlier kernel in the stream
-        // writes: the first stages are requested at once, before the previous
-        // kernel has finished (when the call may overlap it), and the next
-        // kLookahead chunks into L2, so that memory keeps streaming while the
-        // records are built and the copies into the ring hit L2.
-        Cur pf = first_cur();  // next chunk to request into L2
+        // writes: the first kEarly stages are requested at once, before the
+        // previous kernel has finished (when the call may overlap it), the
+        // rest of the ring and the records (workspace) once the record kernel
+        // has completed.
+        Cur pf = first_cur();  // next chunk whose weights are requested
         int pf_k = 0;
         if (active && lane == 0) {
             for (int i = 0; i < L.n_items; ++i) {
                 prefetch_map(&L.wmap[i]);
                 if (!L.it[i].stage_scales) prefetch_map(&L.smap[i]);
             }
-            for (; pf_k < n && pf_k < kStages; ++pf_k, advance(pf)) weights(pf, pf_k);
-            for (; pf_k < n && pf_k < kStages + kLookahead; ++pf_k, advance(pf)) to_l2(pf);
+            for (; pf_k < n && pf_k < kEarly; ++pf_k, advance(pf)) weights(pf, pf_k);
         }
-        if (ws_records) pdl_wait();  // the record counters and the records belong to the workspace
-        uint32_t ready_mask = 0;     // record sets seen complete
+        pdl_wait();  // the records: written by the record kernel, the previous one in the stream
+        if (active && lane == 0)
+            for (; pf_k < n && pf_k < kStages; ++pf_k, advance(pf)) weights(pf, pf_k);
         int issued = 0;
         bool ok = active;
         if (active) {
@@ -629,33 +592,15 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
                 if (lane == 0) {
                     if (k >= kStages) {
                         go = bar_wait(saddr(&empty[s]), (uint32_t)((k / kStages) - 1) & 1u, L.wait_cycles);
-                        if (go) {
-                            weights(c, s);
-                            if (pf_k < n) {
-                                to_l2(pf);
-                                ++pf_k;
-                                advance(pf);
-                            }
-                        }
+                        if (go) weights(c, s);
                     }
-                    if (ws_records && go) {
+                    if (go) {
                         const G8Owner& O = L.own[I.owner];
-                        if (!(ready_mask >> I.owner & 1u)) {  // every record of the set published?
-                            const long long t0 = clock64();
-                            while (!(go = ld_acquire(O.ready) == O.G) && clock64() - t0 <= L.wait_cycles)
-                                __nanosleep(64);
-                            if (go) {
-                                ready_mask |= 1u << I.owner;
-                                asm volatile("fence.proxy.async.global;" ::: "memory");  // read by the async proxy
-                            }
-                        }
-                        if (go) {
-                            const int geff = min(I.C, I.G - c.j * I.C);
-                            const uint32_t bar = saddr(&full[s]);
-                            bar_expect(bar, (uint32_t)(geff * kG8RecBytes));
-                            bulk_copy(base_s + s * kStageBytes + kROff, O.rec + (int64_t)c.j * I.C * kG8RecBytes,
-                                      (uint32_t)(geff * kG8RecBytes), bar);
-                        }
+                        const int geff = min(I.C, I.G - c.j * I.C);
+                        const uint32_t bar = saddr(&full[s]);
+                        bar_expect(bar, (uint32_t)(geff * kG8RecBytes));
+                        bulk_copy(base_s + s * kStageBytes + kROff, O.rec + (int64_t)c.j * I.C * kG8RecBytes,
+                                  (uint32_t)(geff * kG8RecBytes), bar);
                     }
                 }
                 if (!__shfl_sync(0xffffffffu, go, 0)) {
@@ -689,56 +634,13 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
             }
             for (int q = max(0, req - kStages); q < req; ++q)
                 bar_wait(saddr(&full[q % kStages]), (uint32_t)(q / kStages) & 1u, L.wait_cycles);
-            // workspace records: every CTA counts itself done with them once its
-            // consumer warps have published theirs; the last one clears the counters
-            if (ws_records && bar_wait(saddr(&built), 0u, L.wait_cycles) &&
-                atom_add_acq_rel(L.done, 1) == L.nctas - 1) {
-                for (int o = 0; o < L.n_own; ++o) *L.own[o].ready = 0;
-                *L.done = 0;
-            }
         }
         return;
     }
 
-    // ---------------- consumers: records, then rows 32w .. 32w+31 of every tile ----------------
+    // ---------------- consumers: rows 64 rb .. 64 rb + 63 of every tile, half the groups ----------------
+    pdl_wait();  // y and the workspace may still be in use by the previous kernels in the stream
     const int w = warp, g = lane >> 2, t = lane & 3;
-    if (L.local_records) {
-        // slots w, w + 8, ... of the range's records: x into L2 now, built once x may be read
-        const uint16_t* xg[kSlotsPerWarp];
-        bool three[kSlotsPerWarp];
-#pragma unroll
-        for (int k = 0; k < kSlotsPerWarp; ++k) {
-            const int s = w + kCWarps * k;
-            xg[k] = nullptr;
-            three[k] = false;
-            if (s >= rs.total) continue;
-            int i = 0;
-            while (!(rs.count[i] > 0 && s >= rs.base[i] && s < rs.base[i] + rs.count[i])) ++i;
-            int gr = rs.g_lo[i] + (s - rs.base[i]);
-            if (gr >= L.it[i].G) gr -= L.it[i].G;
-            xg[k] = L.it[i].x + (int64_t)gr * kGroup;
-            three[k] = L.it[i].grid == kInt3;
-            if (lane == 0) prefetch_l2(xg[k], kGroup * 2);
-        }
-        pdl_wait();  // x may come from the previous kernel in the stream
-        uint2 xr[kSlotsPerWarp];
-#pragma unroll
-        for (int k = 0; k < kSlotsPerWarp; ++k)
-            if (xg[k]) xr[k] = __ldcg(reinterpret_cast<const uint2*>(xg[k]) + lane);
-#pragma unroll
-        for (int k = 0; k < kSlotsPerWarp; ++k)
-            if (xg[k]) make_record(xr[k], three[k], cache + (w + kCWarps * k) * kG8RecBytes);
-        named_sync(1, kCWarps * 32);  // all of the range's records are in place
-    } else {
-        pdl_wait();  // x and the workspace may still be in use by the previous kernel in the stream
-        uint8_t* scratch = cache + w * kG8RecBytes;
-        int o = 0;
-        for (int b = cta + L.nctas * w; b < L.n_build; b += L.nctas * kCWarps) {
-            while (o + 1 < L.n_own && b >= L.own[o + 1].build_base) ++o;
-            publish_record(L.own[o], b - L.own[o].build_base, scratch);
-        }
-        if (lane == 0) bar_arrive(saddr(&built));
-    }
     if (n == 0) return;
     const int rb = w & 3, gh = w >> 2;
     const LaneOff off = lane_offsets(rb, gh, g, t);
@@ -746,30 +648,27 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
     // the fields of the item under the cursor, in registers (re-read when it changes)
     int it_C = L.it[c.item].C, it_G = L.it[c.item].G, it_cpt = L.it[c.item].cpt, it_T = L.it[c.item].T;
     bool it_three = L.it[c.item].grid == kInt3;
-    int it_rbase = L.local_records ? rs.base[c.item] : 0, it_glo = L.local_records ? rs.g_lo[c.item] : 0;
     bool failed = false;
     int flip = 0;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
     for (int32_t k = 0; k < n; ++k) {
         const int s = k % kStages;
-        if (!failed) {
-            if (!__all_sync(0xffffffffu, bar_wait(saddr(&full[s]), (uint32_t)(k / kStages) & 1u, L.wait_cycles))) {
-                if (lane == 0) atomicAdd(&g_g8_timeouts, 1u);
-                failed = true;  // no result: the rest of the range is written as NaN, the ring is left alone
+        if (!failed) {  // one lane waits for the stage; the warp synchronizes with it
+            int ok = 1;
+            if (lane == 0) {
+                ok = bar_wait(saddr(&full[s]), (uint32_t)(k / kStages) & 1u, L.wait_cycles);
+                if (!ok) atomicAdd(&g_g8_timeouts, 1u);
+                ok = ok && *reinterpret_cast<volatile int*>(&producer_failed) == 0;
             }
-            failed = failed || *reinterpret_cast<volatile int*>(&producer_failed) != 0;
+            // no result after a failed wait: the rest of the range is written as NaN, the ring is left alone
+            failed = __shfl_sync(0xffffffffu, ok, 0) == 0;
         }
         if (!failed) {
             const uint8_t* stage = base + s * kStageBytes;
             const int geff = min(it_C, it_G - c.j * it_C);
             const int scol = (c.j * it_C) & 7;
             const uint8_t* recs = stage + kROff;
-            if (L.local_records) {
-                int d = c.j * it_C - it_glo;  // the chunk's first group in the item's window
-                if (d < 0) d += it_G;
-                recs = cache + (it_rbase + d) * kG8RecBytes;
-            }
             if (it_three) g8_chunk<1>(stage, recs, off, geff, gh, scol, lane, t, acc);
             else g8_chunk<0>(stage, recs, off, geff, gh, scol, lane, t, acc);
             __syncwarp();
@@ -801,10 +700,6 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
                 it_cpt = L.it[c.item].cpt;
                 it_T = L.it[c.item].T;
                 it_three = L.it[c.item].grid == kInt3;
-                if (L.local_records) {
-                    it_rbase = rs.base[c.item];
-                    it_glo = rs.g_lo[c.item];
-                }
             }
         }
     }
@@ -904,13 +799,19 @@ int gemv8_ctas() {
     return ctas[dev];
 }
 
+// The record kernel, then the main kernel as its programmatic dependent
+// (it streams weights while the records are built).  `overlap` lets the
+// record kernel, in turn, start before the previous work in the stream ends.
 cudaError_t launch_gemv8(const G8Launch& L, bool overlap, cudaStream_t st) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (!prepare_device(dev)) return cudaErrorInvalidDevice;
     void* args[] = {const_cast<G8Launch*>(&L)};
-    return launch_with_pdl((const void*)k_gemv8, args, (unsigned)L.nctas, kG8Threads, kG8Smem, st, overlap);
+    const unsigned rec_ctas = (unsigned)((L.n_build + kRecWarps - 1) / kRecWarps);
+    e = launch_with_pdl((const void*)k_g8_records, args, rec_ctas, kRecWarps * 32, 0, st, overlap);
+    if (e != cudaSuccess) return e;
+    return launch_with_pdl((const void*)k_gemv8, args, (unsigned)L.nctas, kG8Threads, kG8Smem, st, true);
 }
 
 unsigned int take_g8_timeouts() {

@@ -102,53 +102,4 @@ TB_HD void part_chunk_range(const Item* it, int n, uint32_t w, uint32_t Q, uint3
     *end = part_first_chunk(it, n, hi);
 }
 
-// Groups of item `it` that the chunks [cb, ce) read, as a cyclic window of
-// the item's G groups: [g_lo, g_lo + count) mod G (count 0: none; G: all).
-// Chunks of one tile read consecutive groups; a range shorter than a tile
-// that crosses a tile boundary reads the end of one tile's groups and the
-// start of the next one's.
-template <class Item>
-TB_HD void part_group_window(const Item& it, uint32_t cb, uint32_t ce, int32_t* g_lo, int32_t* count) {
-    const uint32_t b0 = (uint32_t)it.chunk_base, b1 = b0 + (uint32_t)it.T * (uint32_t)it.cpt;
-    const uint32_t a = cb > b0 ? cb : b0, b = ce < b1 ? ce : b1;
-    *g_lo = 0;
-    *count = 0;
-    if (a >= b) return;
-    const uint32_t cpt = (uint32_t)it.cpt;
-    if (b - a >= cpt) {
-        *count = it.G;
-        return;
-    }
-    const int32_t ja = (int32_t)((a - b0) % cpt), jb = (int32_t)((b - 1 - b0) % cpt);
-    const int32_t lo = ja * it.C, hi = (jb + 1) * it.C < it.G ? (jb + 1) * it.C : it.G;
-    *g_lo = lo;
-    *count = ja <= jb ? hi - lo : it.G - lo + hi;
-}
-
-// Slots of a range's activation records: item i's window takes slots
-// [base[i], base[i] + count[i]) in item order, and shares the slots of an
-// earlier item of the same record set with the same window.
-struct RecSlots {
-    int32_t base[16], g_lo[16], count[16];
-    int32_t total;
-};
-
-template <class Item>
-TB_HD void part_rec_slots(const Item* it, int n, uint32_t cb, uint32_t ce, RecSlots* rs) {
-    rs->total = 0;
-    for (int i = 0; i < n; ++i) {
-        int32_t lo, cnt, base = -1;
-        part_group_window(it[i], cb, ce, &lo, &cnt);
-        for (int j = 0; j < i && base < 0 && cnt > 0; ++j)
-            if (it[j].owner == it[i].owner && rs->count[j] == cnt && rs->g_lo[j] == lo) base = rs->base[j];
-        if (base < 0) {
-            base = rs->total;
-            rs->total += cnt;
-        }
-        rs->base[i] = base;
-        rs->g_lo[i] = lo;
-        rs->count[i] = cnt;
-    }
-}
-
 }  // namespace tb

@@ -21,7 +21,6 @@ F32, BF16 = 0, 1
 MAX_LAYER_ITEMS = 16
 FLAG_OVERLAP_PREVIOUS = 1
 FLAG_TEST_STALL = 0x80000000  # test hook: the batch-1 kernel's waits give up (see include/tb.h)
-FLAG_TEST_WORKSPACE_RECORDS = 0x40000000  # test hook: the batch-1 kernel's records go through the workspace
 NOALLOC_SCRATCH_BYTES = 4 << 20  # TB_NOALLOC_SCRATCH_BYTES
 
 STATUS = {0: "TB_OK", 1: "TB_ERR_ARG", 2: "TB_ERR_SHAPE", 3: "TB_ERR_ALIGN", 4: "TB_ERR_UNSUPPORTED", 5: "TB_ERR_CUDA",

@@ -182,11 +182,10 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
  *   M = 1 (tb_gemv above 2^24 weights, tb_layer_gemv, tb_gate_up_silu):
  *     control: per CTA 256 flagged partial-sum words (tiles whose K range
  *       is split between CTAs are combined in a fixed order by the CTA that
- *       reads the tile's start) and one 256-byte block of record counters:
- *         ceil256(2048 * min(256, T1 * ceil(G / 2))) + 256;
+ *       reads the tile's start):
+ *         ceil256(2048 * min(256, T1 * ceil(G / 2)));
  *     data: the activation records of x (1088 bytes per 128-group, built
- *       once per call when a CTA's own records do not fit in its shared
- *       memory):
+ *       once per call by the call's first kernel):
  *         ceil256(1088 * G);
  *     with G = K/128 and T1 = ceil(N / 256).  tb_layer_workspace_bytes: the
  *     chunks of all items, the records of each distinct (x, code width);
@@ -290,12 +289,6 @@ typedef struct {
  * returns TB_ERR_TIMEOUT.  Nothing faults and the context stays usable. */
 #define TB_FLAG_TEST_STALL 0x80000000u
 
-/* Test hook: the batch-1 kernel builds every activation record once, in
- * the workspace, even when each CTA's records would fit in its shared
- * memory (the path that large ranges take).  Results are bitwise those of
- * the default path. */
-#define TB_FLAG_TEST_WORKSPACE_RECORDS 0x40000000u
-
 /* Workspace bytes of tb_layer_gemv for these items (0 for bad arguments):
  * the batch-1 rule above over all items together -- the tiles and chunks of
  * every item, the records of each distinct (x, code width) -- or 256 when
@@ -308,8 +301,7 @@ TB_API size_t tb_layer_workspace_bytes(const tb_linear_t *items, int n_items);
  * own grid; ThinkBit page, 무엇과 다른가: grids chosen per layer).
  *   items      HOST array of n_items descriptors (read before returning).
  *   n_items    1 .. TB_MAX_LAYER_ITEMS.
- *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS (test hooks: TB_FLAG_TEST_STALL,
- *              TB_FLAG_TEST_WORKSPACE_RECORDS).
+ *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS (test hook: TB_FLAG_TEST_STALL).
  *   workspace  tb_layer_workspace_bytes(items, n_items) bytes.
  * Items in TB_GRID_TERNARY_B3 are not part of the grouped launch: each runs
  * its own GEMV launch after it, in the same stream (K <= 57600), and needs
@@ -337,8 +329,7 @@ TB_API size_t tb_gate_up_workspace_bytes(const tb_linear_t *gate, const tb_linea
  *              grids have the same code width; y of each is written as for
  *              tb_layer_gemv.
  *   h          [N] bf16, device, written.
- *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS (test hook:
- *              TB_FLAG_TEST_WORKSPACE_RECORDS).
+ *   flags      0 or TB_FLAG_OVERLAP_PREVIOUS.
  *   workspace  tb_gate_up_workspace_bytes(gate, up) bytes. */
 TB_API tb_status_t tb_gate_up_silu(const tb_linear_t *gate, const tb_linear_t *up, uint16_t *h, unsigned flags,
                                    void *workspace, size_t workspace_bytes, tb_stream_t stream);

@@ -454,40 +454,12 @@ def test_layer_overlap_flag_and_shared_workspace(oracle):
                 assert torch.equal(y, alone[L][i]), (flags, L, i)
 
 
-def test_workspace_records_path_bitwise(oracle):
-    """The two ways the batch-1 kernel can hold its activation records --
-    in each CTA's shared memory (the default when they fit) and once in the
-    workspace (forced here by the test hook) -- give the same bits, on a
-    layer whose k and v share one x (one record set for both) and whose
-    items mix the grids."""
-    shapes = synth.qwen3_layer_shapes(512, 1536, kv_dim=128)
-    xs = {K: synth.activations(K, seed=3300 + K).to(DEV) for K in {K for _, _, K in shapes}}
-    items = []
-    for i, (name, N, K) in enumerate(shapes):
-        grid = (tb.INT2, tb.INT3, tb.TERNARY)[i % 3]
-        W = synth.gaussian_weights(N, K, seed=3200 + i).to(DEV)
-        s, p, _ = gpu_quantize(W, grid)
-        x = xs[K] if name in ("k", "v") else synth.activations(K, seed=3400 + i).to(DEV)
-        items.append((p, grid, s, x, torch.empty(N, dtype=torch.float32, device=DEV), N, K))
-    tb.tb_layer_gemv(items)
-    torch.cuda.synchronize()
-    local = [it[4].clone() for it in items]
-    for flags in (tb.FLAG_TEST_WORKSPACE_RECORDS, tb.FLAG_TEST_WORKSPACE_RECORDS | tb.FLAG_OVERLAP_PREVIOUS):
-        for it in items:
-            it[4].fill_(float("nan"))
-        tb.tb_layer_gemv(items, flags=flags)
-        torch.cuda.synchronize()
-        for i, it in enumerate(items):
-            assert torch.equal(it[4], local[i]), (flags, i)
-    assert tb.sync_status() == 0
-
-
 @pytest.mark.parametrize("grid", [tb.INT2, tb.INT3])
-def test_gemv_ranges_beyond_shared_records(oracle, grid):
-    """A tall matrix whose CTA ranges each read more than a tile's worth of
-    groups (K = 8192: 64 groups per row) takes the workspace-record path on
-    its own; sampled rows (tile edges, ends, random) against the oracle and
-    the whole output against the forced path bit for bit."""
+def test_gemv_ranges_over_several_tiles(oracle, grid):
+    """A tall matrix whose CTA ranges each cover more than one tile (K = 8192:
+    64 groups per row, 157 tiles of 256 rows): sampled rows (tile edges,
+    ends, random) against the oracle, and the output bit for bit against a
+    second launch with programmatic overlap."""
     N, K = 40000, 8192
     W = synth.gaussian_weights(N, K, seed=3500 + grid)
     s_ref = oracle.scales_absmax(w_np(W), grid)
@@ -500,7 +472,7 @@ def test_gemv_ranges_beyond_shared_records(oracle, grid):
     y = torch.empty(N, dtype=torch.float32, device=DEV)
     tb.tb_layer_gemv([(pd, grid, sd, xd, y, N, K)])
     y2 = torch.empty_like(y)
-    tb.tb_layer_gemv([(pd, grid, sd, xd, y2, N, K)], flags=tb.FLAG_TEST_WORKSPACE_RECORDS)
+    tb.tb_layer_gemv([(pd, grid, sd, xd, y2, N, K)], flags=tb.FLAG_OVERLAP_PREVIOUS)
     assert tb.sync_status() == 0
     assert torch.equal(y, y2)
     assert_within(y[torch.from_numpy(rows).to(DEV)], y64, yabs, "f32", oracle, f"tall grid {grid}")
