@@ -445,6 +445,46 @@ def rows_section(dev, stream):
     del items, arr, wsl, flush
     torch.cuda.empty_cache()
 
+    # decode order: per layer q/k/v in one call on one shared x, o, gate/up with
+    # h = bf16(silu(gate) * up) in one call, down on h -- four dependent calls
+    # per layer (TB_FLAG_OVERLAP_PREVIOUS), 8 layers of the 8B-like stack
+    dl, dby = [], 0
+    for li, mats in enumerate(synth.config3_stack()[:8]):
+        P = {}
+        for m in mats:
+            W = synth.gaussian_weights(m.N, m.K, seed=m.seed, device=dev, dtype=torch.bfloat16)
+            sd = tb.tb_scales_absmax(W, m.grid)
+            P[m.name.split(".")[1]] = (tb.tb_pack(W, m.grid, sd), m.grid, sd, m.N, m.K)
+            dby += algo_bytes(m.N, m.K, m.grid)
+            del W
+        xa = synth.activations(4096, seed=9000 + li, device=dev)
+        xo = synth.activations(4096, seed=9100 + li, device=dev)
+        xm = synth.activations(4096, seed=9200 + li, device=dev)
+        y = {k: torch.empty(v[3], dtype=torch.float32, device=dev) for k, v in P.items()}
+        h = torch.empty(P["gate"][3], dtype=torch.bfloat16, device=dev)
+        it = lambda name, x: (P[name][0], P[name][1], P[name][2], x, y[name], P[name][3], P[name][4])
+        qkv = tb.linear_items([it("q", xa), it("k", xa), it("v", xa)])
+        o = tb.linear_items([it("o", xo)])
+        gu = (it("gate", xm), it("up", xm))
+        down = tb.linear_items([it("down", h)])
+        dl.append((qkv, o, gu, h, down))
+    # one workspace for every call (sized for the largest: calls of different shapes may share it)
+    wsd = tb.workspace(max(max(tb.layer_workspace_bytes(a), tb.layer_workspace_bytes(o), tb.layer_workspace_bytes(d),
+                               tb.gate_up_workspace_bytes(gu[0], gu[1])) for a, o, gu, _, d in dl), dev)
+
+    def decode_pass():
+        for qkv, o, gu, h, down in dl:
+            tb.tb_layer_gemv(qkv, wsd, tb.FLAG_OVERLAP_PREVIOUS)
+            tb.tb_layer_gemv(o, wsd, tb.FLAG_OVERLAP_PREVIOUS)
+            tb.tb_gate_up_silu(gu[0], gu[1], h, ws=wsd, flags=tb.FLAG_OVERLAP_PREVIOUS)
+            tb.tb_layer_gemv(down, wsd, tb.FLAG_OVERLAP_PREVIOUS)
+
+    msd = med(decode_pass, reps=5, inner=1)
+    out["decode_order_layer_8b"] = {"us_per_layer": msd * 1e3 / len(dl), "GB_s": dby / msd / 1e6, "layers": len(dl),
+                                    "calls_per_layer": 4, "algorithmic_bytes_per_layer": dby // len(dl)}
+    del dl, wsd
+    torch.cuda.empty_cache()
+
     # config 5: batch-1 GEMV over all 280 matrices of a 40-layer 14B-like stack
     # (outlier weights, mixed grids), packed by the library; one pass = 40 layer calls
     layers, packed5, by5 = [], 0, 0
@@ -597,8 +637,11 @@ def main():
     cur = torch.cuda.current_stream(dev)
 
     # --- device-resident timing (the headline `value`): graph of one step,
-    # every layer called with the default flags
-    g_step = capture(lambda: S.step(0))
+    # every layer called with TB_FLAG_OVERLAP_PREVIOUS (resident weights: a
+    # call streams its weights while the previous one finishes; activations,
+    # outputs and workspace still wait for it)
+    FLAGS = tb.FLAG_OVERLAP_PREVIOUS
+    g_step = capture(lambda: S.step(FLAGS))
     log = args.clocks_log if (args.clocks_log is None or world == 1) else f"{args.clocks_log}.{rank}"
     with Clocks(local, log) as clk:
         ms = time_region(g_step.replay, args.steps, args.warmup, cur, dist, clk)
@@ -611,10 +654,10 @@ def main():
     avg_layer_bytes = S.step_bytes / n_layers
     achieved = avg_layer_bytes / (us_layer * 1e-6) / 1e9
 
-    # ablation: the same step with programmatic overlap between layers
-    g_ovl = capture(lambda: S.step(tb.FLAG_OVERLAP_PREVIOUS))
-    ms_ovl = time_region(g_ovl.replay, args.steps, args.warmup, cur, dist) / args.steps
-    del g_ovl
+    # ablation: the same step without the overlap flag (each call starts after the previous one ends)
+    g_plain = capture(lambda: S.step(0))
+    ms_plain = time_region(g_plain.replay, args.steps, args.warmup, cur, dist) / args.steps
+    del g_plain
 
     # --- end to end through the public API: each step copies every layer's x
     # from pinned host memory, makes the 36 tb_layer_gemv calls (ctypes, argument
@@ -627,7 +670,7 @@ def main():
 
     def e2e_step():
         S.x_all.copy_(x_host, non_blocking=True)
-        S.step(0)
+        S.step(FLAGS)
         y_host.copy_(S.y_all, non_blocking=True)
 
     ms_e2e = time_region(e2e_step, args.steps, args.warmup, cur, dist)
@@ -650,18 +693,19 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(S.stack, world),
             "decoder_layer_us_per_token": us_layer,
-            "decoder_layer_us_per_token_overlap_flag": ms_ovl * 1e3 / n_layers,
+            "flags": "TB_FLAG_OVERLAP_PREVIOUS",
+            "decoder_layer_us_per_token_no_overlap_flag": ms_plain * 1e3 / n_layers,
             "tokens_per_s_equivalent": 1e6 / (us_layer * n_layers),
             "frac_of_spec_8TBs": value / world / SPEC_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": profile_traffic,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
-                         else "fallback 6.65 TB/s", "kernel": "k_gemv8 (one launch per tb_layer_gemv call)"},
+                         else "fallback 6.65 TB/s", "kernel": "k_gemv8 (with its record kernel, one pair per tb_layer_gemv call)"},
             "e2e": {"value": e2e_value, "unit": "GB/s",
                     "h2d_bytes_per_step": S.x_all.numel() * 2, "d2h_bytes_per_step": S.y_all.numel() * 4,
                     "ms_per_step": ms_e2e / args.steps, "calls": "eager: 36 tb_layer_gemv C-ABI calls per step",
                     "graph_value": e2e_graph_value, "graph_ms_per_step": ms_e2e_graph / args.steps},
-            "gpu_launches": n_layers * args.steps,
+            "gpu_launches": 2 * n_layers * args.steps,  # per call: the record kernel and k_gemv8
             "clocks": clocks,
             "us_x_median_sm_ghz_per_layer": (us_layer * clocks["sm_mhz"] / 1e3) if clocks.get("sm_mhz") else None,
             "rows": rows,

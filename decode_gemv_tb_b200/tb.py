@@ -240,6 +240,13 @@ def tb_layer_gemv(items, ws: torch.Tensor | None = None, flags: int = 0, stream:
                                 stream), "tb_layer_gemv")
 
 
+def gate_up_workspace_bytes(gate, up) -> int:
+    """Workspace bytes of tb_gate_up_silu for gate, up: (packed, grid, scales, x, y, N, K)."""
+    arr = linear_items([gate, up])
+    return int(load().tb_gate_up_workspace_bytes(ctypes.cast(ctypes.byref(arr, 0), ctypes.c_void_p),
+                                                  ctypes.cast(ctypes.byref(arr, ctypes.sizeof(Linear)), ctypes.c_void_p)))
+
+
 def tb_gate_up_silu(gate, up, h: torch.Tensor, ws: torch.Tensor | None = None, flags: int = 0,
                     stream: int | None = None) -> torch.Tensor:
     """gate, up: (packed, grid, scales, x, y, N, K) of equal N and K; writes
