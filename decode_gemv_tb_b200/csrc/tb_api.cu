@@ -164,6 +164,11 @@ tb_status_t launch_items(Item* items, int n, int nt, cudaStream_t st) {
 // largest: no call's data ever reaches another call's control words.
 constexpr int64_t kMaxG8Ctas = 256;      // bound of the CTA count (partial-sum words)
 constexpr int64_t kG8Rows = kG8TileRows;
+// Cost of one 128-group of one 256-row tile in the equal-cost split: a
+// 3-bit group takes about twice the consumer work of a 2-bit one (measured
+// on the 8B-like stack), so every chunk (four 2-bit or two 3-bit groups)
+// costs the same
+constexpr int32_t kG8Cost2 = 2, kG8Cost3 = 4;
 constexpr long long kWaitCycles = 4000000000LL;      // about 2 s
 constexpr long long kTestWaitCycles = 20000000LL;    // about 10 ms (TB_FLAG_TEST_STALL)
 
@@ -222,7 +227,7 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
         s.T = (int32_t)g8_tiles(it.N);
         s.C = g8_chunk_groups(it.grid);
         s.cpt = (s.G + s.C - 1) / s.C;
-        s.unit_cost = it.grid == TB_GRID_INT3 ? 3 : 2;
+        s.unit_cost = it.grid == TB_GRID_INT3 ? kG8Cost3 : kG8Cost2;
         s.grid = it.grid;
         s.ydt = it.ydt;
         s.chunk_base = chunk;
@@ -268,10 +273,13 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
     }
     const int resident = gemv8_ctas();
     if (resident <= 0) return TB_ERR_CUDA;
-    // every quota at least one chunk's cost (4 x 2 or 2 x 3): then every CTA
+    // every quota at least one chunk's cost: then every CTA
     // between a tile's first and last owner owns a chunk of it, which the
     // split-tile combine relies on
-    int64_t nctas = std::max<int64_t>(1, std::min<int64_t>({(int64_t)resident, chunk, kMaxG8Ctas, cost / 8}));
+    int64_t max_chunk_cost = 0;
+    for (int j = 0; j < n; ++j) max_chunk_cost = std::max<int64_t>(max_chunk_cost, (int64_t)L.it[j].C * L.it[j].unit_cost);
+    int64_t nctas =
+        std::max<int64_t>(1, std::min<int64_t>({(int64_t)resident, chunk, kMaxG8Ctas, cost / max_chunk_cost}));
     const int64_t Q = (cost + nctas - 1) / nctas;
     nctas = (cost + Q - 1) / Q;
     L.n_items = n;
