@@ -39,6 +39,14 @@ METRIC = "quantized GEMV achieved HBM GB/s (% of B200 peak); decoder-layer µs/t
 SPEC_HBM_GBS = 8000.0
 
 
+def input_role(m):
+    """The projection's name within its layer (q, k, v, o, gate, up, down)."""
+    return m.name.rsplit(".", 1)[1]
+
+
+SHARING = ("k", "v", "up")  # projections that read the input of q (k, v) or of gate (up)
+
+
 def algo_bytes(N, K, grid, M=1, ybytes=4):
     """packed codes + bf16 scales + activations + outputs of one product."""
     if grid == tb.TERNARY_B3:  # 26 bytes per 128-group, rows padded to 16 bytes
@@ -46,6 +54,12 @@ def algo_bytes(N, K, grid, M=1, ybytes=4):
     else:
         codes = N * K * (3 if grid == synth.INT3 else 2) // 8
     return codes + N * (K // 128) * 2 + M * K * 2 + M * N * ybytes
+
+
+def layer_algo_bytes(mats):
+    """Algorithmic bytes of one decoder layer's projections: each product's
+    own, with an input that q/k/v (gate/up) share counted once."""
+    return sum(algo_bytes(m.N, m.K, m.grid) - (2 * m.K if input_role(m) in SHARING else 0) for m in mats)
 
 
 TRAFFIC_RECORD = os.path.join("profiles", "k_gemv8_traffic.json")
@@ -75,7 +89,7 @@ def workload_config(stack, world):
     """The `config` object of the JSON line (both arms): the decode stack's
     shape, grid mix and bytes."""
     packed = sum(m.N * m.K * (3 if m.grid == synth.INT3 else 2) // 8 for mats in stack for m in mats)
-    step_bytes = sum(algo_bytes(m.N, m.K, m.grid) for mats in stack for m in mats)
+    step_bytes = sum(layer_algo_bytes(mats) for mats in stack)
     return {"workload": f"qwen3_8b_like_decode_stack_{len(stack)}L_mixed_grids", "batch": 1, "layers": len(stack),
             "hidden": 4096, "mlp": 12288, "kv_dim": 1024,
             "grid_mix": {synth.GRID_NAMES[g]: round(v, 4) for g, v in synth.grid_fractions(stack).items()},
@@ -192,9 +206,12 @@ class Clocks:
 # ---------------------------------------------------------------- workload
 
 class DecodeStack:
-    """Packed, resident 36-layer stack with one input and one output per
-    projection; x vectors and y outputs live in single flat buffers so the
-    end-to-end variant moves them with one copy each way per step."""
+    """Packed, resident 36-layer stack.  The inputs are those of a decoder
+    layer: q, k and v read one x (the normed hidden state), gate and up one
+    x, o and down one each, so a layer has four input vectors; every
+    projection has its own output.  x vectors and y outputs live in single
+    flat buffers so the end-to-end variant moves them with one copy each way
+    per step."""
 
     def __init__(self, dev, layers=None):
         self.dev = dev
@@ -207,7 +224,7 @@ class DecodeStack:
         xs, ys = 0, 0
         for mats in stack:
             for m in mats:
-                xs += m.K
+                xs += m.K if input_role(m) not in SHARING else 0
                 ys += m.N
         self.x_all = torch.empty(xs, dtype=torch.bfloat16, device=dev)
         self.y_all = torch.empty(ys, dtype=torch.float32, device=dev)
@@ -216,18 +233,24 @@ class DecodeStack:
         ws_bytes = 0
         for li, mats in enumerate(stack):
             items, b = [], 0
+            shared = {}
             for m in mats:
                 W = synth.gaussian_weights(m.N, m.K, seed=m.seed, device=dev, dtype=torch.bfloat16)
                 s = tb.tb_scales_absmax(W, m.grid)
                 p = tb.tb_pack(W, m.grid, s)
                 del W
-                x = self.x_all[xo:xo + m.K]
-                x.copy_(synth.activations(m.K, seed=m.seed, device=dev))
+                role = input_role(m)
+                if role in SHARING:  # the input of q (gate)
+                    x = shared["q" if role != "up" else "gate"]
+                else:
+                    x = self.x_all[xo:xo + m.K]
+                    x.copy_(synth.activations(m.K, seed=m.seed, device=dev))
+                    xo += m.K
+                    shared[role] = x
                 y = self.y_all[yo:yo + m.N]
-                xo += m.K
                 yo += m.N
                 items.append((p, m.grid, s, x, y, m.N, m.K))
-                b += algo_bytes(m.N, m.K, m.grid)
+                b += algo_bytes(m.N, m.K, m.grid) - (2 * m.K if role in SHARING else 0)
                 self.packed_bytes += p.numel()
             arr = tb.linear_items(items)
             ws_bytes = max(ws_bytes, tb.layer_workspace_bytes(arr))

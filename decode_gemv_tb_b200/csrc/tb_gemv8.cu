@@ -29,26 +29,29 @@
 // the truncation of activations more than 2^42 below their group's largest
 // (include/tb.h states the bound).
 //
-// Data flow.  One kernel per call, one CTA per SM: eight consumer warps and
-// a producer warp.  The work of a call is the sequence of chunks (item, tile
-// of 256 rows, C consecutive groups: C = 4 for the 2-bit container, 2 for 3
-// bits) in item, tile, group order; each CTA owns a contiguous range of
-// equal cost (tb_partition.h).
-//   * Records.  When the records a range reads fit in shared memory (the
-//     usual case: a range covers about one tile of one or two items), the
-//     consumer warps build them there once the previous kernel in the stream
-//     has finished (x prefetched into L2 before that), then meet at a named
-//     barrier.  Otherwise the consumer warps of all CTAs build each record
-//     once, in the workspace, count them per record set, and the producer
-//     copies a chunk's records into its stage once the set is complete.
-//   * Stages.  Each chunk passes through a ring of shared-memory stages.
-//     The producer copies the packed weights (a 2-D tensor copy of 256 rows
-//     x 128 or 96 bytes, no multicast) and the scales (256 rows x 8 groups)
-//     into the stage -- inputs no earlier kernel writes, so the first stages
-//     are requested at once, even before the previous call in the stream has
-//     finished.
-//   * Consumer warp w decodes rows 32w .. 32w+31 with LOP3 masks, runs eight
-//     MMAs per group and accumulates in fp32.
+// Data flow.  Two kernels per call, the second a programmatic dependent of
+// the first:
+//   * k_g8_records: one warp per (record set, group) builds the group's
+//     record (1088 bytes: the eight digit columns in MMA fragment order and
+//     the offset sums) into the workspace.  Projections that read the same x
+//     with the same code width share a record set.  x is requested into L2
+//     at once and read once the previous kernel in the stream has finished.
+//   * k_gemv8: one CTA per SM, eight consumer warps and a producer warp.
+//     The work of a call is the sequence of chunks (item, tile of 256 rows,
+//     C consecutive groups: C = 4 for the 2-bit container, 2 for 3 bits) in
+//     item, tile, group order; each CTA owns a contiguous range of equal
+//     cost (tb_partition.h: a 3-bit group costs twice a 2-bit one, so every
+//     chunk costs the same).
+//   * Stages.  Each chunk passes through a ring of four shared-memory
+//     stages.  The producer copies the packed weights (a 2-D tensor copy of
+//     256 rows x 128 or 96 bytes, no multicast) and the scales (256 rows x 8
+//     groups) into the stage -- inputs no earlier kernel writes, so the first
+//     four stages are requested at once, before the record kernel has
+//     finished -- and, once it has, the chunk's records (one bulk copy).
+//   * Consumer warp w decodes rows 64 (w & 3) .. 64 (w & 3) + 63 of the
+//     tile, for half of the chunk's groups (w >> 2), with LOP3 masks, runs
+//     four MMAs per 16 rows and group and accumulates in fp32; the two
+//     halves of a row block meet in shared memory at the end of a segment.
 // A stage is full when its copies have landed and the producer has
 // arrived; empty when all eight consumers have.  A tile whose groups are
 // split between CTAs is combined by the CTA that reads its first chunk --

@@ -67,7 +67,14 @@ def test_workload_config_names_the_stack(bench):
     assert cfg["parallelism"] == "replicas1"
     mix = cfg["grid_mix"]
     assert abs(sum(mix.values()) - 1.0) < 1e-3
-    # 2.01 GB of algorithmic bytes per step (codes, scales, x and y of all 252 products)
-    step = sum(bench.algo_bytes(m.N, m.K, m.grid) for mats in stack for m in mats)
-    assert cfg["step_algorithmic_bytes"] == step
+    # 2.01 GB of algorithmic bytes per step: codes, scales and y of all 252
+    # products, and the four input vectors of each layer (q/k/v share one,
+    # gate/up another, all of 4096 elements: k, v and up read no bytes of
+    # their own)
+    every = sum(bench.algo_bytes(m.N, m.K, m.grid) for mats in stack for m in mats)
+    step = cfg["step_algorithmic_bytes"]
+    assert every - step == 36 * 3 * 2 * 4096
+    assert step == sum(bench.layer_algo_bytes(mats) for mats in stack)
     assert 2.0e9 < step < 2.02e9
+    roles = [bench.input_role(m) for m in stack[0]]
+    assert roles == ["q", "k", "v", "o", "gate", "up", "down"]
