@@ -387,19 +387,20 @@ def rows_section(dev, stream):
             fl = 2.0 * M * W.shape[0] * W.shape[1]
             by = algo_bytes(W.shape[0], W.shape[1], grid, M=M)
             g[f"{synth.GRID_NAMES[grid]}_M{M}"] = {"us": ms * 1e3, "TFLOP_s": fl / ms / 1e9, "GB_s": by / ms / 1e6}
-    # prefill: 256 batch rows, run by tb_gemm as four blocks of 64 (2-bit)
-    try:
-        s = tb.tb_scales_absmax(W, synth.INT2)
-        p = tb.tb_pack(W, synth.INT2, s)
-        M = 256
-        X = synth.activations(W.shape[1], seed=4256, device=dev, M=M)
-        Y = torch.empty((M, W.shape[0]), dtype=torch.float32, device=dev)
-        ws = tb.workspace(tb.workspace_bytes(M, W.shape[0], W.shape[1]), dev)
-        ms = med(lambda: tb.tb_gemm(p, synth.INT2, s, X, W.shape[0], W.shape[1], Y, ws=ws), inner=3)
-        fl = 2.0 * M * W.shape[0] * W.shape[1]
-        g["int2_M256_prefill_blocks_of_64"] = {"us": ms * 1e3, "TFLOP_s": fl / ms / 1e9}
-    except tb.TBError as e:  # reported in the row; the line still prints
-        g["int2_M256_prefill_blocks_of_64"] = {"error": str(e)[:200]}
+    # prefill: 256 and 1024 batch rows in one tb_gemm launch (blocks of 64 batch rows), both grids
+    for grid in (synth.INT2, synth.INT3):
+        try:
+            s = tb.tb_scales_absmax(W, grid)
+            p = tb.tb_pack(W, grid, s)
+            for M in (256, 1024):
+                X = synth.activations(W.shape[1], seed=4000 + M, device=dev, M=M)
+                Y = torch.empty((M, W.shape[0]), dtype=torch.float32, device=dev)
+                ws = tb.workspace(tb.workspace_bytes(M, W.shape[0], W.shape[1]), dev)
+                ms = med(lambda: tb.tb_gemm(p, grid, s, X, W.shape[0], W.shape[1], Y, ws=ws), inner=3)
+                fl = 2.0 * M * W.shape[0] * W.shape[1]
+                g[f"{synth.GRID_NAMES[grid]}_M{M}_prefill"] = {"us": ms * 1e3, "TFLOP_s": fl / ms / 1e9}
+        except tb.TBError as e:  # reported in the row; the line still prints
+            g[f"{synth.GRID_NAMES[grid]}_prefill"] = {"error": str(e)[:200]}
     out["gemm_gate_17408x5120"] = g
     del bufs, Ws
     torch.cuda.empty_cache()

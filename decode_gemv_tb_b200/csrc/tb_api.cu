@@ -66,18 +66,21 @@ inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 // needs no workspace; its size is reported as this nominal minimum.
 constexpr size_t kNoWorkspace = 256;
 
-// batch sizes from which tb_gemm runs on the tcgen05 path
+// tb_gemm's kernels by batch size: 2 <= M < 32 mma.sync; 32 <= M <= 64 the
+// tcgen05 kernel with the decoded weights in tensor memory; larger (prefill)
+// batches the tcgen05 kernel with both operands in shared memory, every batch
+// row in one launch
 constexpr int64_t kTCMinM = 32;
+constexpr int64_t kSSMinM = 65;
+constexpr long long kSSWaitCycles = 4000000000LL;  // about 2 s at 2 GHz
 
 // Batch-1 products of at most this many weights run the single-launch row
 // kernel (no split-tile combine, no workspace), as do all products in the
 // 5-trits-per-byte layout; larger ones the integer tensor-path kernel.
 constexpr int64_t kRowWarpMaxWeights = (int64_t)1 << 24;
 
-// Batches above 64 rows (prefill) run as consecutive blocks of 64 rows, the
-// last block the remainder, each through the dispatch for its size, in
-// stream order and sharing the workspace.
-constexpr int64_t kGemmBlockM = 64;
+// Largest batch of one tb_gemm call (prefill batches included: the
+// tensor-core kernel takes every batch row in one launch).
 constexpr int64_t kMaxGemmM = (int64_t)1 << 16;
 
 bool use_rowwarp(int grid, int64_t N, int64_t K) {
@@ -320,8 +323,8 @@ extern "C" {
 int tb_version(void) { return 100; }
 
 unsigned int tb_wait_timeouts(void) {
-    const unsigned int a = take_wait_timeouts(), b = take_g8_timeouts();
-    return (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu) ? 0xFFFFFFFFu : a + b;
+    const unsigned int a = take_wait_timeouts(), b = take_g8_timeouts(), c = take_ss_timeouts();
+    return (a == 0xFFFFFFFFu || b == 0xFFFFFFFFu || c == 0xFFFFFFFFu) ? 0xFFFFFFFFu : a + b + c;
 }
 
 tb_status_t tb_sync_status(tb_stream_t stream) {
@@ -384,15 +387,12 @@ tb_status_t tb_unpack(const void* packed, tb_grid_t grid, int64_t N, int64_t K, 
 
 size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (M < 1 || M > kMaxGemmM || !shape_ok(N, K)) return 0;
-    if (M > kGemmBlockM) {  // the largest of its blocks' sizes
-        const int64_t rem = M % kGemmBlockM;
-        return std::max(tb_workspace_bytes(kGemmBlockM, N, K), rem ? tb_workspace_bytes(rem, N, K) : (size_t)0);
-    }
     if (M == 1) {  // the 3-bit chunking (more chunks) bounds both widths
         const Item it = make_item(nullptr, TB_GRID_INT3, nullptr, nullptr, K, nullptr, TB_F32, N, 1, N, K);
         return g8_space(&it, 1, false).need();
     }
-    if (M >= kTCMinM) return 2 * gemm_tc_workspace_bytes(M, N, K);
+    if (M >= kSSMinM) return 2 * gemm_ss_control_bytes(M, N, K);  // control words only
+    if (M >= kTCMinM) return 2 * gemm_tc_workspace_bytes(M, N, K);  // data only
     return kNoWorkspace;
 }
 
@@ -435,17 +435,6 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if (!workspace) return TB_ERR_ARG;
     if (!aligned(X, 16) || ldx % 8 != 0 || !aligned(workspace, 256)) return TB_ERR_ALIGN;
     if (workspace_bytes < tb_workspace_bytes(M, N, K)) return TB_ERR_ARG;  // the contract, whichever kernel runs
-    if (M > kGemmBlockM) {
-        const size_t ysz = y_dtype == TB_F32 ? 4 : 2;
-        for (int64_t m0 = 0; m0 < M; m0 += kGemmBlockM) {
-            const int64_t mb = std::min(kGemmBlockM, M - m0);
-            const tb_status_t s2 = tb_gemm(packed, grid, scales, X + m0 * ldx, ldx,
-                                           static_cast<char*>(Y) + m0 * ldy * ysz, y_dtype, ldy, mb, N, K, workspace,
-                                           workspace_bytes, stream);
-            if (s2 != TB_OK) return s2;
-        }
-        return TB_OK;
-    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // the row kernel: the 5-trit layout (one launch per batch row) and small batch-1 products
     if (is_b3(grid) || (M == 1 && use_rowwarp(grid, N, K))) {
@@ -461,6 +450,13 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if (M == 1) {
         Item it = make_item(packed, grid, scales, X, ldx, Y, y_dtype, N, 1, N, K);
         return launch_g8_items(&it, 1, workspace, workspace_bytes, false, false, st);
+    }
+    if (M >= kSSMinM) {
+        // tiles, batch blocks and groups index 32-bit cursors; chunks are counted in 64 bits
+        if ((N + 127) / 128 * ((M + 63) / 64) >= ((int64_t)1 << 31)) return TB_ERR_SHAPE;
+        // all of its workspace is control words: the front
+        return cuda_status(launch_gemm_ss(packed, grid, scales, X, ldx, Y, y_dtype, ldy, M, N, K, workspace,
+                                          kSSWaitCycles, st));
     }
     if (M >= kTCMinM) {
         if (K / kGroup * 64 > INT_MAX || (N + 127) / 128 > INT_MAX / 16 ||

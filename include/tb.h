@@ -193,14 +193,21 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
  *     (The row kernel behind small tb_gemv calls uses none of it.)
  *   2 <= M < 32: none (the kernel reads X as it is); the size is reported
  *     as 256.
- *   M >= 32 (the tensor-core path), data only: X copied per group into the
- *     MMA's layout, the scales transposed per 128-row tile, a counter per
- *     tile (cleared by the call itself) and the K-split partial sums,
+ *   32 <= M <= 64 (the tensor-core path with the decoded weights in tensor
+ *     memory), data only: X copied per group into the MMA's layout, the
+ *     scales transposed per 128-row tile, a counter per tile (cleared by the
+ *     call itself) and the K-split partial sums,
  *       D = ceil256(G * NP * 256) + ceil256(T * G * 256) + ceil256(4 * T)
  *         + [S > 1] ceil256(T * S * NP * 512),
  *     size 2 D, with NP = M rounded up to 16, T = ceil(N / 128) and S = the
  *     K split, max(1, min(floor((296 + T/2) / T), 16, G)).
- *   M > 64: the larger of the sizes for 64 and for M mod 64 (when not 0).
+ *   M > 64 (prefill: the tensor-core path with both operands in shared
+ *     memory), control only: per CTA (at most 256, at most one per chunk)
+ *     128 x 64 flagged partial-sum words (units whose groups are split
+ *     between CTAs are combined in a fixed order by the CTA that reads the
+ *     unit's first group):
+ *       ceil256(65536 * min(256, T * ceil(M / 64) * G)),
+ *     size twice that.
  * The workspace is
  *   - device memory, 256-byte aligned, at least the size returned here (for
  *     every call that uses it), ZERO-FILLED ONCE when allocated, and again
@@ -229,15 +236,16 @@ TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *s
                            tb_dtype_t y_dtype, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
                            tb_stream_t stream);
 
-/* Small-batch GEMM Y = X W^T, 1 <= M <= 64 (ThinkBit page, 무엇인가: the
+/* GEMM Y = X W^T, 1 <= M <= 65536 (ThinkBit page, 무엇인가: the
  * weights are read once for all M activation rows; 어떻게 동작하나: w = c * s,
  * so every row is the GEMV above on its own activations).  M = 1 runs as
- * tb_gemv; 2 <= M < 32 on mma.sync, from M = 32 on the tcgen05 tensor cores,
- * both with the codewords decoded exactly to bf16; TB_GRID_TERNARY_B3: one
- * GEMV launch per batch row, K <= 57600.  Prefill batches, 64 < M <= 65536,
- * run as consecutive blocks of 64 batch rows (the last one the remainder),
- * each like a call with that M, in stream order: the weights are decoded
- * once per block.
+ * tb_gemv; 2 <= M < 32 on mma.sync, 32 <= M <= 64 on the tcgen05 tensor
+ * cores with the decoded weights in tensor memory; prefill batches,
+ * 64 < M <= 65536, in ONE launch on the tcgen05 tensor cores with both
+ * operands in shared memory, 128 weight rows by blocks of 64 batch rows per
+ * MMA unit (the weights are read from HBM once and decoded once per block);
+ * all with the codewords decoded exactly to bf16.  TB_GRID_TERNARY_B3: one
+ * GEMV launch per batch row, K <= 57600.
  *   X          [M][ldx] bf16, ldx >= K, ldx % 8 == 0, device; finite, |x| < 2^120.
  *   Y          [M][ldy] fp32 or bf16, ldy >= N, device; Y[m][n] for n < N written.
  *   workspace  tb_workspace_bytes(M, N, K) bytes. */
