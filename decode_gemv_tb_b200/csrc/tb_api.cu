@@ -391,7 +391,10 @@ size_t tb_workspace_bytes(int64_t M, int64_t N, int64_t K) {
         const Item it = make_item(nullptr, TB_GRID_INT3, nullptr, nullptr, K, nullptr, TB_F32, N, 1, N, K);
         return g8_space(&it, 1, false).need();
     }
-    if (M >= kSSMinM) return 2 * gemm_ss_control_bytes(M, N, K);  // control words only
+    if (M >= kSSMinM) {
+        const SSSpace sp = gemm_ss_space(M, N, K);
+        return 2 * std::max(sp.control, sp.data);
+    }
     if (M >= kTCMinM) return 2 * gemm_tc_workspace_bytes(M, N, K);  // data only
     return kNoWorkspace;
 }
@@ -454,9 +457,8 @@ tb_status_t tb_gemm(const void* packed, tb_grid_t grid, const uint16_t* scales, 
     if (M >= kSSMinM) {
         // tiles, batch blocks and groups index 32-bit cursors; chunks are counted in 64 bits
         if ((N + 127) / 128 * ((M + 63) / 64) >= ((int64_t)1 << 31)) return TB_ERR_SHAPE;
-        // all of its workspace is control words: the front
         return cuda_status(launch_gemm_ss(packed, grid, scales, X, ldx, Y, y_dtype, ldy, M, N, K, workspace,
-                                          kSSWaitCycles, st));
+                                          workspace_bytes, kSSWaitCycles, st));
     }
     if (M >= kTCMinM) {
         if (K / kGroup * 64 > INT_MAX || (N + 127) / 128 > INT_MAX / 16 ||

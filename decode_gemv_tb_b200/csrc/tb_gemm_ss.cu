@@ -10,18 +10,18 @@
 // Section 무엇인가: the weights are read once for all batch rows, so the
 // product turns from memory-bound (a few rows) into a dense contraction.
 //
-// Work.  A unit is (tile of 128 weight rows, block of 64 batch rows); the
+// Work.  A unit is (tile of 128 weight rows, block of 128 batch rows); the
 // call's work is the sequence of (unit, group) chunks, units in tile order
 // (the batch blocks of a tile are neighbours, so the tile's packed bytes are
 // re-read from L2), groups in k order.  One CTA per SM owns an equal
 // contiguous range of chunks; a unit split between CTAs is finished by the
 // CTA that holds its first chunk (for it the unit is the last segment of its
-// range): the later CTAs publish their partial sums as flagged 64-bit words
-// (fp32 bits, flag) and the finishing CTA adds them in CTA order (bitwise
-// deterministic) and clears them.
+// range): each later CTA writes its partial sums and releases a flag, the
+// finishing CTA acquires the flags (and clears them) and adds the sums in
+// CTA order (bitwise deterministic).
 //
 // Pipeline of a CTA (18 warps), per chunk:
-//   * producer warp: the block's activations of the group (64 rows x 128
+//   * producer warp: the block's activations of the group (128 rows x 128
 //     bf16, rows past M read as zero) as two tensor copies (no multicast)
 //     with 128-byte swizzle -- the MMA's K-major B layout -- into a ring of
 //     activation stages;
@@ -29,13 +29,14 @@
 //     global memory (four groups ahead, in registers), decodes it to the
 //     signed codeword, exactly, as bf16 (tb_device.cuh) and stores it into
 //     one of four A stages in the same swizzled K-major layout;
-//   * MMA warp: eight 128 x 64 x 16 MMAs (kind::f16, bf16 in, fp32 out)
-//     into accumulator d = chunk mod 8 of tensor memory, committed to three
+//   * MMA warp: eight 128 x 128 x 16 MMAs (kind::f16, bf16 in, fp32 out)
+//     into accumulator d = chunk mod 3 of tensor memory, committed to three
 //     mbarriers: the A stage and the activation stage are free, the
 //     accumulator is ready;
 //   * 8 epilogue warps (two per 32 TMEM lanes = 32 rows, each half of the
 //     batch columns): read the accumulator back, release it, and add  s * D
-//     to the row's running sums in registers.  Every product c * x is exact;
+//     to the row's running sums, kept in the last 128 columns of tensor
+//     memory.  Every product c * x is exact;
 //     the sums over a group (8 MMAs) and over groups are fp32.
 // Every wait is bounded.  A wait that gives up is counted
 // (g_ss_timeouts), raises the CTA's abort flag -- every other wait of the
@@ -56,8 +57,7 @@ namespace {
 
 constexpr int kSSRows = 128;        // weight rows per tile (the MMA's M)
 constexpr int kSSStages = 4;        // decoded A operands in shared memory
-constexpr int kSSDBufs = 8;         // accumulators in tensor memory
-constexpr int kSSBlockM = 64;       // batch rows per unit
+constexpr int kSSNP = 128;          // batch rows per unit: the MMA's N (two 64-row blocks share a decode)
 constexpr int kSSDecWarps = 8;      // a thread per half of a row's group
 constexpr int kSSEpiWarps = 8;      // two per 32 TMEM lanes, half the columns each
 constexpr int kSSWarpDec0 = 2;                            // warps 2 .. 9 decode
@@ -68,12 +68,14 @@ constexpr uint64_t kSSMaxCtas = 256;             // bound of the grid (one CTA p
 constexpr int kSSPrefetch = 4;                   // groups of packed codes in flight per decoder thread
 
 __host__ __device__ constexpr int ss_xbytes(int np) { return np * kGroup * 2; }
-// activation stages: eight for up to 32 batch columns, four for 64
-__host__ __device__ constexpr int ss_xstages(int np) { return np <= 32 ? 8 : 4; }
+// activation stages (as many as fit beside the four A stages)
+__host__ __device__ constexpr int ss_xstages(int np) { return np <= 32 ? 8 : (np <= 64 ? 4 : 3); }
+// accumulators in tensor memory: its 512 columns less the running sums' NP
+__host__ __device__ constexpr int ss_dbufs(int np) { return 512 / np - 1; }
 __host__ __device__ constexpr int ss_smem_bytes(int np) {
     return kSSStages * kSSABytes + ss_xstages(np) * ss_xbytes(np) + 1024;
 }
-static_assert(ss_smem_bytes(64) <= 227 * 1024 && ss_smem_bytes(32) <= 227 * 1024, "shared memory");
+static_assert(ss_smem_bytes(kSSNP) + 512 <= 227 * 1024, "shared memory");
 static_assert(kSSStages == 4 && kSSPrefetch % kSSStages == 0, "the decoders' ring is unrolled by its depth");
 
 __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -187,45 +189,47 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr)
         : "memory");
 }
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr)
-                 : "memory");
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
 }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// ---- flagged words (partial sums between CTAs) ----------------------------------------
-__device__ __forceinline__ void st_word(uint64_t* p, uint64_t v) {
-    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+// ---- partial sums between CTAs: a release flag per CTA --------------------------------
+__device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-__device__ __forceinline__ uint64_t ld_word(const uint64_t* p) {
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ uint64_t flagged(float v) { return (1ull << 32) | __float_as_uint(v); }
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 constexpr float kNaN = __builtin_nanf("");
 
-// The value of a published word (v: its first read) once its flag is set,
-// after which the word is cleared; NaN when the CTA has aborted or after `limit` cycles (which
-// aborts the CTA and is counted).
-__device__ __forceinline__ float take_word(uint64_t* w, uint64_t v, long long limit, volatile int* abort) {
-    if (!(v >> 32)) {
-        const long long t0 = clock64();
-        while (!((v = ld_word(w)) >> 32)) {
-            if (*abort) return kNaN;
-            if (clock64() - t0 > limit) {
-                atomicAdd(&g_ss_timeouts, 1u);
-                *abort = 1;
-                return kNaN;
-            }
-            __nanosleep(64);
+// Waits (acquire) until a later CTA has released its flag, then clears it
+// for the next call; gives up when the CTA has aborted or after `limit`
+// cycles (which aborts the CTA and is counted).
+__device__ __forceinline__ void take_flag(uint32_t* f, long long limit, volatile int* abort) {
+    const long long t0 = clock64();
+    while (ld_acquire(f) == 0u) {
+        if (*abort) return;
+        if (clock64() - t0 > limit) {
+            atomicAdd(&g_ss_timeouts, 1u);
+            *abort = 1;
+            return;
         }
+        __nanosleep(64);
     }
-    st_word(w, 0ull);
-    return __uint_as_float((uint32_t)v);
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(0u) : "memory");
 }
 
 }  // namespace
@@ -235,11 +239,13 @@ struct SSArgs {
     const uint8_t* packed;    // [N][rb] packed codes
     const uint16_t* scales;   // [N][G] bf16
     void* Y;                  // [M][ldy]
-    uint64_t* pslots;         // [ctas][128][NP] flagged partial sums (zero between calls)
+    uint32_t* pflag;          // [ctas] release flags of published partial sums (zero between calls)
+    float* pdata;             // [ctas][128][NP] published partial sums
     int64_t N, ldy, rb;
     uint64_t Q;               // chunks: T * MB * G
     long long wait_cycles;
     int32_t M, G, MB, ydt, ctas;
+    int32_t xrows;            // rows of an activation box: min(NP, M) (the MMA's other columns are never stored)
 };
 
 namespace {
@@ -253,9 +259,12 @@ template <int NP, int KIND>
 __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant__ SSArgs A) {
     constexpr int XB = ss_xbytes(NP);
     constexpr int XS = ss_xstages(NP);
+    constexpr int kSSDBufs = ss_dbufs(NP);
+    constexpr int kSSBlockM = NP;  // batch rows per unit
     constexpr int GB = KIND ? 48 : 32;  // packed bytes of one row's group
     constexpr uint32_t kIdesc = ss_idesc(NP);
-    constexpr uint32_t kTmemCols = NP * kSSDBufs <= 128 ? 128 : (NP * kSSDBufs <= 256 ? 256 : 512);
+    constexpr uint32_t kTmemCols = 512;  // kSSDBufs accumulators of NP columns, then NP columns of running sums
+    static_assert(NP * (kSSDBufs + 1) <= (int)kTmemCols, "tensor memory");
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t afull[kSSStages], aempty[kSSStages], xfull[XS], xempty[XS];
     __shared__ __align__(8) uint64_t dfull[kSSDBufs], dfree[kSSDBufs];
@@ -311,7 +320,7 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
                     break;
                 const uint32_t b = u % MB;  // the unit's batch block
                 const uint32_t st = xbase_s + s * XB, bar = saddr(&xfull[s]);
-                bar_arrive_expect(bar, (uint32_t)XB);
+                bar_arrive_expect(bar, (uint32_t)(2 * 128 * A.xrows));
                 tma_2d(st, &A.xmap, (int)(g * kGroup), (int)(b * kSSBlockM), bar);
                 tma_2d(st + NP * 128, &A.xmap, (int)(g * kGroup + 64), (int)(b * kSSBlockM), bar);
                 issued = k + 1;
@@ -438,14 +447,15 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
         }
     } else {
         // ---------------- epilogue: rows 32 (warp % 4) .. + 31, columns NH eh .. NH eh + NH - 1 ----------------
-        constexpr int NH = NP / 2;
+        // The row's running sums of a segment live in tensor memory (the
+        // columns after the accumulators), 16 columns at a time in registers.
+        constexpr int NH = NP / 2, W = 16;
+        static_assert(NH % (2 * W) == 0, "epilogue columns");
         const int qd = warp & 3, eh = (warp - kSSWarpEpi0) >> 2;
         const int r = 32 * qd + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)(eh * NH);
-        float acc[NH];
-#pragma unroll
-        for (int j = 0; j < NH; ++j) acc[j] = 0.f;
-        // scales four chunks ahead (cursor pu, pg)
+        const uint32_t scol = lane_base + (uint32_t)(kSSDBufs * NP);  // running sums
+        // scales four chunks ahead (cursor pt, pbk, pg)
         uint32_t pg = (uint32_t)(q0 % G), pt = (uint32_t)(q0 / G / MB), pbk = (uint32_t)(q0 / G % MB);
         float sq[4] = {0.f, 0.f, 0.f, 0.f};  // the scales of the next block of four chunks
         auto next_scale = [&]() -> float {
@@ -466,6 +476,15 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
         uint32_t u = (uint32_t)(q0 / G), g = (uint32_t)(q0 % G);
         uint64_t seg0 = q0;  // first chunk of the current segment
         bool failed = false;
+        auto zero_sums = [&]() {
+            uint32_t z[W];
+#pragma unroll
+            for (int i = 0; i < W; ++i) z[i] = 0u;
+#pragma unroll
+            for (int cc = 0; cc < NH; cc += W) tmem_st16(scol + cc, z);
+            tmem_st_wait();
+        };
+        zero_sums();
 #pragma unroll 1
         for (int k0 = 0; k0 < n; k0 += 4) {
           // this block's four scales (requested during the previous block); request the next block's
@@ -485,63 +504,105 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
             if (!failed) {
                 tc_fence_after();
                 const uint32_t col = lane_base + (uint32_t)(d * NP);
-                constexpr int W = NH < 16 ? NH : 16;  // columns per load (registers)
-#pragma unroll
-                for (int c0 = 0; c0 < NH; c0 += W) {
-                    uint32_t v[W];
-                    if constexpr (W == 8) tmem_ld8(col + c0, v);
-                    else tmem_ld16(col + c0, v);
+#pragma unroll 1
+                for (int cc = 0; cc < NH; cc += 2 * W) {  // sums += s * D, 32 columns (one wait) at a time
+                    uint32_t v[2][W], a[2][W];
+                    tmem_ld16(col + cc, v[0]);
+                    tmem_ld16(col + cc + W, v[1]);
+                    tmem_ld16(scol + cc, a[0]);
+                    tmem_ld16(scol + cc + W, a[1]);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < W; ++i) acc[c0 + i] = fmaf(sc, __uint_as_float(v[i]), acc[c0 + i]);
+                    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                        for (int i = 0; i < W; ++i)
+                            a[h][i] = __float_as_uint(fmaf(sc, __uint_as_float(v[h][i]), __uint_as_float(a[h][i])));
+                        tmem_st16(scol + cc + h * W, a[h]);
+                    }
                 }
+                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) bar_arrive(saddr(&dfree[d]));
-            } else {
-#pragma unroll
-                for (int j = 0; j < NH; ++j) acc[j] = kNaN;
             }
             // end of the unit or of the range: finish the segment
             const uint64_t q = q0 + (uint64_t)k;
             if (g + 1 == G || k + 1 == n) {
                 const uint64_t ustart = (uint64_t)u * G, uend = ustart + G;
                 const uint32_t t = u / MB, b = u - t * MB;
-                if (seg0 > ustart) {  // a later part of a unit begun by an earlier CTA: publish
-                    uint64_t* w = A.pslots + ((uint64_t)cta * kSSRows + r) * NP + eh * NH;
+                const bool publish = seg0 > ustart;  // a later part of a unit begun by an earlier CTA
+                const uint64_t c1 = (!publish && uend > q1) ? ss_owner(uend - 1, A.Q, P) : cta;
+                const int64_t row = (int64_t)t * kSSRows + r;
+                auto sums = [&](int cc, float (&acc)[W]) {  // this segment's sums, columns cc .. cc + 15
+                    if (!failed) {
+                        uint32_t a[W];
+                        tmem_ld16(scol + cc, a);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < NH; ++j) st_word(w + j, flagged(acc[j]));
-                } else {
-                    if (uend > q1) {  // later CTAs hold the rest of the unit: add their sums in CTA order
-                        const uint64_t c1 = ss_owner(uend - 1, A.Q, P);
+                        for (int i = 0; i < W; ++i) acc[i] = __uint_as_float(a[i]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < W; ++i) acc[i] = kNaN;
+                    }
+                };
+                if (publish) {
+                    // the partial sums, then (all epilogue threads done) one release of this CTA's flag
+                    float* pd = A.pdata + ((uint64_t)cta * kSSRows + r) * NP + eh * NH;
 #pragma unroll 1
-                        for (uint64_t c = cta + 1; c <= c1; ++c) {
-                            uint64_t* w = A.pslots + (c * kSSRows + r) * NP + eh * NH;
+                    for (int cc = 0; cc < NH; cc += W) {
+                        float acc[W];
+                        sums(cc, acc);
 #pragma unroll
-                            for (int j0 = 0; j0 < NH; j0 += 8) {  // eight loads in flight, then the flags
-                                uint64_t v[8];
+                        for (int i = 0; i < W; i += 4)
+                            *reinterpret_cast<float4*>(pd + cc + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+                    }
+                    named_sync(1, kSSEpiWarps * 32);
+                    if (warp == kSSWarpEpi0 && lane == 0) {
+                        __threadfence();
+                        st_release(A.pflag + cta, 1u);
+                    }
+                } else {
+                    if (c1 > cta) {  // one thread acquires the later CTAs' flags (and clears them), then all read
+                        if (warp == kSSWarpEpi0 && lane == 0)
+                            for (uint64_t c = cta + 1; c <= c1; ++c) take_flag(A.pflag + c, A.wait_cycles, abort);
+                        named_sync(1, kSSEpiWarps * 32);
+                    }
+                    const bool lost = *abort != 0;
+#pragma unroll 1
+                    for (int cc = 0; cc < NH; cc += W) {
+                        float acc[W];
+                        sums(cc, acc);
+#pragma unroll 1
+                        for (uint64_t c = cta + 1; c <= c1; ++c) {  // the later CTAs' sums, in CTA order
+                            const float4* pd =
+                                reinterpret_cast<const float4*>(A.pdata + (c * kSSRows + r) * NP + eh * NH + cc);
 #pragma unroll
-                                for (int i = 0; i < 8; ++i) v[i] = ld_word(w + j0 + i);
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) acc[j0 + i] += take_word(w + j0 + i, v[i], A.wait_cycles, abort);
+                            for (int i = 0; i < W / 4; ++i) {
+                                const float4 v = __ldcg(pd + i);
+                                acc[4 * i] += v.x;
+                                acc[4 * i + 1] += v.y;
+                                acc[4 * i + 2] += v.z;
+                                acc[4 * i + 3] += v.w;
                             }
                         }
-                    }
-                    const int64_t row = (int64_t)t * kSSRows + r;
-                    if (row < A.N) {
+                        if (lost) {
 #pragma unroll
-                        for (int j = 0; j < NH; ++j) {
-                            const int64_t m = (int64_t)b * kSSBlockM + eh * NH + j;
-                            if (m < A.M) {
-                                if (A.ydt == kF32) static_cast<float*>(A.Y)[m * A.ldy + row] = acc[j];
-                                else
-                                    static_cast<__nv_bfloat16*>(A.Y)[m * A.ldy + row] = __float2bfloat16_rn(acc[j]);
+                            for (int i = 0; i < W; ++i) acc[i] = kNaN;
+                        }
+                        if (row < A.N) {
+#pragma unroll
+                            for (int i = 0; i < W; ++i) {
+                                const int64_t m = (int64_t)b * kSSBlockM + eh * NH + cc + i;
+                                if (m < A.M) {
+                                    if (A.ydt == kF32) static_cast<float*>(A.Y)[m * A.ldy + row] = acc[i];
+                                    else
+                                        static_cast<__nv_bfloat16*>(A.Y)[m * A.ldy + row] = __float2bfloat16_rn(acc[i]);
+                                }
                             }
                         }
                     }
                 }
-#pragma unroll
-                for (int j = 0; j < NH; ++j) acc[j] = 0.f;
+                if (!failed) zero_sums();
                 seg0 = q + 1;
             }
             if (++g == G) {
@@ -550,6 +611,7 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
             }
           }
         }
+        tc_fence_before();
     }
 
     // ---------------- drain and exit ----------------
@@ -574,7 +636,7 @@ const void* ss_kernel() {
     return reinterpret_cast<const void*>(&k_gemm_ss<NP, KIND>);
 }
 
-const void* pick_kernel(int kind) { return kind ? ss_kernel<64, 1>() : ss_kernel<64, 0>(); }
+const void* pick_kernel(int kind) { return kind ? ss_kernel<kSSNP, 1>() : ss_kernel<kSSNP, 0>(); }
 
 typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -606,20 +668,25 @@ int ss_sms() {
 
 }  // namespace
 
-// batch columns per MMA (prefill batches: 64; the kernel also takes 16 and 32)
-int gemm_ss_np(int64_t M) { return M >= 33 ? 64 : (M >= 17 ? 32 : 16); }
+// batch rows per unit (the MMA's N)
+int gemm_ss_np(int64_t) { return kSSNP; }
 
-size_t gemm_ss_control_bytes(int64_t M, int64_t N, int64_t K) {
+// bytes of the published partial sums' flags (control: zero between calls)
+// and of the sums themselves (data), for a grid of at most 256 CTAs
+SSSpace gemm_ss_space(int64_t M, int64_t N, int64_t K) {
     const int np = gemm_ss_np(M);
-    const uint64_t T = (uint64_t)((N + kSSRows - 1) / kSSRows), MB = (uint64_t)((M + kSSBlockM - 1) / kSSBlockM);
+    const uint64_t T = (uint64_t)((N + kSSRows - 1) / kSSRows), MB = (uint64_t)((M + np - 1) / np);
     const uint64_t Q = T * MB * (uint64_t)(K / kGroup);
     const uint64_t ctas = std::min<uint64_t>(kSSMaxCtas, Q);
-    return (size_t)(((ctas * kSSRows * (uint64_t)np * 8) + 255) / 256 * 256);
+    SSSpace sp;
+    sp.control = (size_t)((4 * ctas + 255) / 256 * 256);
+    sp.data = (size_t)((ctas * kSSRows * (uint64_t)np * 4 + 255) / 256 * 256);
+    return sp;
 }
 
 cudaError_t launch_gemm_ss(const void* packed, int grid, const uint16_t* scales, const uint16_t* X, int64_t ldx,
-                           void* Y, int ydt, int64_t ldy, int64_t M, int64_t N, int64_t K, void* control,
-                           long long wait_cycles, cudaStream_t st) {
+                           void* Y, int ydt, int64_t ldy, int64_t M, int64_t N, int64_t K, void* ws,
+                           size_t ws_bytes, long long wait_cycles, cudaStream_t st) {
     EncodeFn enc = ss_encoder();
     const int sms = ss_sms();
     if (!enc || sms <= 0) return cudaErrorInitializationError;
@@ -629,20 +696,23 @@ cudaError_t launch_gemm_ss(const void* packed, int grid, const uint16_t* scales,
     {  // X: boxes of 64 k x NP batch rows, 128-byte swizzle (the MMA's B layout); rows past M read as zero
         const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
         const cuuint64_t strides[1] = {(cuuint64_t)(ldx * 2)};
-        const cuuint32_t box[2] = {64, (cuuint32_t)np};
+        const cuuint32_t box[2] = {64, (cuuint32_t)std::min<int64_t>(np, M)};
         const cuuint32_t es[2] = {1, 1};
         if (enc(&A.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
-    const uint64_t T = (uint64_t)((N + kSSRows - 1) / kSSRows), MB = (uint64_t)((M + kSSBlockM - 1) / kSSBlockM);
+    const uint64_t T = (uint64_t)((N + kSSRows - 1) / kSSRows), MB = (uint64_t)((M + np - 1) / np);
     const uint64_t G = (uint64_t)(K / kGroup);
     A.packed = static_cast<const uint8_t*>(packed);
     A.rb = row_bytes(grid, K);
     A.scales = scales;
     A.Y = Y;
-    A.pslots = static_cast<uint64_t*>(control);
+    // flags at the front of the workspace, the sums at its back
+    const SSSpace sp = gemm_ss_space(M, N, K);
+    A.pflag = static_cast<uint32_t*>(ws);
+    A.pdata = reinterpret_cast<float*>(static_cast<char*>(ws) + (ws_bytes & ~size_t(255)) - sp.data);
     A.N = N;
     A.ldy = ldy;
     A.Q = T * MB * G;
@@ -651,9 +721,9 @@ cudaError_t launch_gemm_ss(const void* packed, int grid, const uint16_t* scales,
     A.G = (int32_t)G;
     A.MB = (int32_t)MB;
     A.ydt = ydt;
+    A.xrows = (int32_t)std::min<int64_t>(np, M);
     const uint64_t ctas = std::min<uint64_t>(std::min<uint64_t>((uint64_t)sms, kSSMaxCtas), A.Q);
     A.ctas = (int32_t)ctas;
-    if (np != 64) return cudaErrorInvalidValue;  // built for prefill batches (M > 64)
     const void* fn = pick_kernel(kind);
     const int smem = ss_smem_bytes(np);
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -57,15 +57,19 @@ cudaError_t launch_gemv_rowwarp(const void* packed, int grid, const uint16_t* sc
 size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_gemm_tc(const void* packed, int grid, const uint16_t* scales, const uint16_t* X, int64_t ldx,
                            void* Y, int ydt, int64_t ldy, int M, int64_t N, int64_t K, void* ws, cudaStream_t st);
-// GEMM with both MMA operands in shared memory (tb_gemm_ss.cu): one kernel,
-// 2 <= M <= 65536 batch rows in blocks of 64.  `control` holds
-// gemm_ss_control_bytes(M, N, K) bytes of flagged partial-sum words, zero
-// before the call and left zero by it.
+// Prefill GEMM with both MMA operands in shared memory (tb_gemm_ss.cu): one
+// kernel, M > 64 batch rows in blocks of 128.  Its workspace (ws_bytes,
+// 256-byte aligned) holds space.control bytes of flags at the front (zero
+// before the call and left zero by it) and space.data bytes of partial sums
+// at the back.
+struct SSSpace {
+    size_t control, data;
+};
 int gemm_ss_np(int64_t M);
-size_t gemm_ss_control_bytes(int64_t M, int64_t N, int64_t K);
+SSSpace gemm_ss_space(int64_t M, int64_t N, int64_t K);
 cudaError_t launch_gemm_ss(const void* packed, int grid, const uint16_t* scales, const uint16_t* X, int64_t ldx,
-                           void* Y, int ydt, int64_t ldy, int64_t M, int64_t N, int64_t K, void* control,
-                           long long wait_cycles, cudaStream_t st);
+                           void* Y, int ydt, int64_t ldy, int64_t M, int64_t N, int64_t K, void* ws,
+                           size_t ws_bytes, long long wait_cycles, cudaStream_t st);
 unsigned int take_ss_timeouts();
 // bounded device waits that gave up since the last call (clears the count;
 // synchronous); 0xFFFFFFFF if the count cannot be read

@@ -202,12 +202,13 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
  *     size 2 D, with NP = M rounded up to 16, T = ceil(N / 128) and S = the
  *     K split, max(1, min(floor((296 + T/2) / T), 16, G)).
  *   M > 64 (prefill: the tensor-core path with both operands in shared
- *     memory), control only: per CTA (at most 256, at most one per chunk)
- *     128 x 64 flagged partial-sum words (units whose groups are split
+ *     memory): per CTA (at most 256, at most one per chunk) a flag (control)
+ *     and 128 x 128 fp32 partial sums (data; units whose groups are split
  *     between CTAs are combined in a fixed order by the CTA that reads the
  *     unit's first group):
- *       ceil256(65536 * min(256, T * ceil(M / 64) * G)),
- *     size twice that.
+ *       control ceil256(4 C), data ceil256(65536 C),
+ *       C = min(256, T * ceil(M / 128) * G),
+ *     size 2 max(control, data).
  * The workspace is
  *   - device memory, 256-byte aligned, at least the size returned here (for
  *     every call that uses it), ZERO-FILLED ONCE when allocated, and again
@@ -242,7 +243,7 @@ TB_API tb_status_t tb_gemv(const void *packed, tb_grid_t grid, const uint16_t *s
  * tb_gemv; 2 <= M < 32 on mma.sync, 32 <= M <= 64 on the tcgen05 tensor
  * cores with the decoded weights in tensor memory; prefill batches,
  * 64 < M <= 65536, in ONE launch on the tcgen05 tensor cores with both
- * operands in shared memory, 128 weight rows by blocks of 64 batch rows per
+ * operands in shared memory, 128 weight rows by blocks of 128 batch rows per
  * MMA unit (the weights are read from HBM once and decoded once per block);
  * all with the codewords decoded exactly to bf16.  TB_GRID_TERNARY_B3: one
  * GEMV launch per batch row, K <= 57600.

@@ -79,10 +79,11 @@ def test_workspace_sizes(lib):
                 (al(tiles * splits * NP * 128 * 4) if splits > 1 else 0))
         assert tb.workspace_bytes(M, N, K) == 2 * data, (M, N, K)
     for M, N, K in ((65, 100, 5120), (256, 17408, 5120), (257, 7, 1024), (65536, 128, 128)):
-        # prefill path, control words only: per CTA (at most 256, at most one per chunk) 128 rows x 64
-        # flagged 8-byte partial sums; chunks = tiles of 128 rows x blocks of 64 batch rows x groups
-        chunks = (N + 127) // 128 * -(-M // 64) * (K // 128)
-        assert tb.workspace_bytes(M, N, K) == 2 * al(min(256, chunks) * 128 * 64 * 8), (M, N, K)
+        # prefill path: per CTA (at most 256, at most one per chunk) a 4-byte flag (control) and 128 rows x
+        # 128 fp32 partial sums (data); chunks = tiles of 128 rows x blocks of 128 batch rows x groups
+        ctas = min(256, (N + 127) // 128 * -(-M // 128) * (K // 128))
+        control, data = al(4 * ctas), al(ctas * 128 * 128 * 4)
+        assert tb.workspace_bytes(M, N, K) == 2 * max(control, data), (M, N, K)
     for N, K in ((1, 128), (256, 1024), (17408, 5120), (100, 1408), (4096, 12288)):
         # batch 1: control = 256 flagged 8-byte partial words per CTA (at most 256 CTAs, at most one per
         # chunk of two groups); data = the activation records of x (1088 bytes per group); size
@@ -160,10 +161,10 @@ def test_argument_errors_before_launch(lib):
 
 
 def test_prefill_workspace_is_bounded(lib):
-    """Batches above 64 rows run in one launch, in blocks of 64 batch rows:
+    """Batches above 64 rows run in one launch, in blocks of 128 batch rows:
     the workspace grows with the chunks only up to the 256-CTA bound, so a
-    prefill batch needs no more than 2 x 256 x 128 x 64 x 8 bytes."""
-    bound = 2 * 256 * 128 * 64 * 8
+    prefill batch needs no more than 2 x 256 x 128 x 128 x 4 bytes."""
+    bound = 2 * 256 * 128 * 128 * 4
     for N, K in ((100, 5120), (17408, 5120), (7, 1024)):
         for M in (65, 97, 100, 130, 4096 + 17, 65536):
             assert 0 < tb.workspace_bytes(M, N, K) <= bound
