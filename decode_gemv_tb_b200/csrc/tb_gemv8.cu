@@ -437,38 +437,45 @@ __device__ __forceinline__ void pair_epilogue(const G8Launch& L, int item, int64
 // tile that later ranges finish (combine).
 enum SegKind { kWhole = 0, kPublish = 1, kCombine = 2 };
 
-// One row's end of segment (its sum over this range's chunks of the tile).
-__device__ __forceinline__ void finish_row(const G8Launch& L, int cta, int item, uint32_t tile, int kind, int rin,
-                                           uint32_t c1, float sum) {
+// Rows rin and rin + 8 at the end of a segment (sums over this range's
+// chunks of the tile): publish them, or add the later ranges' words in CTA
+// order (the words of both rows and two ranges in flight at a time), then
+// write y.
+__device__ __forceinline__ void finish_rows(const G8Launch& L, int cta, int item, uint32_t tile, int kind, int rin,
+                                            uint32_t c1, float s0, float s1) {
     if (kind == kPublish) {
-        st_word(L.pslots + (int64_t)cta * kG8TileRows + rin, flagged(sum));
+        st_word(L.pslots + (int64_t)cta * kG8TileRows + rin, flagged(s0));
+        st_word(L.pslots + (int64_t)cta * kG8TileRows + rin + 8, flagged(s1));
         return;
     }
     if (kind == kCombine) {  // the later ranges that read this tile, in order
-        for (uint32_t c = (uint32_t)cta + 1; c <= c1; c += 4) {  // four words in flight at a time
+        for (uint32_t c = (uint32_t)cta + 1; c <= c1; c += 2) {
             uint64_t* slot[4];
             uint64_t wv[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                slot[q] = L.pslots + (int64_t)(c + q) * kG8TileRows + rin;
-                wv[q] = c + q <= c1 ? ld_word(slot[q]) : 0;
+            for (int q = 0; q < 4; ++q) {  // q: range c + (q >> 1), row rin + 8 (q & 1)
+                slot[q] = L.pslots + (int64_t)(c + (q >> 1)) * kG8TileRows + rin + 8 * (q & 1);
+                wv[q] = c + (q >> 1) <= c1 ? ld_word(slot[q]) : 0;
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                if (c + q > c1) break;
+                if (c + (q >> 1) > c1) break;
                 float p = __uint_as_float((uint32_t)wv[q]);
                 if (!(wv[q] >> 32) && !wait_word(slot[q], L.wait_cycles, &p)) {
                     atomicAdd(&g_g8_timeouts, 1u);
                     p = __int_as_float(0x7FC00000);
                 }
                 st_word(slot[q], 0);
-                sum += p;
+                if (q & 1) s1 += p;
+                else s0 += p;
             }
         }
     }
     const int64_t row = (int64_t)tile * kG8TileRows + rin;
-    store_y(L.it[item], row, sum);
-    pair_epilogue(L, item, row, sum);
+    store_y(L.it[item], row, s0);
+    store_y(L.it[item], row + 8, s1);
+    pair_epilogue(L, item, row, s0);
+    pair_epilogue(L, item, row + 8, s1);
 }
 
 // End of a warp's segment of a tile: the quad's digit pairs are summed, the
@@ -512,8 +519,7 @@ __device__ __noinline__ void g8_flush(const G8Launch& L, int cta, int rb, int gh
                         L.Q);
     }
     const int rin = 64 * rb + 16 * t + lane_k7(g);  // block 2t; block 2t + 1 is 8 rows on
-    finish_row(L, cta, item, tile, kind, rin, c1, m0);
-    finish_row(L, cta, item, tile, kind, rin + 8, c1, m1);
+    finish_rows(L, cta, item, tile, kind, rin, c1, m0, m1);
 }
 
 __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__ G8Launch L) {
