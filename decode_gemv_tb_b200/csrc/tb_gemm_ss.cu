@@ -143,11 +143,6 @@ __device__ __forceinline__ uint4 ldg_nc16(const void* p) {
                  : "l"(p));
     return v;
 }
-__device__ __forceinline__ uint2 ldg_nc8(const void* p) {
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-    return v;
-}
 
 // ---- tcgen05 -------------------------------------------------------------------------
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -368,13 +363,16 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
         auto load = [&](uint32_t (&w)[HW]) {
             const int64_t row = (int64_t)pt * kSSRows + r;
             if (row < A.N) {
-                const uint8_t* p = A.packed + row * A.rb + (int64_t)pg * GB + (KIND ? 24 : 16) * h;
                 if constexpr (KIND == 0) {
-                    const uint4 v = ldg_nc16(p);
+                    const uint4 v = ldg_nc16(A.packed + row * A.rb + (int64_t)pg * GB + 16 * h);
                     w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
                 } else {
-                    const uint2 v0 = ldg_nc8(p), v1 = ldg_nc8(p + 8), v2 = ldg_nc8(p + 16);
-                    w[0] = v0.x, w[1] = v0.y, w[2] = v1.x, w[3] = v1.y, w[4] = v2.x, w[5] = v2.y;
+                    // 48 bytes = three 16-byte pieces; half 0 takes words 0-5 (pieces 0, 1), half 1 words 6-11
+                    // (pieces 1, 2): two aligned 16-byte loads each
+                    const uint8_t* p = A.packed + row * A.rb + (int64_t)pg * GB + 16 * h;
+                    const uint4 v0 = ldg_nc16(p), v1 = ldg_nc16(p + 16);
+                    if (h == 0) w[0] = v0.x, w[1] = v0.y, w[2] = v0.z, w[3] = v0.w, w[4] = v1.x, w[5] = v1.y;
+                    else w[0] = v0.z, w[1] = v0.w, w[2] = v1.x, w[3] = v1.y, w[4] = v1.z, w[5] = v1.w;
                 }
             } else {
 #pragma unroll
