@@ -504,3 +504,22 @@ def test_gemm_prefill_gate_sampled(oracle, grid, M):
         y64, yabs = oracle.gemv_rows64(p_ref, grid, s_ref, Xb[m], K, rows)
         assert_within(Y[m, rows], y64, yabs, "f32", oracle, f"prefill gate M={M} m={m}")
     assert tb.wait_timeouts() == 0
+
+
+@pytest.mark.parametrize("grid", [tb.TERNARY, tb.INT3])
+def test_gemm_prefill_largest_batch(oracle, grid):
+    """The largest batch one tb_gemm call takes, M = 65536 (512 blocks of 128
+    batch rows), over a ragged 200-row matrix of two groups: sampled batch
+    rows (block boundaries included) against the oracle, all outputs."""
+    N, K, M = 200, 256, 65536
+    W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=5100 + grid)
+    X = synth.activations(K, seed=5200 + grid, M=M)
+    Y = tb.tb_gemm(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), X.to(DEV), N, K).cpu()
+    rng = np.random.default_rng(5300 + grid)
+    ms = np.unique(np.concatenate([[0, 127, 128, 32767, 32768, M - 129, M - 128, M - 1], rng.integers(0, M, 24)]))
+    rows = np.arange(N)
+    Xb = u16(X)
+    for m in ms:
+        y64, yabs = oracle.gemv_rows64(p_ref, grid, s_ref, Xb[m], K, rows)
+        assert_within(Y[m], y64, yabs, "f32", oracle, f"M=65536 m={m}")
+    assert tb.wait_timeouts() == 0
