@@ -387,7 +387,7 @@ def rows_section(dev, stream):
             fl = 2.0 * M * W.shape[0] * W.shape[1]
             by = algo_bytes(W.shape[0], W.shape[1], grid, M=M)
             g[f"{synth.GRID_NAMES[grid]}_M{M}"] = {"us": ms * 1e3, "TFLOP_s": fl / ms / 1e9, "GB_s": by / ms / 1e6}
-    # prefill: 256 and 1024 batch rows in one tb_gemm launch (blocks of 64 batch rows), both grids
+    # prefill: 256 and 1024 batch rows in one tb_gemm launch (blocks of 128 batch rows), both grids
     for grid in (synth.INT2, synth.INT3):
         try:
             s = tb.tb_scales_absmax(W, grid)

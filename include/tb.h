@@ -1,8 +1,9 @@
 /*
  * tb.h -- C interface of libtb_b200: ThinkBit scalar low-bit weights on
- * NVIDIA B200 (sm_100a).  Quantize/pack, unpack, batch-1 GEMV, small-batch
- * GEMM (M <= 64, and prefill batches in blocks of 64) and a grouped
- * launcher for a decoder layer's projections.
+ * NVIDIA B200 (sm_100a).  Quantize/pack, unpack, batch-1 GEMV, GEMM
+ * (small batches up to 64 rows, prefill batches up to 65536 rows in one
+ * launch), a grouped launcher for a decoder layer's projections and the
+ * gate/up pair with its SiLU-gated output.
  *
  * What the method fixes -- ThinkBit page, "ThinkBit은 2비트 양자화에서 추론
  * 능력 보존을 추론 평가로 검증한다" (onedev.kr/papers/1416):

@@ -307,8 +307,9 @@ def test_gemm_strided_bf16_out(oracle):
 @pytest.mark.parametrize("grid", GRIDS)
 @pytest.mark.parametrize("M", [65, 100, 128, 161])
 def test_gemm_prefill_blocks(oracle, grid, M):
-    """Batches above 64 rows run in one launch as blocks of 64 batch rows
-    (ragged last blocks of 1, 36 and 33 rows: rows past M read as zero)."""
+    """Batches above 64 rows run in one launch as blocks of 128 batch rows
+    (M = 65, 100: one ragged block; 161: a full block and a ragged one of
+    33 rows; rows past M are never stored)."""
     N, K = 80, 768
     W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=3100 + M)
     X = synth.activations(K, seed=3200 + M, M=M)
@@ -489,7 +490,7 @@ def test_zz_no_bounded_wait_gave_up():
 @pytest.mark.parametrize("M", [256, 1000])
 def test_gemm_prefill_gate_sampled(oracle, grid, M):
     """Prefill at the Qwen3-14B-like gate shape (17408 x 5120), M = 256 and
-    1000 batch rows (16 blocks of 64, the last ragged): 64 sampled output
+    1000 batch rows (8 blocks of 128, the last ragged): 64 sampled output
     rows (tile boundaries included) for 24 sampled batch rows (block
     boundaries included) against the oracle."""
     N, K = 17408, 5120
@@ -498,7 +499,7 @@ def test_gemm_prefill_gate_sampled(oracle, grid, M):
     Y = tb.tb_gemm(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), X.to(DEV), N, K).cpu()
     rng = np.random.default_rng(M + 7 * grid)
     rows = np.unique(np.concatenate([[0, 127, 128, N - 129, N - 128, N - 1], rng.integers(0, N, 58)]))
-    ms = np.unique(np.concatenate([[0, 63, 64, M - 1], rng.integers(0, M, 20)]))
+    ms = np.unique(np.concatenate([[0, 63, 64, 127, 128, M - 1], rng.integers(0, M, 20)]))
     Xb = u16(X)
     for m in ms:
         y64, yabs = oracle.gemv_rows64(p_ref, grid, s_ref, Xb[m], K, rows)
