@@ -52,8 +52,9 @@ struct Launch {
 // the accumulator start values of digit columns 2t, 2t+1 and the float
 // 2^(14 t - F) (64 bytes).
 constexpr int kG8RecBytes = 1088;
-constexpr int kG8Warps = 8;      // consumer warps of k_gemv8
-constexpr int kG8TileRows = 256;  // rows of a tile: 8 consumer warps x 32 rows
+constexpr int kG8TileRows = 256;  // rows of a tile
+constexpr int kG8WarpRows = 32;   // rows of a tile one consumer warp works on
+constexpr int kG8Warps = 2 * kG8TileRows / kG8WarpRows;  // consumer warps of k_gemv8: two per row block
 
 struct G8Item {
     const uint16_t* x;       // [K] bf16 activations

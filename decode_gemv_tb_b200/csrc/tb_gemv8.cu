@@ -36,7 +36,7 @@
 //     the offset sums) into the workspace.  Projections that read the same x
 //     with the same code width share a record set.  x is requested into L2
 //     at once and read once the previous kernel in the stream has finished.
-//   * k_gemv8: one CTA per SM, eight consumer warps and a producer warp.
+//   * k_gemv8: one CTA per SM, sixteen consumer warps and a producer warp.
 //     The work of a call is the sequence of chunks (item, tile of 256 rows,
 //     C consecutive groups: C = 4 for the 2-bit container, 2 for 3 bits) in
 //     item, tile, group order; each CTA owns a contiguous range of equal
@@ -48,12 +48,15 @@
 //     groups) into the stage -- inputs no earlier kernel writes, so the first
 //     four stages are requested at once, before the record kernel has
 //     finished -- and, once it has, the chunk's records (one bulk copy).
-//   * Consumer warp w decodes rows 64 (w & 3) .. 64 (w & 3) + 63 of the
-//     tile, for half of the chunk's groups (w >> 2), with LOP3 masks, runs
-//     four MMAs per 16 rows and group and accumulates in fp32; the two
-//     halves of a row block meet in shared memory at the end of a segment.
+//   * Sixteen consumer warps: warp w decodes the 32 rows of row block
+//     w mod 8 of the tile, for half of the chunk's groups (w / 8), with LOP3
+//     masks, runs four MMAs per 16 rows and group and accumulates in fp32;
+//     the two halves of a row block meet in shared memory at the end of a
+//     segment.  (Twice the warps of 64-row blocks hide more of the decode's
+//     fixed latencies; the record kernel's CTAs are kept small so that a
+//     waiting one never keeps the next call's main CTA off its SM.)
 // A stage is full when its copies have landed and the producer has
-// arrived; empty when all eight consumers have.  A tile whose groups are
+// arrived; empty when all consumers have.  A tile whose groups are
 // split between CTAs is combined by the CTA that reads its first chunk --
 // for which it is the last segment of its range, so the others have long
 // finished theirs: each later CTA publishes its partial sum of the tile's
@@ -74,6 +77,10 @@ __device__ unsigned int g_g8_timeouts = 0;  // bounded waits of this file's kern
 namespace {
 
 constexpr int kCWarps = kG8Warps;                  // consumer warps
+constexpr int kRB = kG8WarpRows;                   // rows of a consumer warp's row block
+constexpr int kNRB = kG8TileRows / kRB;            // row blocks of a tile (a warp pair each)
+constexpr int kRT = kRB / 16;                      // 16-row MMA tiles of a warp
+constexpr int kBL = kRB / 32;                      // 8-row blocks a lane finishes (blocks kBL t .. kBL t + kBL - 1)
 constexpr int kProducer = kCWarps;                 // the producer warp
 constexpr int kG8Threads = (kCWarps + 1) * 32;
 constexpr int kStages = 4;
@@ -82,7 +89,7 @@ constexpr int kSOff = 32768;                       // scales box: 256 rows x 8 b
 constexpr int kROff = kSOff + 4096;                // records copied from the workspace: up to 4 x 1088 bytes
 constexpr int kStageBytes = 41984;                 // >= kROff + 4 * kG8RecBytes, a multiple of 1 KB
 constexpr int kG8Smem = kStages * kStageBytes + 1024;  // + alignment slack (swizzled boxes: 1 KB)
-constexpr int kRecWarps = 8;                       // warps of a CTA of the record kernel
+constexpr int kRecWarps = 2;                       // warps of a CTA of the record kernel (small: see above)
 
 static_assert(kROff + 4 * kG8RecBytes <= kStageBytes, "stage layout");
 static_assert(kG8Smem <= 227 * 1024, "shared memory");
@@ -322,12 +329,12 @@ __global__ void __launch_bounds__(kRecWarps * 32) k_g8_records(const __grid_cons
 }
 
 // ---- consumer layout --------------------------------------------------------------
-// Consumer warp w works on the 64 rows 64 rb .. 64 rb + 63 of every tile
-// (rb = w & 3) and on half of every chunk's groups (gh = w >> 2: local
-// groups gh C/2 .. gh C/2 + C/2 - 1), so that each record is read by four
-// warps, not eight.  Lane (g, t) takes part in MMA rows g and g + 8 of the
-// warp's four 16-row MMA tiles rt: 8-row blocks i = 2 rt (rows g) and
-// i = 2 rt + 1 (rows g + 8), tile row 64 rb + 8 i + k7 with
+// Consumer warp w works on the kRB rows kRB rb .. kRB rb + kRB - 1 of every
+// tile (rb = w mod kNRB) and on half of every chunk's groups (gh = w / kNRB:
+// local groups gh C/2 .. gh C/2 + C/2 - 1), so that each record is read by
+// half of the warps.  Lane (g, t) takes part in MMA rows g and g + 8 of the
+// warp's kRT 16-row MMA tiles rt: 8-row blocks i = 2 rt (rows g) and
+// i = 2 rt + 1 (rows g + 8), tile row kRB rb + 8 i + k7 with
 // k7 = 2 (g & 3) + (g >> 2).  The eight lane groups of a block differ in
 // row & 7 = k7, which keeps the 128-byte-swizzled weight loads free of bank
 // conflicts, and block i of a lane is block 0 plus i x 8 rows: a constant
@@ -343,7 +350,7 @@ struct LaneOff {
 
 __device__ __forceinline__ LaneOff lane_offsets(int rb, int gh, int g, int t) {
     LaneOff o;
-    const int k7 = lane_k7(g), r = 64 * rb + k7;
+    const int k7 = lane_k7(g), r = kRB * rb + k7;
 #pragma unroll
     for (int q = 0; q < 2; ++q)
         o.w2[q] = (uint32_t)(r * 128 + (((2 * (2 * gh + q) + (t >> 1)) ^ k7) << 4) + 8 * (t & 1));
@@ -353,17 +360,17 @@ __device__ __forceinline__ LaneOff lane_offsets(int rb, int gh, int g, int t) {
 }
 
 // The warp's groups of one chunk (geff groups present; `recs` holds the
-// chunk's records in order) for the lane's eight row blocks.
+// chunk's records in order) for the lane's 2 kRT row blocks.
 template <int KIND>
 __device__ __forceinline__ void g8_chunk(const uint8_t* stage, const uint8_t* recs, const LaneOff& o, int geff,
-                                         int gh, int scol, int lane, int t, float (&acc)[8]) {
+                                         int gh, int scol, int lane, int t, float (&acc)[2 * kRT]) {
     constexpr int C = KIND ? 2 : 4, CW = C / 2, WROW = KIND ? 96 * 8 : 128 * 8;
     const int gl0 = gh * CW;
     if (gl0 >= geff) return;  // the ragged end of a row: this half has no group
     // the scales of the warp's groups, per row block (2-bit: two bf16 in one word; 3-bit: one, as fp32 bits)
-    uint32_t sv[8];
+    uint32_t sv[2 * kRT];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 2 * kRT; ++i) {
         const uint8_t* p = stage + o.sc + 128 * i + 2 * (scol + gl0);
         sv[i] = KIND ? (uint32_t)*reinterpret_cast<const uint16_t*>(p) << 16 : *reinterpret_cast<const uint32_t*>(p);
     }
@@ -377,7 +384,7 @@ __device__ __forceinline__ void g8_chunk(const uint8_t* stage, const uint8_t* re
         const float et = __uint_as_float(H.z);
         const uint8_t* wb = stage + (KIND ? o.w3 : o.w2[q]);
 #pragma unroll
-        for (int rt = 0; rt < 4; ++rt) {
+        for (int rt = 0; rt < kRT; ++rt) {
             uint32_t R[2][8];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -437,80 +444,81 @@ __device__ __forceinline__ void pair_epilogue(const G8Launch& L, int item, int64
 // tile that later ranges finish (combine).
 enum SegKind { kWhole = 0, kPublish = 1, kCombine = 2 };
 
-// Rows rin and rin + 8 at the end of a segment (sums over this range's
+// Rows rin + 8 b (b < kBL) at the end of a segment (sums over this range's
 // chunks of the tile): publish them, or add the later ranges' words in CTA
-// order (the words of both rows and two ranges in flight at a time), then
-// write y.
+// order (the words of the lane's rows and two ranges in flight at a time),
+// then write y.
 __device__ __forceinline__ void finish_rows(const G8Launch& L, int cta, int item, uint32_t tile, int kind, int rin,
-                                            uint32_t c1, float s0, float s1) {
+                                            uint32_t c1, float (&s)[kBL]) {
     if (kind == kPublish) {
-        st_word(L.pslots + (int64_t)cta * kG8TileRows + rin, flagged(s0));
-        st_word(L.pslots + (int64_t)cta * kG8TileRows + rin + 8, flagged(s1));
+#pragma unroll
+        for (int b = 0; b < kBL; ++b) st_word(L.pslots + (int64_t)cta * kG8TileRows + rin + 8 * b, flagged(s[b]));
         return;
     }
     if (kind == kCombine) {  // the later ranges that read this tile, in order
         for (uint32_t c = (uint32_t)cta + 1; c <= c1; c += 2) {
-            uint64_t* slot[4];
-            uint64_t wv[4];
+            uint64_t* slot[2 * kBL];
+            uint64_t wv[2 * kBL];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {  // q: range c + (q >> 1), row rin + 8 (q & 1)
-                slot[q] = L.pslots + (int64_t)(c + (q >> 1)) * kG8TileRows + rin + 8 * (q & 1);
-                wv[q] = c + (q >> 1) <= c1 ? ld_word(slot[q]) : 0;
+            for (int q = 0; q < 2 * kBL; ++q) {  // q: range c + q / kBL, row rin + 8 (q % kBL)
+                slot[q] = L.pslots + (int64_t)(c + q / kBL) * kG8TileRows + rin + 8 * (q % kBL);
+                wv[q] = c + q / kBL <= c1 ? ld_word(slot[q]) : 0;
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (c + (q >> 1) > c1) break;
+            for (int q = 0; q < 2 * kBL; ++q) {
+                if (c + q / kBL > c1) break;
                 float p = __uint_as_float((uint32_t)wv[q]);
                 if (!(wv[q] >> 32) && !wait_word(slot[q], L.wait_cycles, &p)) {
                     atomicAdd(&g_g8_timeouts, 1u);
                     p = __int_as_float(0x7FC00000);
                 }
                 st_word(slot[q], 0);
-                if (q & 1) s1 += p;
-                else s0 += p;
+                s[q % kBL] += p;
             }
         }
     }
     const int64_t row = (int64_t)tile * kG8TileRows + rin;
-    store_y(L.it[item], row, s0);
-    store_y(L.it[item], row + 8, s1);
-    pair_epilogue(L, item, row, s0);
-    pair_epilogue(L, item, row + 8, s1);
+#pragma unroll
+    for (int b = 0; b < kBL; ++b) store_y(L.it[item], row + 8 * b, s[b]);
+#pragma unroll
+    for (int b = 0; b < kBL; ++b) pair_epilogue(L, item, row + 8 * b, s[b]);
 }
 
 // End of a warp's segment of a tile: the quad's digit pairs are summed, the
 // group half gh = 1 hands its sums to gh = 0 through shared memory (double
 // buffered by `flip`), which adds them (gh 0 + gh 1) and finishes the rows.
 struct Acc8 {
-    float v[8];
+    float v[2 * kRT];
 };
 
 __device__ __noinline__ void g8_flush(const G8Launch& L, int cta, int rb, int gh, int item, uint32_t tile, int kind,
                                       const Acc8 acc, float* pairbuf, int flip) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    float v[8];
+    float v[2 * kRT];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {  // the same sum in all four lanes of the quad
+    for (int i = 0; i < 2 * kRT; ++i) {  // the same sum in all four lanes of the quad
         v[i] = acc.v[i] + __shfl_xor_sync(0xffffffffu, acc.v[i], 1);
         v[i] += __shfl_xor_sync(0xffffffffu, v[i], 2);
     }
-    // lane t keeps blocks 2t and 2t + 1
-    float m0 = v[0], m1 = v[1];
+    // lane t keeps blocks kBL t .. kBL t + kBL - 1
+    float m[kBL];
+#pragma unroll
+    for (int b = 0; b < kBL; ++b) m[b] = v[b];
 #pragma unroll
     for (int q = 1; q < 4; ++q)
         if (t == q) {
-            m0 = v[2 * q];
-            m1 = v[2 * q + 1];
+#pragma unroll
+            for (int b = 0; b < kBL; ++b) m[b] = v[kBL * q + b];
         }
-    float* pb = pairbuf + flip * kG8TileRows + rb * 64 + 2 * lane;
+    float* pb = pairbuf + flip * kG8TileRows + rb * kRB + kBL * lane;
     if (gh == 1) {
-        pb[0] = m0;
-        pb[1] = m1;
+#pragma unroll
+        for (int b = 0; b < kBL; ++b) pb[b] = m[b];
     }
     named_sync(2 + rb, 64);
     if (gh == 1) return;
-    m0 += pb[0];
-    m1 += pb[1];
+#pragma unroll
+    for (int b = 0; b < kBL; ++b) m[b] += pb[b];
     const G8Item& I = L.it[item];
     uint32_t c1 = 0;
     if (kind == kCombine) {
@@ -518,8 +526,8 @@ __device__ __noinline__ void g8_flush(const G8Launch& L, int cta, int rb, int gh
         c1 = part_owner((uint32_t)I.cost_base + tile * (uint32_t)I.G * uc + (uint32_t)(I.cpt - 1) * (uint32_t)I.C * uc,
                         L.Q);
     }
-    const int rin = 64 * rb + 16 * t + lane_k7(g);  // block 2t; block 2t + 1 is 8 rows on
-    finish_rows(L, cta, item, tile, kind, rin, c1, m0, m1);
+    const int rin = kRB * rb + 8 * kBL * t + lane_k7(g);  // block kBL t; the next ones 8 rows on each
+    finish_rows(L, cta, item, tile, kind, rin, c1, m);
 }
 
 __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__ G8Launch L) {
@@ -651,7 +659,7 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
     pdl_wait();  // y and the workspace may still be in use by the previous kernels in the stream
     const int w = warp, g = lane >> 2, t = lane & 3;
     if (n == 0) return;
-    const int rb = w & 3, gh = w >> 2;
+    const int rb = w % kNRB, gh = w / kNRB;
     const LaneOff off = lane_offsets(rb, gh, g, t);
     Cur c = first_cur();
     // the fields of the item under the cursor, in registers (re-read when it changes)
@@ -659,7 +667,9 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
     bool it_three = L.it[c.item].grid == kInt3;
     bool failed = false;
     int flip = 0;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float acc[2 * kRT];
+#pragma unroll
+    for (int i = 0; i < 2 * kRT; ++i) acc[i] = 0.f;
 #pragma unroll 1
     for (int32_t k = 0; k < n; ++k) {
         const int s = k % kStages;
@@ -684,7 +694,7 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
             if (lane == 0) bar_arrive(saddr(&empty[s]));
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = __int_as_float(0x7FC00000);
+            for (int i = 0; i < 2 * kRT; ++i) acc[i] = __int_as_float(0x7FC00000);
         }
         const bool more = k + 1 < n;
         if (c.j + 1 == it_cpt || !more) {  // end of the range's segment of this tile
@@ -692,11 +702,11 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
             const int kind = first < cb ? kPublish : (first + (uint32_t)it_cpt > ce ? kCombine : kWhole);
             Acc8 a8;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) a8.v[i] = acc[i];
+            for (int i = 0; i < 2 * kRT; ++i) a8.v[i] = acc[i];
             g8_flush(L, cta, rb, gh, c.item, c.tile, kind, a8, pairbuf, flip);
             flip ^= 1;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+            for (int i = 0; i < 2 * kRT; ++i) acc[i] = 0.f;
         }
         // advance the cursor (the item's fields are reloaded only when it changes)
         if (++c.j == it_cpt) {
