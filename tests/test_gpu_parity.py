@@ -524,3 +524,21 @@ def test_gemm_prefill_largest_batch(oracle, grid):
         y64, yabs = oracle.gemv_rows64(p_ref, grid, s_ref, Xb[m], K, rows)
         assert_within(Y[m], y64, yabs, "f32", oracle, f"M=65536 m={m}")
     assert tb.wait_timeouts() == 0
+
+
+@pytest.mark.parametrize("grid", [tb.INT2, tb.INT3])
+def test_gemm_prefill_is_deterministic(oracle, grid):
+    """Units split between CTAs are combined in CTA order: two prefill calls
+    on the same inputs give bitwise the same result (and a third, after a
+    call of another shape through the same workspace, too)."""
+    N, K, M = 4096, 5120, 300
+    W, _, s_ref, p_ref = oracle_problem(oracle, grid, N, K, seed=5400 + grid)
+    X = synth.activations(K, seed=5500 + grid, M=M).to(DEV)
+    p, s = to_dev_packed(p_ref), to_dev_bits(s_ref)
+    ws = tb.workspace(max(tb.workspace_bytes(M, N, K), tb.workspace_bytes(77, N, K)), DEV)
+    y1 = tb.tb_gemm(p, grid, s, X, N, K, ws=ws)
+    y2 = tb.tb_gemm(p, grid, s, X, N, K, ws=ws)
+    tb.tb_gemm(p, grid, s, X[:77].contiguous(), N, K, ws=ws)
+    y3 = tb.tb_gemm(p, grid, s, X, N, K, ws=ws)
+    assert torch.equal(y1, y2) and torch.equal(y1, y3)
+    assert tb.wait_timeouts() == 0
