@@ -89,7 +89,7 @@ constexpr int kSOff = 32768;                       // scales box: 256 rows x 8 b
 constexpr int kROff = kSOff + 4096;                // records copied from the workspace: up to 4 x 1088 bytes
 constexpr int kStageBytes = 41984;                 // >= kROff + 4 * kG8RecBytes, a multiple of 1 KB
 constexpr int kG8Smem = kStages * kStageBytes + 1024;  // + alignment slack (swizzled boxes: 1 KB)
-constexpr int kRecWarps = 2;                       // warps of a CTA of the record kernel (small: see above)
+constexpr int kRecWarps = 1;                       // warps of a CTA of the record kernel (small: see above)
 
 static_assert(kROff + 4 * kG8RecBytes <= kStageBytes, "stage layout");
 static_assert(kG8Smem <= 227 * 1024, "shared memory");
