@@ -165,13 +165,18 @@ tb_status_t launch_items(Item* items, int n, int nt, cudaStream_t st) {
 // read and sit at the BACK.  A call needs 2 max(control, data) bytes,
 // so calls of different shapes can share one workspace sized for the
 // largest: no call's data ever reaches another call's control words.
-constexpr int64_t kMaxG8Ctas = 256;      // bound of the CTA count (partial-sum words)
+constexpr int64_t kMaxG8Ctas = 512;      // bound of the CTA count (partial-sum words)
 constexpr int64_t kG8Rows = kG8TileRows;
 // Cost of one 128-group of one 256-row tile in the equal-cost split: a
 // 3-bit group takes about twice the consumer work of a 2-bit one (measured
 // on the 8B-like stack), so every chunk (four 2-bit or two 3-bit groups)
 // costs the same
 constexpr int32_t kG8Cost2 = 2, kG8Cost3 = 4;
+// chunks per SM from which a call runs two CTAs per SM: below it (single
+// q/k/v, o, down or gate/up calls of an 8B-like layer) one CTA per SM with
+// a deeper ring finishes first; from it (a whole layer in one call) two
+// independent rings per SM stream faster
+constexpr int64_t kG8TwoPerSm = 8;
 constexpr long long kWaitCycles = 4000000000LL;      // about 2 s
 constexpr long long kTestWaitCycles = 20000000LL;    // about 10 ms (TB_FLAG_TEST_STALL)
 
@@ -274,7 +279,13 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
         if (!encode_g8_wmap(&L.wmap[j], items[j].packed, items[j].grid, s.N, items[j].K)) return TB_ERR_CUDA;
         if (!s.stage_scales && !encode_g8_smap(&L.smap[j], s.scales, s.N, s.G)) return TB_ERR_CUDA;
     }
-    const int resident = gemv8_ctas();
+    // many chunks per SM: two CTAs per SM (two independent rings); else one
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return TB_ERR_CUDA;
+    const bool two = chunk >= (int64_t)kG8TwoPerSm * sms;
+    const int resident = gemv8_ctas(two);
     if (resident <= 0) return TB_ERR_CUDA;
     // every quota at least one chunk's cost: then every CTA
     // between a tile's first and last owner owns a chunk of it, which the
@@ -302,7 +313,7 @@ tb_status_t launch_g8_items(const Item* items, int n, void* ws, size_t ws_bytes,
     }
     L.stall = stall ? 1 : 0;
     L.wait_cycles = stall ? kTestWaitCycles : kWaitCycles;
-    return cuda_status(launch_gemv8(L, overlap, st));
+    return cuda_status(launch_gemv8(L, two, overlap, st));
 }
 
 // the items of a layer call that run on the integer tensor path

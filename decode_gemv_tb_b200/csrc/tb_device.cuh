@@ -53,8 +53,6 @@ struct Launch {
 // 2^(14 t - F) (64 bytes).
 constexpr int kG8RecBytes = 1088;
 constexpr int kG8TileRows = 256;  // rows of a tile
-constexpr int kG8WarpRows = 32;   // rows of a tile one consumer warp works on
-constexpr int kG8Warps = 2 * kG8TileRows / kG8WarpRows;  // consumer warps of k_gemv8: two per row block
 
 struct G8Item {
     const uint16_t* x;       // [K] bf16 activations
@@ -83,7 +81,7 @@ struct G8Range {
     uint32_t cb, ce;
     int32_t item, tile, j;
 };
-constexpr int kMaxG8Ranges = 256;
+constexpr int kMaxG8Ranges = 512;
 
 struct G8Launch {
     CUtensorMap wmap[kMaxItems];  // packed weights: bytes x rows, box (C groups) x 256 rows

@@ -36,25 +36,32 @@
 //     the offset sums) into the workspace.  Projections that read the same x
 //     with the same code width share a record set.  x is requested into L2
 //     at once and read once the previous kernel in the stream has finished.
-//   * k_gemv8: one CTA per SM, sixteen consumer warps and a producer warp.
+//   * k_gemv8 in one of two layouts, chosen per call by its chunks per
+//     SM: one CTA per SM with sixteen consumer warps, a producer warp and
+//     four stages (calls of a few chunks per SM), or two CTAs per SM, each
+//     eight consumer warps, a producer and two stages (two independent
+//     rings per SM; calls of many chunks per SM).
 //     The work of a call is the sequence of chunks (item, tile of 256 rows,
 //     C consecutive groups: C = 4 for the 2-bit container, 2 for 3 bits) in
 //     item, tile, group order; each CTA owns a contiguous range of equal
 //     cost (tb_partition.h: a 3-bit group costs twice a 2-bit one, so every
 //     chunk costs the same).
-//   * Stages.  Each chunk passes through a ring of four shared-memory
-//     stages.  The producer copies the packed weights (a 2-D tensor copy of
+//   * Stages.  Each chunk passes through a ring of shared-memory stages
+//     per CTA.  The producer copies the packed weights (a 2-D tensor copy of
 //     256 rows x 128 or 96 bytes, no multicast) and the scales (256 rows x 8
-//     groups) into the stage -- inputs no earlier kernel writes, so the first
-//     four stages are requested at once, before the record kernel has
-//     finished -- and, once it has, the chunk's records (one bulk copy).
-//   * Sixteen consumer warps: warp w decodes the 32 rows of row block
-//     w mod 8 of the tile, for half of the chunk's groups (w / 8), with LOP3
-//     masks, runs four MMAs per 16 rows and group and accumulates in fp32;
-//     the two halves of a row block meet in shared memory at the end of a
-//     segment.  (Twice the warps of 64-row blocks hide more of the decode's
-//     fixed latencies; the record kernel's CTAs are kept small so that a
-//     waiting one never keeps the next call's main CTA off its SM.)
+//     groups) into the stage -- inputs no earlier kernel writes, so both
+//     first stages are requested at once, before the record kernel has finished --
+//     and, once it has, the chunk's records (one bulk copy).
+//   * Consumer warp w decodes the rows of row block w mod R of the tile
+//     (R = 8 blocks of 32 rows, or 4 of 64 rows in the two-CTA layout),
+//     for half of the chunk's groups (w / R), with LOP3 masks, runs four MMAs
+//     per 16 rows and group and accumulates in fp32; the two halves of a row
+//     block meet in shared memory at the end of a segment.  (Sixteen
+//     consumer warps per SM hide more of the decode's fixed latencies than
+//     eight; on long ranges two CTAs with independent rings more than one
+//     with sixteen warps, on short ones the deeper ring of one CTA wins.
+//     The record kernel's CTAs are one warp, so that waiting ones
+//     never keep the next call's main CTAs off their SM.)
 // A stage is full when its copies have landed and the producer has
 // arrived; empty when all consumers have.  A tile whose groups are
 // split between CTAs is combined by the CTA that reads its first chunk --
@@ -76,23 +83,35 @@ __device__ unsigned int g_g8_timeouts = 0;  // bounded waits of this file's kern
 
 namespace {
 
-constexpr int kCWarps = kG8Warps;                  // consumer warps
-constexpr int kRB = kG8WarpRows;                   // rows of a consumer warp's row block
-constexpr int kNRB = kG8TileRows / kRB;            // row blocks of a tile (a warp pair each)
-constexpr int kRT = kRB / 16;                      // 16-row MMA tiles of a warp
-constexpr int kBL = kRB / 32;                      // 8-row blocks a lane finishes (blocks kBL t .. kBL t + kBL - 1)
-constexpr int kProducer = kCWarps;                 // the producer warp
-constexpr int kG8Threads = (kCWarps + 1) * 32;
-constexpr int kStages = 4;
-constexpr int kEarly = kStages;                    // stages filled before the previous kernel has finished
 constexpr int kSOff = 32768;                       // scales box: 256 rows x 8 bf16
 constexpr int kROff = kSOff + 4096;                // records copied from the workspace: up to 4 x 1088 bytes
 constexpr int kStageBytes = 41984;                 // >= kROff + 4 * kG8RecBytes, a multiple of 1 KB
-constexpr int kG8Smem = kStages * kStageBytes + 1024;  // + alignment slack (swizzled boxes: 1 KB)
+
+// The two layouts of k_gemv8, chosen per call by its chunks per SM (host):
+//   G8One: one CTA per SM, sixteen consumer warps of 32 rows, four stages
+//     (calls with few chunks per SM: deep rings, few split tiles);
+//   G8Two: two CTAs per SM, each eight consumer warps of 64 rows and two
+//     stages (calls with many chunks per SM: two independent rings).
+template <int WR, int NS, int MINB>
+struct G8Cfg {
+    static constexpr int kRB = WR;                    // rows of a consumer warp's row block
+    static constexpr int kNRB = kG8TileRows / WR;     // row blocks of a tile (a warp pair each)
+    static constexpr int kRT = WR / 16;               // 16-row MMA tiles of a warp
+    static constexpr int kBL = WR / 32;               // 8-row blocks a lane finishes (kBL t .. kBL t + kBL - 1)
+    static constexpr int kCWarps = 2 * kNRB;          // consumer warps
+    static constexpr int kProducer = kCWarps;         // the producer warp
+    static constexpr int kThreads = (kCWarps + 1) * 32;
+    static constexpr int kStages = NS;
+    static constexpr int kEarly = NS;                 // stages filled before the previous kernel has finished
+    static constexpr int kMinBlocks = MINB;           // CTAs per SM
+    static constexpr int kSmem = NS * kStageBytes + 1024;  // + alignment slack (swizzled boxes: 1 KB)
+    static_assert(kSmem * MINB <= 227 * 1024, "shared memory");
+};
+using G8One = G8Cfg<32, 4, 1>;
+using G8Two = G8Cfg<64, 2, 2>;
 constexpr int kRecWarps = 1;                       // warps of a CTA of the record kernel (small: see above)
 
 static_assert(kROff + 4 * kG8RecBytes <= kStageBytes, "stage layout");
-static_assert(kG8Smem <= 227 * 1024, "shared memory");
 
 // ---- small PTX helpers ------------------------------------------------------
 __device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -348,9 +367,10 @@ struct LaneOff {
     uint32_t sc;     // scales, column 0
 };
 
+template <class Cfg>
 __device__ __forceinline__ LaneOff lane_offsets(int rb, int gh, int g, int t) {
     LaneOff o;
-    const int k7 = lane_k7(g), r = kRB * rb + k7;
+    const int k7 = lane_k7(g), r = Cfg::kRB * rb + k7;
 #pragma unroll
     for (int q = 0; q < 2; ++q)
         o.w2[q] = (uint32_t)(r * 128 + (((2 * (2 * gh + q) + (t >> 1)) ^ k7) << 4) + 8 * (t & 1));
@@ -361,16 +381,16 @@ __device__ __forceinline__ LaneOff lane_offsets(int rb, int gh, int g, int t) {
 
 // The warp's groups of one chunk (geff groups present; `recs` holds the
 // chunk's records in order) for the lane's 2 kRT row blocks.
-template <int KIND>
+template <class Cfg, int KIND>
 __device__ __forceinline__ void g8_chunk(const uint8_t* stage, const uint8_t* recs, const LaneOff& o, int geff,
-                                         int gh, int scol, int lane, int t, float (&acc)[2 * kRT]) {
+                                         int gh, int scol, int lane, int t, float (&acc)[2 * Cfg::kRT]) {
     constexpr int C = KIND ? 2 : 4, CW = C / 2, WROW = KIND ? 96 * 8 : 128 * 8;
     const int gl0 = gh * CW;
     if (gl0 >= geff) return;  // the ragged end of a row: this half has no group
     // the scales of the warp's groups, per row block (2-bit: two bf16 in one word; 3-bit: one, as fp32 bits)
-    uint32_t sv[2 * kRT];
+    uint32_t sv[2 * Cfg::kRT];
 #pragma unroll
-    for (int i = 0; i < 2 * kRT; ++i) {
+    for (int i = 0; i < 2 * Cfg::kRT; ++i) {
         const uint8_t* p = stage + o.sc + 128 * i + 2 * (scol + gl0);
         sv[i] = KIND ? (uint32_t)*reinterpret_cast<const uint16_t*>(p) << 16 : *reinterpret_cast<const uint32_t*>(p);
     }
@@ -384,7 +404,7 @@ __device__ __forceinline__ void g8_chunk(const uint8_t* stage, const uint8_t* re
         const float et = __uint_as_float(H.z);
         const uint8_t* wb = stage + (KIND ? o.w3 : o.w2[q]);
 #pragma unroll
-        for (int rt = 0; rt < kRT; ++rt) {
+        for (int rt = 0; rt < Cfg::kRT; ++rt) {
             uint32_t R[2][8];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -448,8 +468,10 @@ enum SegKind { kWhole = 0, kPublish = 1, kCombine = 2 };
 // chunks of the tile): publish them, or add the later ranges' words in CTA
 // order (the words of the lane's rows and two ranges in flight at a time),
 // then write y.
+template <class Cfg>
 __device__ __forceinline__ void finish_rows(const G8Launch& L, int cta, int item, uint32_t tile, int kind, int rin,
-                                            uint32_t c1, float (&s)[kBL]) {
+                                            uint32_t c1, float (&s)[Cfg::kBL]) {
+    constexpr int kBL = Cfg::kBL;
     if (kind == kPublish) {
 #pragma unroll
         for (int b = 0; b < kBL; ++b) st_word(L.pslots + (int64_t)cta * kG8TileRows + rin + 8 * b, flagged(s[b]));
@@ -487,12 +509,15 @@ __device__ __forceinline__ void finish_rows(const G8Launch& L, int cta, int item
 // End of a warp's segment of a tile: the quad's digit pairs are summed, the
 // group half gh = 1 hands its sums to gh = 0 through shared memory (double
 // buffered by `flip`), which adds them (gh 0 + gh 1) and finishes the rows.
-struct Acc8 {
-    float v[2 * kRT];
+template <class Cfg>
+struct AccT {
+    float v[2 * Cfg::kRT];
 };
 
+template <class Cfg>
 __device__ __noinline__ void g8_flush(const G8Launch& L, int cta, int rb, int gh, int item, uint32_t tile, int kind,
-                                      const Acc8 acc, float* pairbuf, int flip) {
+                                      const AccT<Cfg> acc, float* pairbuf, int flip) {
+    constexpr int kRT = Cfg::kRT, kBL = Cfg::kBL, kRB = Cfg::kRB;
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     float v[2 * kRT];
 #pragma unroll
@@ -527,10 +552,13 @@ __device__ __noinline__ void g8_flush(const G8Launch& L, int cta, int rb, int gh
                         L.Q);
     }
     const int rin = kRB * rb + 8 * kBL * t + lane_k7(g);  // block kBL t; the next ones 8 rows on each
-    finish_rows(L, cta, item, tile, kind, rin, c1, m);
+    finish_rows<Cfg>(L, cta, item, tile, kind, rin, c1, m);
 }
 
-__global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__ G8Launch L) {
+template <class Cfg>
+__global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks) k_gemv8(const __grid_constant__ G8Launch L) {
+    constexpr int kStages = Cfg::kStages, kEarly = Cfg::kEarly, kCWarps = Cfg::kCWarps, kProducer = Cfg::kProducer;
+    constexpr int kNRB = Cfg::kNRB, kRT = Cfg::kRT;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
     __shared__ int producer_failed;  // set before the producer completes stages it could not fill
@@ -660,7 +688,7 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
     const int w = warp, g = lane >> 2, t = lane & 3;
     if (n == 0) return;
     const int rb = w % kNRB, gh = w / kNRB;
-    const LaneOff off = lane_offsets(rb, gh, g, t);
+    const LaneOff off = lane_offsets<Cfg>(rb, gh, g, t);
     Cur c = first_cur();
     // the fields of the item under the cursor, in registers (re-read when it changes)
     int it_C = L.it[c.item].C, it_G = L.it[c.item].G, it_cpt = L.it[c.item].cpt, it_T = L.it[c.item].T;
@@ -688,8 +716,8 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
             const int geff = min(it_C, it_G - c.j * it_C);
             const int scol = (c.j * it_C) & 7;
             const uint8_t* recs = stage + kROff;
-            if (it_three) g8_chunk<1>(stage, recs, off, geff, gh, scol, lane, t, acc);
-            else g8_chunk<0>(stage, recs, off, geff, gh, scol, lane, t, acc);
+            if (it_three) g8_chunk<Cfg, 1>(stage, recs, off, geff, gh, scol, lane, t, acc);
+            else g8_chunk<Cfg, 0>(stage, recs, off, geff, gh, scol, lane, t, acc);
             __syncwarp();
             if (lane == 0) bar_arrive(saddr(&empty[s]));
         } else {
@@ -700,10 +728,10 @@ __global__ void __launch_bounds__(kG8Threads, 1) k_gemv8(const __grid_constant__
         if (c.j + 1 == it_cpt || !more) {  // end of the range's segment of this tile
             const uint32_t first = (uint32_t)L.it[c.item].chunk_base + c.tile * (uint32_t)it_cpt;
             const int kind = first < cb ? kPublish : (first + (uint32_t)it_cpt > ce ? kCombine : kWhole);
-            Acc8 a8;
+            AccT<Cfg> a8;
 #pragma unroll
             for (int i = 0; i < 2 * kRT; ++i) a8.v[i] = acc[i];
-            g8_flush(L, cta, rb, gh, c.item, c.tile, kind, a8, pairbuf, flip);
+            g8_flush<Cfg>(L, cta, rb, gh, c.item, c.tile, kind, a8, pairbuf, flip);
             flip ^= 1;
 #pragma unroll
             for (int i = 0; i < 2 * kRT; ++i) acc[i] = 0.f;
@@ -760,8 +788,10 @@ bool prepare_device(int dev) {
     static bool ready[64] = {false};
     if (dev < 0 || dev >= 64) return false;
     if (!ready[dev]) {
-        if (cudaFuncSetAttribute((const void*)k_gemv8, cudaFuncAttributeMaxDynamicSharedMemorySize, kG8Smem) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute((const void*)k_gemv8<G8One>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 G8One::kSmem) != cudaSuccess ||
+            cudaFuncSetAttribute((const void*)k_gemv8<G8Two>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 G8Two::kSmem) != cudaSuccess)
             return false;
         ready[dev] = true;
     }
@@ -802,26 +832,28 @@ bool encode_g8_smap(CUtensorMap* map, const uint16_t* scales, int64_t N, int64_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int gemv8_ctas() {
-    static int ctas[64] = {0};
+int gemv8_ctas(bool two) {
+    static int ctas[64][2] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (ctas[dev] == 0) {
+    int& c = ctas[dev][two ? 1 : 0];
+    if (c == 0) {
         int sms = 0, per_sm = 0;
         if (!prepare_device(dev)) return 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv8, kG8Threads, kG8Smem) != cudaSuccess ||
-            per_sm < 1)
-            return 0;
-        ctas[dev] = sms * per_sm;
+        const cudaError_t e =
+            two ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv8<G8Two>, G8Two::kThreads, G8Two::kSmem)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv8<G8One>, G8One::kThreads, G8One::kSmem);
+        if (e != cudaSuccess || per_sm < 1) return 0;
+        c = sms * per_sm;
     }
-    return ctas[dev];
+    return c;
 }
 
 // The record kernel, then the main kernel as its programmatic dependent
 // (it streams weights while the records are built).  `overlap` lets the
 // record kernel, in turn, start before the previous work in the stream ends.
-cudaError_t launch_gemv8(const G8Launch& L, bool overlap, cudaStream_t st) {
+cudaError_t launch_gemv8(const G8Launch& L, bool two, bool overlap, cudaStream_t st) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -830,7 +862,11 @@ cudaError_t launch_gemv8(const G8Launch& L, bool overlap, cudaStream_t st) {
     const unsigned rec_ctas = (unsigned)((L.n_build + kRecWarps - 1) / kRecWarps);
     e = launch_with_pdl((const void*)k_g8_records, args, rec_ctas, kRecWarps * 32, 0, st, overlap);
     if (e != cudaSuccess) return e;
-    return launch_with_pdl((const void*)k_gemv8, args, (unsigned)L.nctas, kG8Threads, kG8Smem, st, true);
+    if (two)
+        return launch_with_pdl((const void*)k_gemv8<G8Two>, args, (unsigned)L.nctas, G8Two::kThreads, G8Two::kSmem,
+                               st, true);
+    return launch_with_pdl((const void*)k_gemv8<G8One>, args, (unsigned)L.nctas, G8One::kThreads, G8One::kSmem, st,
+                           true);
 }
 
 unsigned int take_g8_timeouts() {

@@ -32,14 +32,17 @@ struct G8Launch;
 // Batch-1 GEMV on the integer tensor path (tb_gemv8.cu): one kernel,
 // k_gemv8.  `overlap` launches it as a programmatic dependent of the
 // previous work (it streams weights before that work has finished).
-cudaError_t launch_gemv8(const G8Launch& L, bool overlap, cudaStream_t st);
+// `two`: the layout of two CTAs per SM (calls of many chunks per SM), else
+// one CTA per SM.
+cudaError_t launch_gemv8(const G8Launch& L, bool two, bool overlap, cudaStream_t st);
 // weights of one matrix (box: one chunk x 256 rows) / its scales [N][G] (G % 8 == 0)
 bool encode_g8_wmap(CUtensorMap* map, const void* packed, int grid, int64_t N, int64_t K);
 bool encode_g8_smap(CUtensorMap* map, const uint16_t* scales, int64_t N, int64_t Gp);
 // groups per chunk (4 for the 2-bit container, 2 for 3 bits)
 int g8_chunk_groups(int grid);
-// CTAs of k_gemv8 resident at once on the current device (0 on error)
-int gemv8_ctas();
+// CTAs of k_gemv8 resident at once on the current device in the layout
+// `two` (0 on error)
+int gemv8_ctas(bool two);
 // bounded waits of k_gemv8 that gave up since the last call (clears)
 unsigned int take_g8_timeouts();
 

@@ -184,7 +184,7 @@ TB_API tb_status_t tb_unpack(const void *packed, tb_grid_t grid, int64_t N, int6
  *     control: per CTA 256 flagged partial-sum words (tiles whose K range
  *       is split between CTAs are combined in a fixed order by the CTA that
  *       reads the tile's start):
- *         ceil256(2048 * min(256, T1 * ceil(G / 2)));
+ *         ceil256(2048 * min(512, T1 * ceil(G / 2)));
  *     data: the activation records of x (1088 bytes per 128-group, built
  *       once per call by the call's first kernel):
  *         ceil256(1088 * G);

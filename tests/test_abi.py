@@ -85,11 +85,11 @@ def test_workspace_sizes(lib):
         control, data = al(4 * ctas), al(ctas * 128 * 128 * 4)
         assert tb.workspace_bytes(M, N, K) == 2 * max(control, data), (M, N, K)
     for N, K in ((1, 128), (256, 1024), (17408, 5120), (100, 1408), (4096, 12288)):
-        # batch 1: control = 256 flagged 8-byte partial words per CTA (at most 256 CTAs, at most one per
+        # batch 1: control = 256 flagged 8-byte partial words per CTA (at most 512 CTAs, at most one per
         # chunk of two groups); data = the activation records of x (1088 bytes per group); size
         # 2 max(control, data)
         G, tiles = K // 128, (N + 255) // 256
-        ctas = min(256, tiles * -(-G // 2))
+        ctas = min(512, tiles * -(-G // 2))
         control, data = al(2048 * ctas), al(1088 * G)
         assert tb.workspace_bytes(1, N, K) == 2 * max(control, data)
     assert tb.workspace_bytes(0, 8, 128) == 0 and tb.workspace_bytes(1, 8, 100) == 0
@@ -105,13 +105,13 @@ def test_workspace_sizes(lib):
     # chunks of two 3-bit groups or four 2-bit groups per 256-row tile
     chunks = sum((N + 255) // 256 * -(-(K // 128) // (2 if grid == 2 else 4)) for N, K, grid, _ in shapes)
     rec = sum(al(1088 * (K // 128)) for i, (_, K, _, _) in enumerate(shapes) if i != 2)
-    control, data = al(2048 * min(256, chunks)), rec
+    control, data = al(2048 * min(512, chunks)), rec
     assert tb.layer_workspace_bytes(items) == 2 * max(control, data)
     # a layer whose records outweigh its control words
     wide = (tb.Linear * 2)()
     wide[0] = tb.Linear(FAKE, FAKE, X1, FAKE, 256, 1 << 17, 1, 0)
     wide[1] = tb.Linear(FAKE, FAKE, X2, FAKE, 256, 1 << 17, 2, 0)
-    control, data = al(2048 * 256), 2 * al(1088 * 1024)
+    control, data = al(2048 * 512), 2 * al(1088 * 1024)
     assert data > control and tb.layer_workspace_bytes(wide) == 2 * data
 
 
@@ -222,7 +222,7 @@ def test_gate_up_workspace_and_errors(lib):
         G, T = K // 128, (N + 255) // 256
         chunks = sum(T * -(-G // (2 if gr == 2 else 4)) for gr in (gg, gu))
         shared = (gg == 2) == (gu == 2)  # same x: one record set when the code widths agree
-        control = al(2048 * min(256, chunks)) + al(8 * N)
+        control = al(2048 * min(512, chunks)) + al(8 * N)
         data = al(1088 * G) * (1 if shared else 2)
         assert lib.tb_gate_up_workspace_bytes(g, u) == 2 * max(control, data)
     two = (tb.Linear * 2)()

@@ -479,6 +479,29 @@ def test_gemv_ranges_over_several_tiles(oracle, grid):
     assert_within(y[torch.from_numpy(rows).to(DEV)], y64, yabs, "f32", oracle, f"tall grid {grid}")
 
 
+@pytest.mark.parametrize("grid", [tb.INT2, tb.INT3])
+@pytest.mark.parametrize("tiles_less", [1, 0])
+def test_gemv_both_cta_layouts(oracle, grid, tiles_less):
+    """A call of 8 chunks per SM or more runs two CTAs per SM, a smaller one
+    one CTA: a 2-bit matrix of K = 8192 (16 chunks per 256-row tile) with
+    SMs / 2 tiles sits exactly at the switch, one tile fewer just below it
+    (3 bits: twice the chunks, both above).  Sampled rows (tile edges, ends,
+    random) against the oracle."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    K = 8192
+    N = 256 * (sms // 2 - tiles_less) - 17  # ragged last tile
+    W = synth.gaussian_weights(N, K, seed=3700 + grid + tiles_less)
+    s_ref = oracle.scales_absmax(w_np(W), grid)
+    p_ref, _ = oracle.pack(w_np(W), grid, s_ref)
+    x = synth.activations(K, seed=3800 + grid)
+    rng = np.random.default_rng(7 + grid)
+    rows = np.unique(np.concatenate([[0, 1, N - 1], np.arange(255, N, 256 * 8), rng.integers(0, N, 40)]))
+    y64, yabs = oracle.gemv_rows64(p_ref, grid, s_ref, u16(x), K, rows)
+    y = tb.tb_gemv(to_dev_packed(p_ref), grid, to_dev_bits(s_ref), x.to(DEV), N, K)
+    assert tb.sync_status() == 0
+    assert_within(y[torch.from_numpy(rows).to(DEV)], y64, yabs, "f32", oracle, f"{N}x{K} grid {grid}")
+
+
 def test_zz_no_bounded_wait_gave_up():
     """After every test above: no device-side bounded wait (TMA copies,
     tensor-core hand-offs) timed out, so every result above is a real one."""
