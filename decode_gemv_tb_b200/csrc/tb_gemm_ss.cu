@@ -194,6 +194,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// the registers of a tcgen05.ld, tied to a point after tmem_ld_wait (the wait
+// names no register, so without this the compiler may use them before it)
+__device__ __forceinline__ void tmem_regs_after_wait(uint32_t (&r)[16]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]));
+}
 
 // ---- partial sums between CTAs: a release flag per CTA --------------------------------
 __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
@@ -510,6 +518,10 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
                     tmem_ld16(scol + cc, a[0]);
                     tmem_ld16(scol + cc + W, a[1]);
                     tmem_ld_wait();
+                    tmem_regs_after_wait(v[0]);
+                    tmem_regs_after_wait(v[1]);
+                    tmem_regs_after_wait(a[0]);
+                    tmem_regs_after_wait(a[1]);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -536,6 +548,7 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
                         uint32_t a[W];
                         tmem_ld16(scol + cc, a);
                         tmem_ld_wait();
+                        tmem_regs_after_wait(a);
 #pragma unroll
                         for (int i = 0; i < W; ++i) acc[i] = __uint_as_float(a[i]);
                     } else {
@@ -554,6 +567,7 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
                         for (int i = 0; i < W; i += 4)
                             *reinterpret_cast<float4*>(pd + cc + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
                     }
+                    __threadfence();  // each thread's own sums, before the barrier that precedes the release
                     named_sync(1, kSSEpiWarps * 32);
                     if (warp == kSSWarpEpi0 && lane == 0) {
                         __threadfence();

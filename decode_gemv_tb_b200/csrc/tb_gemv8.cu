@@ -624,6 +624,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks) k_gemv8(const 
             for (; pf_k < n && pf_k < kEarly; ++pf_k, advance(pf)) weights(pf, pf_k);
         }
         pdl_wait();  // the records: written by the record kernel, the previous one in the stream
+        // they were written through the generic proxy; the bulk copies read them through the async one
+        asm volatile("fence.proxy.async.global;" ::: "memory");
         if (active && lane == 0)
             for (; pf_k < n && pf_k < kStages; ++pf_k, advance(pf)) weights(pf, pf_k);
         int issued = 0;
