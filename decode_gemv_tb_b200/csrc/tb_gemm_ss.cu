@@ -20,7 +20,7 @@
 // finishing CTA acquires the flags (and clears them) and adds the sums in
 // CTA order (bitwise deterministic).
 //
-// Pipeline of a CTA (18 warps), per chunk:
+// Pipeline of a CTA (19 warps), per chunk:
 //   * producer warp: the block's activations of the group (128 rows x 128
 //     bf16, rows past M read as zero) as two tensor copies (no multicast)
 //     with 128-byte swizzle -- the MMA's K-major B layout -- into a ring of
@@ -29,8 +29,9 @@
 //     global memory (four groups ahead, in registers), decodes it to the
 //     signed codeword, exactly, as bf16 (tb_device.cuh) and stores it into
 //     one of four A stages in the same swizzled K-major layout;
-//   * MMA warp: eight 128 x 128 x 16 MMAs (kind::f16, bf16 in, fp32 out)
-//     into accumulator d = chunk mod 3 of tensor memory, committed to three
+//   * MMA warps (the even chunks, the odd chunks): eight 128 x 128 x 16 MMAs
+//     (kind::f16, bf16 in, fp32 out) into accumulator d = chunk mod 2 of
+//     tensor memory, committed to three
 //     mbarriers: the A stage and the activation stage are free, the
 //     accumulator is ready;
 //   * 8 epilogue warps (two per 32 TMEM lanes = 32 rows, each half of the
@@ -62,16 +63,21 @@ constexpr int kSSDecWarps = 8;      // a thread per half of a row's group
 constexpr int kSSEpiWarps = 8;      // two per 32 TMEM lanes, half the columns each
 constexpr int kSSWarpDec0 = 2;                            // warps 2 .. 9 decode
 constexpr int kSSWarpEpi0 = kSSWarpDec0 + kSSDecWarps;   // warps 10 .. 17 finish
-constexpr int kSSThreads = (kSSWarpEpi0 + kSSEpiWarps) * 32;
+// warps 1 and 18 issue the MMAs of the even and the odd chunks: an MMA
+// holds its issuing thread for about 150 cycles, so one warp cannot keep
+// pace with the decoders
+constexpr int kSSWarpMma1 = kSSWarpEpi0 + kSSEpiWarps;
+constexpr int kSSThreads = (kSSWarpMma1 + 1) * 32;
 constexpr int kSSABytes = kSSRows * kGroup * 2;  // decoded group, bf16
 constexpr uint64_t kSSMaxCtas = 256;             // bound of the grid (one CTA per SM)
 constexpr int kSSPrefetch = 4;                   // groups of packed codes in flight per decoder thread
 
 __host__ __device__ constexpr int ss_xbytes(int np) { return np * kGroup * 2; }
 // activation stages (as many as fit beside the four A stages)
-__host__ __device__ constexpr int ss_xstages(int np) { return np <= 32 ? 8 : (np <= 64 ? 4 : 3); }
+// (stage and accumulator counts are even: each is then waited on by one MMA warp, in order)
+__host__ __device__ constexpr int ss_xstages(int np) { return np <= 32 ? 8 : (np <= 64 ? 4 : 2); }
 // accumulators in tensor memory: its 512 columns less the running sums' NP
-__host__ __device__ constexpr int ss_dbufs(int np) { return 512 / np - 1; }
+__host__ __device__ constexpr int ss_dbufs(int np) { return (512 / np - 1) & ~1; }
 __host__ __device__ constexpr int ss_smem_bytes(int np) {
     return kSSStages * kSSABytes + ss_xstages(np) * ss_xbytes(np) + 1024;
 }
@@ -311,7 +317,7 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_sh;
-    int issued = 0, committed = 0;  // producer: chunks requested; MMA warp: chunks committed
+    int issued = 0, committed = 0;  // producer: chunks requested; MMA warp: its last chunk committed, plus one
 
     if (warp == 0) {
         // ---------------- producer: the activations of every chunk, XS ahead ----------------
@@ -333,9 +339,10 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
                 }
             }
         }
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        for (int k = 0; k < n; ++k) {
+    } else if (warp == 1 || warp == kSSWarpMma1) {
+        // ---------------- MMA issuers: chunk k by warp 1 (k even) or kSSWarpMma1 (k odd) ----------------
+        static_assert(kSSStages % 2 == 0 && XS % 2 == 0 && kSSDBufs % 2 == 0, "one waiting warp per stage");
+        for (int k = warp == 1 ? 0 : 1; k < n; k += 2) {
             const int s = k % kSSStages, x = k % XS, d = k % kSSDBufs;
             if (!__all_sync(0xffffffffu, bar_wait(saddr(&afull[s]), (uint32_t)(k / kSSStages) & 1u, A.wait_cycles,
                                                   abort)))
@@ -632,7 +639,7 @@ __global__ void __launch_bounds__(kSSThreads, 1) k_gemm_ss(const __grid_constant
         if (warp == 0 && lane == 0)  // the newest copy of each stage (older ones landed before it was refilled)
             for (int k = issued > XS ? issued - XS : 0; k < issued; ++k)
                 bar_drain(saddr(&xfull[k % XS]), (uint32_t)(k / XS) & 1u, A.wait_cycles);
-        if (warp == 1 && committed > 0)  // commits complete in order
+        if ((warp == 1 || warp == kSSWarpMma1) && committed > 0)  // each warp's commits complete in order
             bar_drain(saddr(&dfull[(committed - 1) % kSSDBufs]), (uint32_t)((committed - 1) / kSSDBufs) & 1u,
                       A.wait_cycles);
     }
